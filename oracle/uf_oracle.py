@@ -1,0 +1,275 @@
+"""fp64 CPU oracle for chunk-causal block-sparse attention over a rolling KV window.
+
+TEST INFRASTRUCTURE.  Only the tests, ``__graft_entry__.smoke()`` and the CPU
+baseline leg of ``bench.py`` may import this module.  The product path (the
+CUDA library and its Python binding) never calls it and shares no code with it.
+
+Every function computes the plain definition of its step, in float64, with no
+blocking, fusion or reordering beyond what that definition states.  Inputs are
+float64 numpy arrays (exact upcasts of the bf16 values the GPU receives).
+
+Sources (page title, then section / equation):
+
+* Ultra Flash (papernotes.org notes), Method, key design 3: the 3-D token grid
+  is cut into non-overlapping blocks; per attention layer the query and key
+  tokens of each block are mean-pooled, blocks are scored by the dot product of
+  the pooled query and key, and each head keeps its top-k scoring blocks, under
+  a strict temporal causal mask.
+* Ultra Flash (papernotes.org notes), Method, key design 4: dynamic cache
+  management -- reuse of the last denoising step's KV cache instead of a rerun,
+  and adaptive cropping of the SR model's KV window length.
+* FlashDecoder (xllm-io blog), Sec. 3, Eq. 4: the cached keys/values have shape
+  B x G x (W_frm * L_frm) x D_h, with G grouped-query KV heads.
+* FlashDecoder (xllm-io blog), Algorithm 1 (streaming inference): after each
+  frame the cache becomes the tail (W_frm - 1) frames of the old cache followed
+  by the new frame's K/V; causality comes from the processing order, not from a
+  token mask (Sec. 3.3, "causality through processing order").
+
+Readings taken where the pages are silent or ambiguous (each is listed in the
+design notes of the repository):
+
+* Blocks are contiguous runs of ``blk`` tokens in the caller's token order,
+  counted within each chunk; the last block of a chunk is partial when ``blk``
+  does not divide the chunk length.  Blocks never straddle chunks.
+* The query chunk is the newest chunk of the window (it was appended just
+  before attention).  Inside the window there is no token-level mask: each query
+  token may attend to every token of every kept block, including blocks of its
+  own chunk ("chunk-causal").
+* Pooled block score = mean(q_block) . mean(k_block) / sqrt(D); no softmax is
+  applied to pooled scores (it would not change the ranking).
+* Selection per (batch, query head, q-block i): the diagonal block
+  d_i = (n_valid - 1) * nb + i (same block of the newest chunk) is always kept;
+  the other blocks are ranked by (score descending, logical index ascending) and
+  the first k - 1 are kept.  k is clamped to the number of blocks in the window.
+* Under GQA, query head h reads KV head h // (H / G); masks are per query head.
+* LSE is the natural log of sum(exp(scale * q . k)) over kept tokens.
+"""
+from __future__ import annotations
+
+import math
+from typing import List, Optional, Sequence, Tuple
+
+import numpy as np
+
+__all__ = [
+    "RollingWindow",
+    "block_ranges",
+    "window_blocks",
+    "pool_blocks",
+    "block_scores",
+    "select_blocks",
+    "block_mask",
+    "block_sparse_attention",
+]
+
+
+# --------------------------------------------------------------------------
+# Rolling KV window
+# --------------------------------------------------------------------------
+class RollingWindow:
+    """The last ``keep_chunks`` chunks of K and V, oldest first.
+
+    FlashDecoder, Eq. 4 / Algorithm 1: a fixed window whose memory does not grow
+    with the stream (the oldest frame leaves when a new one arrives).  Ultra
+    Flash key design 4 adds two cache operations, read here as:
+
+    * ``replace_newest``: the newest chunk's K/V are overwritten by a new
+      computation of the same chunk (no eviction);
+    * ``keep_chunks``: the window is cropped to at most ``keep_chunks`` chunks
+      (oldest dropped first), ``1 <= keep_chunks <= W``.
+    """
+
+    def __init__(self, W: int):
+        if W < 1:
+            raise ValueError("window capacity must be >= 1")
+        self.W = W
+        self.k: List[np.ndarray] = []
+        self.v: List[np.ndarray] = []
+
+    def append(self, k_new: np.ndarray, v_new: np.ndarray,
+               keep_chunks: Optional[int] = None, replace_newest: bool = False) -> None:
+        keep = self.W if keep_chunks is None else keep_chunks
+        if not 1 <= keep <= self.W:
+            raise ValueError("keep_chunks must be in [1, W]")
+        if replace_newest:
+            if not self.k:
+                raise ValueError("replace_newest on an empty window")
+            self.k[-1] = np.array(k_new, dtype=np.float64)
+            self.v[-1] = np.array(v_new, dtype=np.float64)
+        else:
+            self.k.append(np.array(k_new, dtype=np.float64))
+            self.v.append(np.array(v_new, dtype=np.float64))
+        while len(self.k) > keep:
+            self.k.pop(0)
+            self.v.pop(0)
+
+    @property
+    def n_valid(self) -> int:
+        return len(self.k)
+
+
+# --------------------------------------------------------------------------
+# Blocks
+# --------------------------------------------------------------------------
+def block_ranges(Lc: int, blk: int) -> List[Tuple[int, int]]:
+    """[start, stop) token ranges of the blocks of one chunk (Ultra Flash key
+    design 3: non-overlapping blocks; last one partial)."""
+    if Lc < 1 or blk < 1:
+        raise ValueError("Lc and blk must be positive")
+    return [(s, min(s + blk, Lc)) for s in range(0, Lc, blk)]
+
+
+def window_blocks(n_chunks: int, Lc: int, blk: int) -> List[Tuple[int, int, int]]:
+    """Logical kv blocks of a window of ``n_chunks`` chunks, oldest first:
+    block j -> (chunk index c, start, stop) with j = c * nb + r."""
+    return [(c, s, e) for c in range(n_chunks) for (s, e) in block_ranges(Lc, blk)]
+
+
+# --------------------------------------------------------------------------
+# Block mask: pooling, scores, top-k
+# --------------------------------------------------------------------------
+def pool_blocks(x: np.ndarray, blk: int) -> np.ndarray:
+    """Mean of each block's own tokens.
+
+    x: [B, L, heads, D] -> [B, heads, nblocks, D] (Ultra Flash key design 3:
+    in-block mean pooling of queries and keys).
+    """
+    B, L, Hx, D = x.shape
+    ranges = block_ranges(L, blk)
+    out = np.empty((B, Hx, len(ranges), D), dtype=np.float64)
+    for n, (s, e) in enumerate(ranges):
+        out[:, :, n, :] = x[:, s:e, :, :].mean(axis=1)
+    return out
+
+
+def block_scores(qpool: np.ndarray, kpool: np.ndarray, scale: float) -> np.ndarray:
+    """Pooled block scores (Ultra Flash key design 3: dot product of pooled
+    query and key blocks), scaled by ``scale``.
+
+    qpool [B, H, NQ, D], kpool [B, G, NKV, D] -> [B, H, NQ, NKV]; query head h
+    reads KV head h // (H // G) (grouped-query attention, FlashDecoder Eq. 4).
+    """
+    B, H, NQ, D = qpool.shape
+    G = kpool.shape[1]
+    if H % G:
+        raise ValueError("H must be a multiple of G")
+    rep = H // G
+    out = np.empty((B, H, NQ, kpool.shape[2]), dtype=np.float64)
+    for b in range(B):
+        for h in range(H):
+            out[b, h] = (qpool[b, h] @ kpool[b, h // rep].T) * scale
+    return out
+
+
+def select_blocks(scores: np.ndarray, k: int, diag: Sequence[int]):
+    """Per-row top-k block selection with a forced diagonal block.
+
+    scores [B, H, NQ, NKV]; diag[i] = logical index of q-block i's own block.
+    Returns (idx [B, H, NQ, k_eff] ascending int32, cnt [B, H, NQ] int32,
+    boundary [B, H, NQ, 2] float64).  ``boundary`` holds the score of the last
+    kept non-diagonal block and of the first dropped one (NaN when there is
+    none); rows where the two are closer than the near-tie tolerance may
+    legitimately differ between two correct implementations.
+    """
+    B, H, NQ, NKV = scores.shape
+    k_eff = min(k, NKV)
+    if k_eff < 1:
+        raise ValueError("k must be >= 1")
+    idx = np.empty((B, H, NQ, k_eff), dtype=np.int32)
+    cnt = np.full((B, H, NQ), k_eff, dtype=np.int32)
+    boundary = np.full((B, H, NQ, 2), np.nan)
+    all_j = np.arange(NKV)
+    for b in range(B):
+        for h in range(H):
+            for i in range(NQ):
+                d = diag[i]
+                cand = all_j[all_j != d]
+                s = scores[b, h, i, cand]
+                # rank: score descending, then logical index ascending
+                order = cand[np.lexsort((cand, -s))]
+                chosen = order[: k_eff - 1]
+                idx[b, h, i] = np.sort(np.append(chosen, d))
+                if k_eff - 1 >= 1:
+                    boundary[b, h, i, 0] = scores[b, h, i, order[k_eff - 2]]
+                if k_eff - 1 < len(order):
+                    boundary[b, h, i, 1] = scores[b, h, i, order[k_eff - 1]]
+    return idx, cnt, boundary
+
+
+def block_mask(q: np.ndarray, window: RollingWindow, blk: int, k: int,
+               scale: Optional[float] = None):
+    """The whole mask step for the newest chunk's queries.
+
+    q [B, Lc, H, D]; the window holds n_valid chunks of K [B, Lc, G, D].
+    Returns dict(idx, cnt, scores, boundary, qpool, kpool).
+    """
+    B, Lc, H, D = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    n_valid = window.n_valid
+    if n_valid < 1:
+        raise ValueError("empty window")
+    nb = len(block_ranges(Lc, blk))
+    qpool = pool_blocks(q, blk)                                     # [B,H,NQ,D]
+    kpool = np.concatenate([pool_blocks(kc, blk) for kc in window.k], axis=2)  # [B,G,NKV,D]
+    scores = block_scores(qpool, kpool, scale)
+    diag = [(n_valid - 1) * nb + i for i in range(nb)]
+    idx, cnt, boundary = select_blocks(scores, k, diag)
+    return dict(idx=idx, cnt=cnt, scores=scores, boundary=boundary, qpool=qpool, kpool=kpool)
+
+
+# --------------------------------------------------------------------------
+# Block-sparse attention
+# --------------------------------------------------------------------------
+def block_sparse_attention(q: np.ndarray, window: RollingWindow, blk: int,
+                           idx: Optional[np.ndarray] = None, cnt: Optional[np.ndarray] = None,
+                           scale: Optional[float] = None,
+                           items: Optional[Sequence[Tuple[int, int, int]]] = None):
+    """Softmax attention of the newest chunk's queries over the kept blocks.
+
+    For each (batch b, query head h, q-block i), the queries of block i attend
+    to every token of the kept kv blocks idx[b, h, i, :cnt] (all window blocks
+    when ``idx`` is None: density 1.0 = dense chunk-causal attention):
+
+        s = scale * q . k,  O = sum(exp(s - m) v) / sum(exp(s - m)),
+        LSE = m + ln(sum(exp(s - m)))
+
+    (Ultra Flash key design 3: attention restricted to the kept blocks;
+    FlashDecoder Sec. 3.3: no token mask inside the window.)
+
+    q [B, Lc, H, D]; returns (O [B, Lc, H, D], LSE [B, H, Lc]).  When ``items``
+    lists (b, h, i) work items, only those rows are computed (others NaN).
+    """
+    B, Lc, H, D = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    kwin = np.concatenate(window.k, axis=1)     # [B, n*Lc, G, D] logical token order
+    vwin = np.concatenate(window.v, axis=1)
+    G = kwin.shape[2]
+    rep = H // G
+    qranges = block_ranges(Lc, blk)
+    kvblocks = window_blocks(window.n_valid, Lc, blk)
+    nkv = len(kvblocks)
+    O = np.full((B, Lc, H, D), np.nan)
+    LSE = np.full((B, H, Lc), np.nan)
+    if items is None:
+        items = [(b, h, i) for b in range(B) for h in range(H) for i in range(len(qranges))]
+    for (b, h, i) in items:
+        if idx is None:
+            kept = range(nkv)
+        else:
+            n = idx.shape[-1] if cnt is None else int(cnt[b, h, i])
+            kept = [int(j) for j in idx[b, h, i, :n]]
+        cols = np.concatenate([np.arange(c * Lc + s, c * Lc + e) for (c, s, e) in
+                               (kvblocks[j] for j in kept)])
+        s0, e0 = qranges[i]
+        qi = q[b, s0:e0, h, :]
+        kk = kwin[b, cols, h // rep, :]
+        vv = vwin[b, cols, h // rep, :]
+        s = (qi @ kk.T) * scale
+        m = s.max(axis=1, keepdims=True)
+        p = np.exp(s - m)
+        l = p.sum(axis=1)
+        O[b, s0:e0, h, :] = (p @ vv) / l[:, None]
+        LSE[b, h, s0:e0] = m[:, 0] + np.log(l)
+    return O, LSE
