@@ -1,0 +1,142 @@
+// kv_append.cuh -- rolling-window append / evict of one chunk's K and V.
+//
+// FlashDecoder (xllm-io blog), Algorithm 1: after each frame the cache is the
+// tail (W - 1) frames of the old cache followed by the new frame's K/V; Eq. 4
+// fixes the cache layout B x G x (W L) x D_h.  Ultra Flash (papernotes notes),
+// key design 4: reuse of the last denoising step's KV (here: overwrite the
+// newest chunk) and adaptive cropping of the SR KV window (here: keep_chunks).
+//
+// One thread block per (block r of the chunk, KV head g, batch b).  256
+// threads = 16 token lanes x 16 sixteen-byte column chunks of a 256-byte token
+// row, so every warp moves two whole rows per instruction on both sides.  The
+// block also reduces its tokens' K into the slot's pooled-K row (fp32 mean over
+// the block's true tokens), which the block-mask call reads instead of
+// re-reading the window.  The last thread block to finish commits the new
+// window state to meta; every block read the old state before counting in, so
+// no block can observe a half-updated window.
+#pragma once
+
+#include "uf_device.cuh"
+
+namespace uf {
+
+struct AppendParams {
+  const __nv_bfloat16 *k_new;  // [B, Lc, G, D]
+  const __nv_bfloat16 *v_new;
+  __nv_bfloat16 *k;            // [B, G, W*Lslot, D]
+  __nv_bfloat16 *v;
+  float *kpool;                // [B, G, W*nb, D]
+  int32_t *meta;               // {start, n_valid, counter, reserved}
+  int32_t G, W, Lc, nb, lslot, keep, replace;
+};
+
+// New window state and the slot the chunk goes to (see uf_kv_append).
+__device__ __forceinline__ void append_plan(int32_t start, int32_t n, int32_t W, int32_t keep, int32_t replace,
+                                            int32_t &slot, int32_t &start2, int32_t &n2) {
+  if (replace && n > 0) {
+    slot = (start + n - 1) % W;
+    start2 = start;
+    n2 = n;
+  } else {
+    slot = (start + n) % W;   // free: at most keep-1 <= W-1 chunks survive eviction
+    const int32_t evict = max(0, n + 1 - keep);
+    start2 = (start + evict) % W;
+    n2 = n - evict + 1;
+  }
+  if (n2 > keep) {            // crop (replace with a smaller keep_chunks)
+    start2 = (start2 + (n2 - keep)) % W;
+    n2 = keep;
+  }
+}
+
+template <int BLK>
+__global__ void __launch_bounds__(256) kv_append_kernel(const AppendParams p) {
+  constexpr int D = 128;
+  constexpr int PASSES = BLK / 16;
+  const int r = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int tid = threadIdx.x, tl = tid >> 4, dc = tid & 15;
+
+  __shared__ int32_t s_plan[3];
+  __shared__ __align__(16) float s_red[16][D];
+
+  if (tid == 0) {
+    int32_t start = __ldcg(p.meta + 0), n = __ldcg(p.meta + 1);
+    if (start < 0 || start >= p.W || n < 0 || n > p.W) {
+      record_error(UF_EBOUNDS);
+      start = 0;
+      n = 0;
+    }
+    int32_t slot, start2, n2;
+    append_plan(start, n, p.W, p.keep, p.replace, slot, start2, n2);
+    s_plan[0] = slot;
+    s_plan[1] = start2;
+    s_plan[2] = n2;
+  }
+  __syncthreads();
+  const int slot = s_plan[0];
+
+  const int t0 = r * BLK;
+  const int cnt = min(BLK, p.Lc - t0);
+  const size_t src_stride = static_cast<size_t>(p.G) * D;                       // elements per token
+  const __nv_bfloat16 *ksrc = p.k_new + (static_cast<size_t>(b) * p.Lc + t0) * src_stride + g * D + dc * 8;
+  const __nv_bfloat16 *vsrc = p.v_new + (static_cast<size_t>(b) * p.Lc + t0) * src_stride + g * D + dc * 8;
+  const size_t dst_row0 = (static_cast<size_t>(b) * p.G + g) * p.W * p.lslot + static_cast<size_t>(slot) * p.lslot + t0;
+  __nv_bfloat16 *kdst = p.k + dst_row0 * D + dc * 8;
+  __nv_bfloat16 *vdst = p.v + dst_row0 * D + dc * 8;
+
+  uint4 kr[PASSES], vr[PASSES];
+#pragma unroll
+  for (int m = 0; m < PASSES; ++m) {
+    const int t = tl + 16 * m;
+    if (t < cnt) {
+      kr[m] = __ldg(reinterpret_cast<const uint4 *>(ksrc + t * src_stride));
+      vr[m] = __ldg(reinterpret_cast<const uint4 *>(vsrc + t * src_stride));
+    } else {
+      kr[m] = make_uint4(0, 0, 0, 0);   // padding rows of the chunk's last block
+      vr[m] = make_uint4(0, 0, 0, 0);
+    }
+  }
+  float acc[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+#pragma unroll
+  for (int m = 0; m < PASSES; ++m) {
+    const int t = tl + 16 * m;
+    *reinterpret_cast<uint4 *>(kdst + static_cast<size_t>(t) * D) = kr[m];
+    *reinterpret_cast<uint4 *>(vdst + static_cast<size_t>(t) * D) = vr[m];
+    const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&kr[m]);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 f = __bfloat1622float2(h2[e]);
+      acc[2 * e] += f.x;
+      acc[2 * e + 1] += f.y;
+    }
+  }
+  // block mean of K over the block's true tokens (padding rows hold zeros)
+  *reinterpret_cast<float4 *>(&s_red[tl][dc * 8]) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+  *reinterpret_cast<float4 *>(&s_red[tl][dc * 8 + 4]) = make_float4(acc[4], acc[5], acc[6], acc[7]);
+  __syncthreads();
+  if (tid < D) {
+    float s = 0.f;
+#pragma unroll
+    for (int q = 0; q < 16; ++q) s += s_red[q][tid];
+    const size_t prow = (static_cast<size_t>(b) * p.G + g) * p.W * p.nb + static_cast<size_t>(slot) * p.nb + r;
+    p.kpool[prow * D + tid] = s / static_cast<float>(cnt);
+  }
+
+  // commit the new window state once every block has read the old one
+  __syncthreads();
+  if (tid == 0) {
+    __threadfence();
+    const int32_t total = static_cast<int32_t>(gridDim.x * gridDim.y * gridDim.z);
+    const int32_t prev = atomicAdd(p.meta + 2, 1);
+    if (prev == total - 1) {
+      atomicExch(p.meta + 0, s_plan[1]);
+      atomicExch(p.meta + 1, s_plan[2]);
+      atomicExch(p.meta + 2, 0);
+      __threadfence();
+    }
+  }
+}
+
+}  // namespace uf

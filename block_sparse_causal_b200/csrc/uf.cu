@@ -1,0 +1,359 @@
+// uf.cu -- C ABI of libuf.so: argument checks, TMA tensor maps, launches.
+//
+// Single translation unit: the kernels live in the included headers so that the
+// device error word is one symbol per device.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <atomic>
+#include <mutex>
+
+#include "uf.h"
+#include "uf_device.cuh"
+#include "kv_append.cuh"
+#include "block_mask.cuh"
+#include "attention.cuh"
+
+namespace {
+
+constexpr int32_t UF_VERSION = 100;   // 0.1.0
+constexpr int32_t kMaxW = 64;
+constexpr int32_t kMaxMaskNKV = 5000; // pooled-score row kept in shared memory
+constexpr int32_t kMaxDevices = 64;
+std::atomic<long long> g_wait_limit{1LL << 31};
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int32_t ceil_div(int32_t a, int32_t b) { return (a + b - 1) / b; }
+
+bool dims_ok(int32_t B, int32_t G, int32_t D, int32_t W, int32_t Lc, int32_t blk) {
+  if (B < 1 || G < 1 || W < 1 || W > kMaxW || Lc < 1) return false;
+  if (D != 128) return false;
+  if (blk != 64 && blk != 128) return false;
+  // every element offset of the window buffers must fit the 32-bit row math
+  const long long lslot = static_cast<long long>(ceil_div(Lc, blk)) * blk;
+  if (static_cast<long long>(W) * lslot >= (1LL << 30)) return false;
+  const long long bytes = static_cast<long long>(B) * G * W * lslot * D * 2;
+  return bytes <= (1LL << 40);
+}
+
+bool cache_ok(const uf_kv_cache *c) {
+  if (!c) return false;
+  if (!dims_ok(c->B, c->G, c->D, c->W, c->Lc, c->blk)) return false;
+  if (!c->k || !c->v || !c->kpool || !c->meta) return false;
+  if (!aligned16(c->k) || !aligned16(c->v) || !aligned16(c->kpool) || !aligned16(c->meta)) return false;
+  return true;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *,
+                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    cudaDriverEntryPointQueryResult q;
+    void *p = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// bf16 tensor map, 128-byte swizzle, box {64, box[1..]} (64 bf16 = 128 bytes inner).
+bool make_map(CUtensorMap *m, const void *base, int rank, const cuuint64_t *dims, const cuuint64_t *strides,
+              const cuuint32_t *box) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint32_t es[5] = {1, 1, 1, 1, 1};
+  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void *>(base), dims, strides, box, es,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+thread_local const char *t_last_cuda_error = "no error";
+
+int32_t cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return UF_OK;
+  t_last_cuda_error = cudaGetErrorString(e);
+  return UF_ECUDA;
+}
+
+// Raise a kernel's dynamic shared-memory limit to at least `bytes` (per device,
+// only when a launch needs more than any earlier one).
+template <typename K>
+int32_t ensure_smem(K kernel, int bytes, std::atomic<int> (&done)[kMaxDevices]) {
+  int dev = 0;
+  const int32_t st = cuda_status(cudaGetDevice(&dev));
+  if (st != UF_OK) return st;
+  if (dev < 0 || dev >= kMaxDevices) return UF_EUNSUPPORTED;
+  if (done[dev].load() >= bytes) return UF_OK;
+  const int32_t st2 = cuda_status(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
+  if (st2 != UF_OK) return st2;
+  done[dev].store(bytes);
+  return UF_OK;
+}
+
+int32_t launch_status() { return cuda_status(cudaGetLastError()); }
+
+std::atomic<int> g_attn128_smem[kMaxDevices], g_attn64_smem[kMaxDevices], g_mask128_smem[kMaxDevices],
+    g_mask64_smem[kMaxDevices];
+
+}  // namespace
+
+extern "C" {
+
+int32_t uf_version(void) { return UF_VERSION; }
+
+const char *uf_strerror(int32_t status) {
+  switch (status) {
+    case UF_OK: return "UF_OK";
+    case UF_EINVAL: return "UF_EINVAL: invalid argument";
+    case UF_ECUDA: return "UF_ECUDA: CUDA call or kernel launch failed";
+    case UF_ETIMEOUT: return "UF_ETIMEOUT: a kernel pipeline wait exceeded its bound";
+    case UF_EBOUNDS: return "UF_EBOUNDS: a kernel found an out-of-range index or window state";
+    case UF_EUNSUPPORTED: return "UF_EUNSUPPORTED: request not supported by this build";
+    default: return "UF_UNKNOWN";
+  }
+}
+
+int32_t uf_kv_cache_bytes(int32_t B, int32_t G, int32_t D, int32_t W, int32_t Lc, int32_t blk, size_t *kv_bytes,
+                          size_t *kpool_bytes, size_t *meta_bytes) {
+  if (!dims_ok(B, G, D, W, Lc, blk)) return UF_EINVAL;
+  const size_t nb = static_cast<size_t>(ceil_div(Lc, blk));
+  const size_t lslot = nb * blk;
+  if (kv_bytes) *kv_bytes = static_cast<size_t>(B) * G * W * lslot * D * 2;
+  if (kpool_bytes) *kpool_bytes = static_cast<size_t>(B) * G * W * nb * D * 4;
+  if (meta_bytes) *meta_bytes = 4 * sizeof(int32_t);
+  return UF_OK;
+}
+
+int32_t uf_kv_cache_init(uf_kv_cache *c, void *k, void *v, float *kpool, int32_t *meta, int32_t B, int32_t G,
+                         int32_t D, int32_t W, int32_t Lc, int32_t blk) {
+  if (!c) return UF_EINVAL;
+  uf_kv_cache t;
+  t.k = k;
+  t.v = v;
+  t.kpool = kpool;
+  t.meta = meta;
+  t.B = B;
+  t.G = G;
+  t.D = D;
+  t.W = W;
+  t.Lc = Lc;
+  t.blk = blk;
+  t.host_start = 0;
+  t.host_n_valid = 0;
+  if (!cache_ok(&t)) return UF_EINVAL;
+  *c = t;
+  return UF_OK;
+}
+
+int32_t uf_kv_reset(uf_kv_cache *c, uf_stream_t s) {
+  if (!cache_ok(c)) return UF_EINVAL;
+  const int32_t st = cuda_status(cudaMemsetAsync(c->meta, 0, 4 * sizeof(int32_t), reinterpret_cast<cudaStream_t>(s)));
+  if (st != UF_OK) return st;
+  c->host_start = 0;
+  c->host_n_valid = 0;
+  return UF_OK;
+}
+
+int32_t uf_kv_append(uf_kv_cache *c, const void *k_new, const void *v_new, int32_t keep_chunks, int32_t flags,
+                     uf_stream_t s) {
+  if (!cache_ok(c)) return UF_EINVAL;
+  if (!k_new || !v_new || !aligned16(k_new) || !aligned16(v_new)) return UF_EINVAL;
+  if (keep_chunks < 1 || keep_chunks > c->W) return UF_EINVAL;
+  if (flags & ~UF_APPEND_REPLACE_NEWEST) return UF_EINVAL;
+  const int32_t replace = (flags & UF_APPEND_REPLACE_NEWEST) ? 1 : 0;
+  if (replace && c->host_n_valid == 0) return UF_EINVAL;
+
+  uf::AppendParams p;
+  p.k_new = static_cast<const __nv_bfloat16 *>(k_new);
+  p.v_new = static_cast<const __nv_bfloat16 *>(v_new);
+  p.k = static_cast<__nv_bfloat16 *>(c->k);
+  p.v = static_cast<__nv_bfloat16 *>(c->v);
+  p.kpool = c->kpool;
+  p.meta = c->meta;
+  p.G = c->G;
+  p.W = c->W;
+  p.Lc = c->Lc;
+  p.nb = ceil_div(c->Lc, c->blk);
+  p.lslot = p.nb * c->blk;
+  p.keep = keep_chunks;
+  p.replace = replace;
+  const dim3 grid(p.nb, c->G, c->B);
+  cudaGetLastError();
+  if (c->blk == 128)
+    uf::kv_append_kernel<128><<<grid, 256, 0, reinterpret_cast<cudaStream_t>(s)>>>(p);
+  else
+    uf::kv_append_kernel<64><<<grid, 256, 0, reinterpret_cast<cudaStream_t>(s)>>>(p);
+  const int32_t st = launch_status();
+  if (st != UF_OK) return st;
+  // host mirror (same rule as the kernel)
+  int32_t start2, n2;
+  const int32_t start = c->host_start, n = c->host_n_valid, W = c->W, keep = keep_chunks;
+  if (replace && n > 0) {
+    start2 = start;
+    n2 = n;
+  } else {
+    const int32_t evict = n + 1 - keep > 0 ? n + 1 - keep : 0;
+    start2 = (start + evict) % W;
+    n2 = n - evict + 1;
+  }
+  if (n2 > keep) {
+    start2 = (start2 + (n2 - keep)) % W;
+    n2 = keep;
+  }
+  c->host_start = start2;
+  c->host_n_valid = n2;
+  return UF_OK;
+}
+
+int32_t uf_block_mask(const void *q, int32_t H, const uf_kv_cache *c, int32_t k, int32_t *idx, int32_t *cnt,
+                      float *scores, uf_stream_t s) {
+  if (!cache_ok(c)) return UF_EINVAL;
+  if (!q || !idx || !cnt || !aligned16(q)) return UF_EINVAL;
+  if (!aligned16(idx) || !aligned16(cnt) || (scores && !aligned16(scores))) return UF_EINVAL;
+  if (H < 1 || H % c->G != 0) return UF_EINVAL;
+  const int32_t nb = ceil_div(c->Lc, c->blk);
+  const int32_t nkv_max = c->W * nb;
+  if (k < 1 || k > nkv_max) return UF_EINVAL;
+  if (c->host_n_valid < 1) return UF_EINVAL;
+  if (nkv_max > kMaxMaskNKV) return UF_EUNSUPPORTED;
+
+  uf::MaskParams p;
+  p.q = static_cast<const __nv_bfloat16 *>(q);
+  p.kpool = c->kpool;
+  p.meta = c->meta;
+  p.idx = idx;
+  p.cnt = cnt;
+  p.scores = scores;
+  p.H = H;
+  p.G = c->G;
+  p.W = c->W;
+  p.Lc = c->Lc;
+  p.nb = nb;
+  p.k = k;
+  p.scale = 1.0f / sqrtf(static_cast<float>(c->D));
+  const int smem = (uf::MASK_TQ * 128 + 16 * 128 + uf::MASK_KT * uf::MASK_KSTRIDE + uf::MASK_TQ * nkv_max) * 4;
+  const dim3 grid(ceil_div(nb, uf::MASK_TQ), H, c->B);
+  cudaGetLastError();
+  if (c->blk == 128) {
+    const int32_t e = ensure_smem(uf::block_mask_kernel<128>, smem, g_mask128_smem);
+    if (e != UF_OK) return e;
+    uf::block_mask_kernel<128><<<grid, 256, smem, reinterpret_cast<cudaStream_t>(s)>>>(p);
+  } else {
+    const int32_t e = ensure_smem(uf::block_mask_kernel<64>, smem, g_mask64_smem);
+    if (e != UF_OK) return e;
+    uf::block_mask_kernel<64><<<grid, 256, smem, reinterpret_cast<cudaStream_t>(s)>>>(p);
+  }
+  return launch_status();
+}
+
+int32_t uf_block_sparse_attn(const void *q, int32_t H, const uf_kv_cache *c, const int32_t *idx, const int32_t *cnt,
+                             int32_t k, float scale, void *o, float *lse, uf_stream_t s) {
+  if (!cache_ok(c)) return UF_EINVAL;
+  if (!q || !o || !aligned16(q) || !aligned16(o)) return UF_EINVAL;
+  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return UF_EINVAL;
+  if (H < 1 || H % c->G != 0) return UF_EINVAL;
+  if (!(scale > 0.f) || !isfinite(scale)) return UF_EINVAL;
+  const int32_t nb = ceil_div(c->Lc, c->blk);
+  if (idx) {
+    if (k < 1 || k > c->W * nb) return UF_EINVAL;
+    if (reinterpret_cast<uintptr_t>(idx) & 3u) return UF_EINVAL;
+    if (cnt && (reinterpret_cast<uintptr_t>(cnt) & 3u)) return UF_EINVAL;
+  } else {
+    k = 0;
+    cnt = nullptr;
+  }
+  if (c->host_n_valid < 1) return UF_EINVAL;
+  const long long items = static_cast<long long>(c->B) * H * nb;
+  if (items >= (1LL << 31)) return UF_EINVAL;
+
+  const int32_t lslot = nb * c->blk;
+  CUtensorMap tq, tk, tv;
+  {
+    const cuuint64_t dims[4] = {128, static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(c->Lc),
+                                static_cast<cuuint64_t>(c->B)};
+    // byte strides of dims 1..3 (head, token, batch)
+    const cuuint64_t strides[3] = {256, static_cast<cuuint64_t>(H) * 256, static_cast<cuuint64_t>(c->Lc) * H * 256};
+    const cuuint32_t box[4] = {64, 1, 128, 1};
+    if (!make_map(&tq, q, 4, dims, strides, box)) return UF_ECUDA;
+  }
+  {
+    const cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(c->W) * lslot, static_cast<cuuint64_t>(c->B) * c->G};
+    const cuuint64_t strides[2] = {256, static_cast<cuuint64_t>(c->W) * lslot * 256};
+    const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(c->blk), 1};
+    if (!make_map(&tk, c->k, 3, dims, strides, box)) return UF_ECUDA;
+    if (!make_map(&tv, c->v, 3, dims, strides, box)) return UF_ECUDA;
+  }
+  uf::AttnParams p;
+  p.meta = c->meta;
+  p.idx = idx;
+  p.cnt = cnt;
+  p.o = static_cast<__nv_bfloat16 *>(o);
+  p.lse = lse;
+  p.H = H;
+  p.G = c->G;
+  p.W = c->W;
+  p.Lc = c->Lc;
+  p.nb = nb;
+  p.lslot = lslot;
+  p.k = k;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.wait_limit = g_wait_limit.load();
+  cudaGetLastError();
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(s);
+  if (c->blk == 128) {
+    constexpr int smem = uf::AttnSmem<128>::DYN;
+    const int32_t e = ensure_smem(uf::attn_kernel<128>, smem, g_attn128_smem);
+    if (e != UF_OK) return e;
+    uf::attn_kernel<128><<<static_cast<unsigned>(items), uf::ATTN_THREADS, smem, st>>>(tq, tk, tv, p);
+  } else {
+    constexpr int smem = uf::AttnSmem<64>::DYN;
+    const int32_t e = ensure_smem(uf::attn_kernel<64>, smem, g_attn64_smem);
+    if (e != UF_OK) return e;
+    uf::attn_kernel<64><<<static_cast<unsigned>(items), uf::ATTN_THREADS, smem, st>>>(tq, tk, tv, p);
+  }
+  return launch_status();
+}
+
+int32_t uf_get_error(int32_t *status, int32_t clear) {
+  if (!status) return UF_EINVAL;
+  int32_t st = cuda_status(cudaDeviceSynchronize());
+  if (st != UF_OK) return st;
+  int32_t v = 0;
+  st = cuda_status(cudaMemcpyFromSymbol(&v, uf::g_error_word, sizeof(v)));
+  if (st != UF_OK) return st;
+  if (clear) {
+    const int32_t z = 0;
+    st = cuda_status(cudaMemcpyToSymbol(uf::g_error_word, &z, sizeof(z)));
+    if (st != UF_OK) return st;
+  }
+  *status = v;
+  return UF_OK;
+}
+
+const char *uf_last_cuda_error(void) { return t_last_cuda_error; }
+
+int32_t uf_set_wait_limit(int64_t cycles) {
+  if (cycles < 1000) return UF_EINVAL;
+  g_wait_limit.store(cycles);
+  return UF_OK;
+}
+
+int32_t uf_debug_wait_timeout(int64_t cycles, uf_stream_t s) {
+  if (cycles < 1000 || cycles > (1LL << 40)) return UF_EINVAL;
+  cudaGetLastError();
+  uf::wait_timeout_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(s)>>>(cycles);
+  return launch_status();
+}
+
+}  // extern "C"

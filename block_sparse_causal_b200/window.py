@@ -1,0 +1,37 @@
+"""Owner of one rolling KV window's device buffers (torch allocations)."""
+from __future__ import annotations
+
+import math
+
+import torch
+
+from . import _uf
+
+
+class KVWindow:
+    """Allocates k, v, kpool and meta for a window of W chunks on ``device``
+    (sizes from ``uf_kv_cache_bytes``) and holds the ``uf_kv_cache``
+    descriptor that the library calls take."""
+
+    def __init__(self, B: int, G: int, W: int, Lc: int, blk: int = 128, D: int = 128, device="cuda"):
+        kv_bytes, kpool_bytes, meta_bytes = _uf.uf_kv_cache_bytes(B, G, D, W, Lc, blk)
+        self.B, self.G, self.D, self.W, self.Lc, self.blk = B, G, D, W, Lc, blk
+        self.nb = math.ceil(Lc / blk)
+        self.lslot = self.nb * blk
+        self.k = torch.zeros(kv_bytes // 2, dtype=torch.bfloat16, device=device).view(B, G, W * self.lslot, D)
+        self.v = torch.zeros_like(self.k)
+        self.kpool = torch.zeros(kpool_bytes // 4, dtype=torch.float32, device=device).view(B, G, W * self.nb, D)
+        self.meta = torch.zeros(meta_bytes // 4, dtype=torch.int32, device=device)
+        self.desc = _uf.uf_kv_cache_init(self.k, self.v, self.kpool, self.meta, B, G, D, W, Lc, blk)
+
+    @property
+    def n_valid(self) -> int:
+        """Host mirror of the number of chunks in the window."""
+        return self.desc.host_n_valid
+
+    def reset(self, stream=None) -> None:
+        _uf.uf_kv_reset(self.desc, stream)
+
+    def append(self, k_new, v_new, keep_chunks: int | None = None, replace_newest: bool = False, stream=None):
+        _uf.uf_kv_append(self.desc, k_new, v_new, self.W if keep_chunks is None else keep_chunks,
+                         _uf.UF_APPEND_REPLACE_NEWEST if replace_newest else 0, stream)

@@ -1,0 +1,231 @@
+/*
+ * uf.h -- C ABI of the chunk-causal block-sparse attention library (libuf.so)
+ *
+ * Three calls make up one attention layer of a streaming video DiT, per chunk:
+ *
+ *   uf_kv_append         rolling-window append / evict of the new chunk's K and V
+ *   uf_block_mask        per-head block mean-pooling of Q and K, pooled block
+ *                        scores, top-k block selection with the diagonal kept
+ *   uf_block_sparse_attn softmax attention of the chunk's queries over the kept
+ *                        blocks of the window (bf16 in, fp32 softmax, bf16 O and
+ *                        fp32 LSE), grouped-query aware
+ *
+ * Conventions shared by every call
+ *   - Every buffer is owned by the caller.  Pointers named "device" point to
+ *     device memory of the current CUDA device; they must be 16-byte aligned.
+ *   - No call allocates memory, synchronises the device or reads device data
+ *     back to the host.  Work is enqueued on the caller's stream `s` (a
+ *     cudaStream_t; NULL = legacy default stream) and runs asynchronously.
+ *   - Every call returns a status (uf_status).  Argument errors are detected on
+ *     the host before anything is enqueued (UF_EINVAL, nothing launched).  A
+ *     launch failure returns UF_ECUDA.  Errors found by a kernel while running
+ *     (an out-of-range block index, a pipeline wait that exceeded its bound)
+ *     are recorded in a device-side error word, read with uf_get_error().
+ *   - bf16 = IEEE bfloat16 (2 bytes), fp32 = IEEE binary32, int32 = int32_t.
+ *   - Shapes are listed outermost first; the last dimension is contiguous.
+ *
+ * Notation: B batch, H query heads, G KV heads (H % G == 0), D head dim (128),
+ * Lc tokens per chunk, W window capacity in chunks, blk tokens per block
+ * (64 or 128), nb = ceil(Lc / blk) blocks per chunk, Lslot = nb * blk tokens
+ * per ring slot (the chunk padded to a whole number of blocks),
+ * n_valid <= W chunks currently in the window, NKV = n_valid * nb.
+ */
+#ifndef UF_H
+#define UF_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; declared here so this header needs no CUDA header. */
+typedef struct CUstream_st *uf_stream_t;
+
+typedef enum uf_status {
+  UF_OK = 0,
+  UF_EINVAL = 1,      /* bad argument: shape, alignment, NULL pointer, range   */
+  UF_ECUDA = 2,       /* a CUDA runtime / driver call or launch failed         */
+  UF_ETIMEOUT = 3,    /* a kernel pipeline wait exceeded its bound (device)    */
+  UF_EBOUNDS = 4,     /* a kernel found an out-of-range index or state (device)*/
+  UF_EUNSUPPORTED = 5 /* valid request this build does not implement           */
+} uf_status;
+
+/* Flags of uf_kv_append. */
+#define UF_APPEND_REPLACE_NEWEST 1
+
+/*
+ * Rolling KV window ("cache") descriptor: plain data, caller-owned.
+ *
+ * Ring of W slots, each holding one chunk of Lslot tokens.  Logical chunk
+ * c (0 = oldest of the window) lives in physical slot (start + c) % W; logical
+ * kv block j of the window is block j % nb of logical chunk j / nb.  The
+ * physical order is never visible through the API.
+ *
+ *   k, v   device bf16 [B, G, W * Lslot, D].  Rows past Lc inside a slot (the
+ *          padding of the chunk's last block) are zeroed by uf_kv_append.
+ *   kpool  device fp32 [B, G, W * nb, D]: mean of K over the true tokens of
+ *          each block of each slot, written by uf_kv_append, read by
+ *          uf_block_mask (pooling K once per chunk instead of once per call).
+ *   meta   device int32[4] = {start, n_valid, append_counter, reserved}.  The
+ *          window state lives on the device so that a captured sequence of
+ *          calls stays correct when replayed.  Zeroed by uf_kv_reset.
+ *   host_start, host_n_valid: host mirror of meta[0..1], updated by
+ *          uf_kv_append / uf_kv_reset and used only for host-side argument
+ *          checks.
+ *
+ * Sources: FlashDecoder (xllm-io blog), Sec. 3, Eq. 4 (cache shape
+ * B x G x (W_frm L_frm) x D_h under grouped-query attention) and Algorithm 1
+ * (the cache keeps the tail W_frm - 1 frames and appends the new frame);
+ * HiStream (aipapers summary), innovation 2 (a fixed-size attention window
+ * keeps the KV cache from growing with video length).
+ */
+typedef struct uf_kv_cache {
+  void *k;
+  void *v;
+  float *kpool;
+  int32_t *meta;
+  int32_t B, G, D, W, Lc, blk;
+  int32_t host_start, host_n_valid;
+} uf_kv_cache;
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+int32_t uf_version(void);
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *uf_strerror(int32_t status);
+
+/*
+ * Byte sizes of the caller-owned buffers of a window with these dimensions:
+ * *kv_bytes for each of k and v, *kpool_bytes for kpool, *meta_bytes for meta.
+ * Any output pointer may be NULL.  Host only.  UF_EINVAL on bad dimensions
+ * (D != 128, blk not 64 or 128, W < 1 or W > 64, any size < 1, or a buffer
+ * larger than 2^40 bytes).
+ */
+int32_t uf_kv_cache_bytes(int32_t B, int32_t G, int32_t D, int32_t W, int32_t Lc, int32_t blk,
+                          size_t *kv_bytes, size_t *kpool_bytes, size_t *meta_bytes);
+
+/*
+ * Fill *c with the given buffers and dimensions and mark the host mirror
+ * empty.  Host only: does not touch device memory (call uf_kv_reset before the
+ * first append).  UF_EINVAL on NULL / misaligned pointers or bad dimensions.
+ */
+int32_t uf_kv_cache_init(uf_kv_cache *c, void *k, void *v, float *kpool, int32_t *meta,
+                         int32_t B, int32_t G, int32_t D, int32_t W, int32_t Lc, int32_t blk);
+
+/* Empty the window: zero meta on stream s and reset the host mirror. */
+int32_t uf_kv_reset(uf_kv_cache *c, uf_stream_t s);
+
+/*
+ * Append the new chunk's keys and values to the window (FlashDecoder,
+ * Algorithm 1: the cache becomes the tail of the previous window followed by
+ * the new frame's K/V; Ultra Flash notes, key design 4: reuse of the last
+ * denoising step's KV cache and adaptive cropping of the SR KV window).
+ *
+ *   k_new, v_new  device bf16 [B, Lc, G, D] (token-major, as a fused QKV
+ *                 projection writes them).  Read only.
+ *   keep_chunks   1..W: after the call the window holds at most keep_chunks
+ *                 chunks; the oldest are evicted first (pass W for a plain
+ *                 rolling window, less to crop it).
+ *   flags         0, or UF_APPEND_REPLACE_NEWEST: overwrite the newest chunk
+ *                 (a recomputation of the same chunk) instead of appending.
+ *                 Rejected (UF_EINVAL) when the host mirror says the window is
+ *                 empty; on the device an empty window turns it into an append.
+ *
+ * Writes the chunk into its ring slot of k / v (transposing BLGD -> BGLD),
+ * zeroes the slot's padding rows, writes the slot's block means into kpool and
+ * advances meta (the last thread block to finish commits the new state).
+ * One kernel launch.  Calls on the same cache must be stream-ordered.
+ */
+int32_t uf_kv_append(uf_kv_cache *c, const void *k_new, const void *v_new,
+                     int32_t keep_chunks, int32_t flags, uf_stream_t s);
+
+/*
+ * Dynamic block mask of the newest chunk's queries (Ultra Flash notes, Method,
+ * key design 3: tokens are cut into non-overlapping blocks; queries and keys
+ * are mean-pooled per block; blocks are scored by the dot product of the
+ * pooled query and key; each head keeps its top-k highest-scoring blocks).
+ *
+ *   q       device bf16 [B, Lc, H, D]: queries of the newest chunk of the
+ *           window (the chunk appended last).  H % c->G == 0.
+ *   k       kept blocks per q-block, counting the diagonal; 1 <= k <= W * nb.
+ *           On the device it is clamped to NKV (first chunks of a stream).
+ *   idx     device int32 [B, H, nb, k] out: logical kv block ids of the kept
+ *           blocks of each (b, h, q-block i) row, ascending; entries past
+ *           cnt are set to -1.
+ *   cnt     device int32 [B, H, nb] out: kept blocks per row = min(k, NKV).
+ *   scores  optional device fp32 [B, H, nb, W * nb] out (NULL = not written):
+ *           pooled scores mean(q_i) . mean(k_j) / sqrt(D) in logical order;
+ *           columns >= NKV are not written.
+ *
+ * Selection rule per row: the diagonal block d_i = (n_valid - 1) * nb + i is
+ * always kept; the other blocks are ranked by (score descending, logical id
+ * ascending) and the first k - 1 are kept.  Pooling means divide by the true
+ * token count of each block (the chunk's last block may be partial).  Scores
+ * are computed in fp32.  One kernel launch.
+ */
+int32_t uf_block_mask(const void *q, int32_t H, const uf_kv_cache *c, int32_t k,
+                      int32_t *idx, int32_t *cnt, float *scores, uf_stream_t s);
+
+/*
+ * Block-sparse chunk-causal attention (Ultra Flash notes, key design 3:
+ * attention computed only over the kept blocks; FlashDecoder Sec. 3.3:
+ * causality by processing order, no token mask inside the window; Eq. 4:
+ * grouped-query KV heads).
+ *
+ *   q      device bf16 [B, Lc, H, D]: queries of the newest chunk.
+ *   idx    device int32 [B, H, nb, k] logical kv block ids (any order, no
+ *          duplicates; as written by uf_block_mask), or NULL for dense
+ *          attention over every block of the window (density 1.0).
+ *   cnt    device int32 [B, H, nb]: number of valid entries of each idx row
+ *          (1..k); NULL = every row has k entries.  Ignored when idx is NULL.
+ *   k      row stride of idx (ignored when idx is NULL).
+ *   scale  softmax scale applied to q . k (1 / sqrt(D) for standard attention).
+ *   o      device bf16 [B, Lc, H, D] out: sum_j softmax_j(scale q.k_j) v_j over
+ *          the valid tokens of the kept blocks; query head h reads KV head
+ *          h / (H / G).
+ *   lse    optional device fp32 [B, H, Lc] out: natural-log
+ *          log-sum-exp of scale * q . k over the same tokens (NULL = skip).
+ *
+ * Device checks: an idx entry outside [0, NKV) is replaced by the row's
+ * diagonal block and UF_EBOUNDS is recorded; a row with cnt < 1 gets O = 0,
+ * LSE = -inf and UF_EBOUNDS.  One kernel launch (tcgen05 tensor cores, TMA).
+ */
+int32_t uf_block_sparse_attn(const void *q, int32_t H, const uf_kv_cache *c,
+                             const int32_t *idx, const int32_t *cnt, int32_t k, float scale,
+                             void *o, float *lse, uf_stream_t s);
+
+/*
+ * Read the device-side error word of the current device (the first error a
+ * kernel recorded since the last clear) into *status; clear it if `clear` is
+ * non-zero.  Synchronises the device (this is the one call that does).
+ */
+int32_t uf_get_error(int32_t *status, int32_t clear);
+
+/*
+ * Text of the last CUDA error that made a call of this thread return
+ * UF_ECUDA (static string, never NULL; "no error" if none).
+ */
+const char *uf_last_cuda_error(void);
+
+/*
+ * Set the bound on every pipeline wait inside the kernels, in SM clock cycles
+ * (default 2^31, about one second at B200 clocks).  A wait that reaches the
+ * bound records UF_ETIMEOUT and makes its kernel return early.  Host only;
+ * applies to launches made after the call.  UF_EINVAL if cycles < 1000.
+ */
+int32_t uf_set_wait_limit(int64_t cycles);
+
+/*
+ * Self-test of the bounded-wait path: launch one thread that waits on a
+ * pipeline barrier that nothing will ever complete, with a bound of `cycles`.
+ * The kernel records UF_ETIMEOUT and returns; it never hangs.  For tests.
+ */
+int32_t uf_debug_wait_timeout(int64_t cycles, uf_stream_t s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* UF_H */

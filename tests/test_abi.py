@@ -1,0 +1,141 @@
+"""C-ABI checks that need no GPU: the library loads, exports every entry point
+the header declares, and rejects bad arguments on the host before any CUDA
+call is made."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "uf.h")
+
+
+@pytest.fixture(scope="module")
+def uf(built_lib):
+    return built_lib
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[a-z_0-9]+\s*\*?\s*(uf_[a-z_0-9]+)\s*\(", text, flags=re.M)))
+
+
+def test_header_declares_the_three_calls():
+    names = declared_functions()
+    for n in ("uf_kv_append", "uf_block_mask", "uf_block_sparse_attn"):
+        assert n in names
+    assert len(names) >= 10
+
+
+def test_library_exports_every_declared_symbol(uf):
+    lib = ctypes.CDLL(os.path.join(ROOT, "block_sparse_causal_b200", "libuf.so"))
+    for n in declared_functions():
+        assert hasattr(lib, n), n
+    out = subprocess.run(["nm", "-D", "--defined-only", lib._name], capture_output=True, text=True).stdout
+    exported = set(re.findall(r" T (uf_[a-z_0-9]+)$", out, flags=re.M))
+    assert set(declared_functions()) <= exported
+
+
+def test_version_and_strerror(uf):
+    assert uf.uf_version() >= 100
+    for code in range(6):
+        assert uf.strerror(code).startswith("UF_")
+    assert uf.strerror(99) == "UF_UNKNOWN"
+
+
+def test_cache_bytes(uf):
+    kv, kp, meta = uf.uf_kv_cache_bytes(1, 12, 128, 2, 18720, 128)
+    assert kv == 1 * 12 * 2 * (147 * 128) * 128 * 2
+    assert kp == 1 * 12 * 2 * 147 * 128 * 4
+    assert meta == 16
+    kv, kp, _ = uf.uf_kv_cache_bytes(1, 2, 128, 2, 256, 64)
+    assert kv == 2 * 2 * 256 * 128 * 2 and kp == 2 * 2 * 4 * 128 * 4
+    for bad in [(0, 12, 128, 2, 100, 128), (1, 12, 64, 2, 100, 128), (1, 12, 128, 0, 100, 128),
+                (1, 12, 128, 65, 100, 128), (1, 12, 128, 2, 0, 128), (1, 12, 128, 2, 100, 32)]:
+        with pytest.raises(uf.UfError) as e:
+            uf.uf_kv_cache_bytes(*bad)
+        assert e.value.status == uf.UF_EINVAL
+
+
+class FakeTensor:
+    """Stands in for a device tensor: only its address is read on the host."""
+
+    def __init__(self, addr):
+        self.addr = addr
+
+    def data_ptr(self):
+        return self.addr
+
+
+def _cache(uf, **kw):
+    d = dict(B=1, G=2, D=128, W=2, Lc=300, blk=128)
+    d.update(kw)
+    return uf.uf_kv_cache_init(FakeTensor(0x100000), FakeTensor(0x200000), FakeTensor(0x300000),
+                               FakeTensor(0x400000), d["B"], d["G"], d["D"], d["W"], d["Lc"], d["blk"])
+
+
+def test_cache_init_validates_on_host(uf):
+    c = _cache(uf)
+    assert (c.B, c.G, c.W, c.Lc, c.blk, c.host_n_valid) == (1, 2, 2, 300, 128, 0)
+    with pytest.raises(uf.UfError):
+        uf.uf_kv_cache_init(FakeTensor(0x100008), FakeTensor(0x200000), FakeTensor(0x300000),
+                            FakeTensor(0x400000), 1, 2, 128, 2, 300, 128)     # misaligned k
+    with pytest.raises(uf.UfError):
+        uf.uf_kv_cache_init(None, FakeTensor(0x200000), FakeTensor(0x300000), FakeTensor(0x400000),
+                            1, 2, 128, 2, 300, 128)
+    with pytest.raises(uf.UfError):
+        _cache(uf, D=64)
+
+
+def test_calls_reject_bad_arguments_before_launch(uf):
+    c = _cache(uf)
+    q = FakeTensor(0x500000)
+    kn, vn = FakeTensor(0x600000), FakeTensor(0x700000)
+    # append: keep_chunks out of range, unknown flag, replace on an empty window, misaligned input
+    for keep, flags, k_new in [(0, 0, kn), (3, 0, kn), (2, 4, kn), (2, uf.UF_APPEND_REPLACE_NEWEST, kn),
+                               (2, 0, FakeTensor(0x600002))]:
+        with pytest.raises(uf.UfError) as e:
+            uf.uf_kv_append(c, k_new, vn, keep, flags, stream=0)
+        assert e.value.status == uf.UF_EINVAL
+    idx, cnt = FakeTensor(0x800000), FakeTensor(0x900000)
+    # mask / attention on an empty window (host mirror) are rejected
+    with pytest.raises(uf.UfError):
+        uf.uf_block_mask(q, 2, c, 2, idx, cnt, None, stream=0)
+    with pytest.raises(uf.UfError):
+        uf.uf_block_sparse_attn(q, 2, c, None, None, 0, 0.088, FakeTensor(0xA00000), None, stream=0)
+    c.host_n_valid = 1   # pretend one chunk is in the window; still no launch below
+    for H, k in [(3, 2), (0, 2), (2, 0), (2, 7)]:        # H % G != 0, H < 1, k < 1, k > W * nb (= 6)
+        with pytest.raises(uf.UfError) as e:
+            uf.uf_block_mask(q, H, c, k, idx, cnt, None, stream=0)
+        assert e.value.status == uf.UF_EINVAL
+    for scale in (0.0, -1.0, float("inf"), float("nan")):
+        with pytest.raises(uf.UfError) as e:
+            uf.uf_block_sparse_attn(q, 2, c, None, None, 0, scale, FakeTensor(0xA00000), None, stream=0)
+        assert e.value.status == uf.UF_EINVAL
+    with pytest.raises(uf.UfError):
+        uf.uf_block_sparse_attn(q, 2, c, idx, cnt, 9, 0.088, FakeTensor(0xA00000), None, stream=0)
+    with pytest.raises(uf.UfError):
+        uf.uf_block_sparse_attn(q, 2, c, None, None, 0, 0.088, FakeTensor(0xA00001), None, stream=0)
+
+
+def test_wait_limit_bounds(uf):
+    with pytest.raises(uf.UfError):
+        uf.uf_set_wait_limit(10)
+    uf.uf_set_wait_limit(1 << 31)
+    with pytest.raises(uf.UfError):
+        uf.uf_debug_wait_timeout(5, stream=0)
+
+
+def test_binding_fails_loudly_without_library(tmp_path):
+    # a copy of the package without libuf.so must refuse to import (no CPU fallback)
+    import shutil
+    import sys
+    pkg = os.path.join(ROOT, "block_sparse_causal_b200")
+    dst = tmp_path / "block_sparse_causal_b200"
+    shutil.copytree(pkg, dst, ignore=shutil.ignore_patterns("*.so", "__pycache__", "csrc"))
+    code = "import block_sparse_causal_b200"
+    res = subprocess.run([sys.executable, "-c", code], cwd=tmp_path, capture_output=True, text=True)
+    assert res.returncode != 0 and "not built" in res.stderr
