@@ -1,0 +1,482 @@
+#!/usr/bin/env python3
+"""Benchmark of the chunk-causal block-sparse attention hot path on B200.
+
+One step = one chunk of one attention layer: uf_kv_append (the new chunk's K/V
+into the rolling window) -> uf_block_mask (pool, score, top-k) ->
+uf_block_sparse_attn, on seeded synthetic inputs of the chosen workload, with
+the window already full (steady state).  Inputs are resident in HBM before
+the timed region; every step's working set (Q, new K/V, the window, O) is
+larger than the 126 MB L2, so no flush is needed between steps.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--config 1k_sr] [--impl ours|reference]
+
+Under torchrun (N > 1) every rank runs an independent replica on its own GPU
+(weak scaling; the path needs no data exchange).  Rank 0 prints one JSON line.
+``--impl reference`` times the fp64 CPU oracle on bounded samples of the same
+workload instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from workloads import CONFIGS, chunk_inputs  # noqa: E402
+
+METRIC = "block-sparse chunk attn ms/chunk & kept-block TFLOP/s (% bf16 peak), 1 B200"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+ATTN_PROFILE = os.path.join(ROOT, "profiles", "attn_1k_sr_traffic.txt")
+ATTN_SOURCES = ["block_sparse_causal_b200/csrc/attention.cuh", "block_sparse_causal_b200/csrc/uf_device.cuh"]
+
+
+# ----------------------------------------------------------------- helpers --
+def load_peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            p = json.load(f)
+        return {k: float(p[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+    except (OSError, KeyError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for rel in ATTN_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def attn_traffic_per_launch(config_name: str):
+    """DRAM bytes per attention launch from the committed ncu summary, or None
+    when there is none for this workload or the kernel changed since."""
+    if config_name != "1k_sr" or not os.path.exists(ATTN_PROFILE):
+        return None
+    txt = open(ATTN_PROFILE).read()
+    m_hash = re.search(r"^source_hash:\s*(\S+)", txt, flags=re.M)
+    m_bytes = re.search(r"^traffic_bytes_per_launch:\s*([0-9.eE+]+)", txt, flags=re.M)
+    if not m_hash or not m_bytes or m_hash.group(1) != kernel_source_hash():
+        return None
+    return float(m_bytes.group(1))
+
+
+def valid_counts(cfg, device):
+    """Valid tokens of each q-block [nb] and of each logical kv block of a full window [W*nb]."""
+    vq = torch.full((cfg.nb,), cfg.blk, dtype=torch.float64, device=device)
+    vq[-1] = cfg.last_block_tokens
+    vkv = vq.repeat(cfg.W)
+    return vq, vkv
+
+
+def kept_flops(cfg, idx, cnt, device):
+    """Algorithmic attention FLOPs of one call: 4 * D per (query token, kept kv
+    token) pair (QK^T and PV), summed over kept (q-block, kv-block) pairs."""
+    vq, vkv = valid_counts(cfg, device)
+    if idx is None:
+        return 4.0 * cfg.D * cfg.B * cfg.H * float(vq.sum()) * float(vkv.sum())
+    k = idx.shape[-1]
+    pos = torch.arange(k, device=device)
+    live = pos.view(1, 1, 1, k) < cnt.unsqueeze(-1)
+    kv_tok = torch.where(live, vkv[idx.clamp(min=0).long()], torch.zeros((), dtype=torch.float64, device=device))
+    per_item = kv_tok.sum(-1) * vq.view(1, 1, -1)
+    return 4.0 * cfg.D * float(per_item.sum())
+
+
+def append_bytes(cfg):
+    # read K,V of the chunk; write them into the slot (incl. padding rows); write pooled K
+    chunk = cfg.B * cfg.Lc * cfg.G * cfg.D * 2
+    slot = cfg.B * cfg.lslot * cfg.G * cfg.D * 2
+    return 2 * chunk + 2 * slot + cfg.B * cfg.G * cfg.nb * cfg.D * 4
+
+
+def mask_bytes(cfg, k):
+    # read Q once; pooled K of the window once per KV head; write idx and cnt
+    return (cfg.B * cfg.Lc * cfg.H * cfg.D * 2 + cfg.B * cfg.G * cfg.nkv() * cfg.D * 4
+            + cfg.B * cfg.H * cfg.nb * (k + 1) * 4)
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock, power and throttle reasons while running."""
+
+    FIELDS = ("index,pci.bus_id,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device=None):
+        self.pci = ""
+        if device is not None:
+            props = torch.cuda.get_device_properties(device)
+            bus, dev, dom = (getattr(props, n, None) for n in ("pci_bus_id", "pci_device_id", "pci_domain_id"))
+            if isinstance(bus, int) and isinstance(dev, int):
+                self.pci = f"{bus:02x}:{dev:02x}.0"       # matches the tail of nvidia-smi's pci.bus_id
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.15)
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 10:
+                continue
+            if self.pci and not parts[1].lower().endswith(self.pci):
+                continue
+            rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(r[2]) for r in rows if num(r[2]) is not None]
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            for n, v in zip(names, r[6:10]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": num(rows[0][3]),
+                "power_w_max": max((num(r[4]) or 0.0) for r in rows), "samples": len(rows),
+                "reasons": sorted(reasons)}
+
+
+# --------------------------------------------------------------- GPU arm ----
+def run_ours(args, cfg, rank, world, device):
+    import block_sparse_causal_b200 as uf
+    stream = torch.cuda.current_stream()
+    k = cfg.k_for() if not cfg.dense else cfg.nkv()
+    scale = 1.0 / math.sqrt(cfg.D)
+
+    # seeded chunks, generated on the host, resident in HBM before timing
+    n_distinct = 3
+    host_chunks = [chunk_inputs(cfg, args.seed + 1000 * rank, t) for t in range(cfg.W + n_distinct)]
+    dev_chunks = [{n: x.to(device) for n, x in c.items()} for c in host_chunks]
+    win = uf.KVWindow(cfg.B, cfg.G, cfg.W, cfg.Lc, cfg.blk, cfg.D, device=device)
+    win.reset()
+    for t in range(cfg.W):                       # fill the window
+        win.append(dev_chunks[t]["k"], dev_chunks[t]["v"], keep_chunks=cfg.W)
+    o = torch.empty(cfg.B, cfg.Lc, cfg.H, cfg.D, dtype=torch.bfloat16, device=device)
+    lse = torch.empty(cfg.B, cfg.H, cfg.Lc, dtype=torch.float32, device=device)
+    n_idx = args.steps + args.warmup
+    idx = [torch.empty(cfg.B, cfg.H, cfg.nb, k, dtype=torch.int32, device=device) for _ in range(n_idx)]
+    cnt = [torch.empty(cfg.B, cfg.H, cfg.nb, dtype=torch.int32, device=device) for _ in range(n_idx)]
+
+    def step(s, chunk, ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        win.append(chunk["k"], chunk["v"], keep_chunks=cfg.W)
+        if ev is not None:
+            ev[1].record(stream)
+        if cfg.dense:
+            if ev is not None:
+                ev[2].record(stream)
+            uf.uf_block_sparse_attn(chunk["q"], cfg.H, win.desc, None, None, 0, scale, o, lse)
+        else:
+            uf.uf_block_mask(chunk["q"], cfg.H, win.desc, k, idx[s], cnt[s])
+            if ev is not None:
+                ev[2].record(stream)
+            uf.uf_block_sparse_attn(chunk["q"], cfg.H, win.desc, idx[s], cnt[s], k, scale, o, lse)
+        if ev is not None:
+            ev[3].record(stream)
+
+    launches_per_step = 2 if cfg.dense else 3
+    for s in range(args.warmup):
+        step(s, dev_chunks[cfg.W + s % n_distinct])
+    torch.cuda.synchronize()
+    if uf.uf_get_error() != 0:
+        raise RuntimeError("device-side error during warm-up")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(device)
+    sampler.start()
+    barrier(world)
+    torch.cuda.synchronize()
+    t_start.record(stream)
+    for s in range(args.steps):
+        step(args.warmup + s, dev_chunks[cfg.W + (args.warmup + s) % n_distinct], evs[s])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clocks = sampler.stop()
+    elapsed_ms = t_start.elapsed_time(t_end)
+    per = {"append": 0.0, "mask": 0.0, "attn": 0.0}
+    for ev in evs:
+        per["append"] += ev[0].elapsed_time(ev[1])
+        per["mask"] += ev[1].elapsed_time(ev[2])
+        per["attn"] += ev[2].elapsed_time(ev[3])
+    per = {n: v / args.steps for n, v in per.items()}
+    if uf.uf_get_error() != 0:
+        raise RuntimeError("device-side error during the timed steps")
+
+    flops = [kept_flops(cfg, None if cfg.dense else idx[args.warmup + s],
+                        None if cfg.dense else cnt[args.warmup + s], device) for s in range(args.steps)]
+    flops_per_step = sum(flops) / len(flops)
+    max_ms = all_max(elapsed_ms, world, device)
+
+    # e2e: the same steps through the C ABI from pinned host buffers, with the
+    # inputs copied in and O / LSE copied out inside the timed region
+    pinned = [{n: x.pin_memory() for n, x in c.items()} for c in host_chunks[cfg.W:]]
+    stage = {n: torch.empty_like(x, device=device) for n, x in dev_chunks[0].items()}
+    o_host = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    lse_host = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+    e2e_steps = max(3, min(args.steps, 50))
+
+    def e2e_step(s):
+        src = pinned[s % n_distinct]
+        for n in ("q", "k", "v"):
+            stage[n].copy_(src[n], non_blocking=True)
+        step(s % n_idx, stage)
+        o_host.copy_(o, non_blocking=True)
+        lse_host.copy_(lse, non_blocking=True)
+
+    e2e_step(0)
+    torch.cuda.synchronize()
+    sampler2 = ClockSampler(device)
+    sampler2.start()
+    barrier(world)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for s in range(e2e_steps):
+        e2e_step(s + 1)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    sampler2.stop()
+    e2e_ms = all_max(e0.elapsed_time(e1), world, device) / e2e_steps
+    h2d = sum(stage[n].numel() * stage[n].element_size() for n in ("q", "k", "v"))
+    d2h = o.numel() * o.element_size() + lse.numel() * lse.element_size()
+
+    ms_per_step = max_ms / args.steps
+    value = world * flops_per_step / (ms_per_step * 1e-3) / 1e12
+    peaks, peaks_src = load_peaks()
+    attn_tflops = flops_per_step / (per["attn"] * 1e-3) / 1e12
+    traffic = attn_traffic_per_launch(args.config)
+    hbm = peaks["hbm_gbs"]
+    kernels = {
+        "append": {"ms": per["append"], "GB/s": append_bytes(cfg) / (per["append"] * 1e-3) / 1e9},
+        "attn": {"ms": per["attn"], "TFLOP/s": attn_tflops},
+    }
+    kernels["append"]["frac_of_measured_hbm"] = kernels["append"]["GB/s"] / hbm
+    if not cfg.dense:
+        kernels["mask"] = {"ms": per["mask"], "GB/s": mask_bytes(cfg, k) / (per["mask"] * 1e-3) / 1e9}
+        kernels["mask"]["frac_of_measured_hbm"] = kernels["mask"]["GB/s"] / hbm
+    result = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_per_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {
+            "workload": args.config, "description": cfg.description, "B": cfg.B, "H": cfg.H, "G": cfg.G,
+            "D": cfg.D, "Lc": cfg.Lc, "W": cfg.W, "blk": cfg.blk, "k": k,
+            "density": cfg.density, "kept_flops_per_step": flops_per_step,
+            "step": "uf_kv_append + " + ("" if cfg.dense else "uf_block_mask + ") + "uf_block_sparse_attn",
+            "l2": "no flush: every step's working set (%.0f MB) exceeds the 126 MB L2" % (
+                (cfg.B * cfg.Lc * (cfg.H * 2 + cfg.G * 2) * cfg.D * 2
+                 + 2 * cfg.B * cfg.G * cfg.nkv() * cfg.blk * cfg.D * 2) / 1e6),
+            "parallelism": "replicas" if world > 1 else "single",
+        },
+        "ms_per_chunk": ms_per_step,
+        "kernels": kernels,
+        "roofline": {
+            "bound": "tensor",
+            "achieved": attn_tflops,
+            "peak": peaks["bf16_tflops"],
+            "unit": "TFLOP/s",
+            "frac": attn_tflops / peaks["bf16_tflops"],
+            "traffic": traffic,
+            "kernel": "uf::attn_kernel<128>" if cfg.blk == 128 else "uf::attn_kernel<64>",
+            "peak_source": f"{peaks_src} bf16 dense burst (cuBLAS 8192^3)",
+        },
+        "e2e": {"value": world * flops_per_step / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "clocks": clocks,
+        "gpu_launches": launches_per_step * args.steps,
+    }
+    return result
+
+
+# --------------------------------------------------------- CPU oracle arm ---
+class OracleSample:
+    """The fp64 oracle (as it stands) on a bounded sample of the workload: the
+    mask of one query head over the full window, then attention for up to
+    ``n_items`` work items of that head.  Inputs are prepared once."""
+
+    def __init__(self, cfg, seed):
+        import oracle
+        from workloads import to_f64
+        self.oracle = oracle
+        self.cfg = cfg
+        chunks = [chunk_inputs(cfg, seed, t) for t in range(cfg.W)]
+        self.win = oracle.RollingWindow(cfg.W)
+        for c in chunks:
+            self.win.append(to_f64(c["k"][:, :, 0:1]), to_f64(c["v"][:, :, 0:1]))
+        self.q = to_f64(chunks[-1]["q"][:, :, 0:1])
+        self.k = cfg.k_for() if not cfg.dense else cfg.nkv()
+        self.vq = [cfg.blk] * (cfg.nb - 1) + [cfg.last_block_tokens]
+        self.vkv = self.vq * cfg.W
+
+    def run(self, n_items, budget_s, first_item=0):
+        """Returns (kept FLOPs computed, seconds, description)."""
+        cfg = self.cfg
+        t0 = time.perf_counter()
+        m = self.oracle.block_mask(self.q, self.win, cfg.blk, self.k)
+        flops = 0.0
+        done = 0
+        while done < n_items and time.perf_counter() - t0 < budget_s:
+            i = (first_item + done) % cfg.nb
+            self.oracle.block_sparse_attention(self.q, self.win, cfg.blk, m["idx"], m["cnt"], items=[(0, 0, i)])
+            flops += 4.0 * cfg.D * self.vq[i] * sum(self.vkv[j] for j in m["idx"][0, 0, i])
+            done += 1
+        dt = time.perf_counter() - t0
+        return flops, dt, (f"mask of 1 head ({cfg.nb} q-blocks over {cfg.nkv()} kv blocks) "
+                           f"+ attention of {done} work items")
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [d.get("num_threads") for d in threadpool_info() if d.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count()
+
+
+def cpu_baseline(cfg, seed):
+    flops, dt, desc = OracleSample(cfg, seed).run(n_items=10_000, budget_s=12.0)
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": desc + f", {dt:.1f} s of fp64 numpy", "seconds": dt}
+
+
+def run_reference(args, cfg):
+    # each step: the oracle on a bounded sample (one head's mask + 1 work item)
+    sample = OracleSample(cfg, args.seed)
+    for s in range(args.warmup):
+        sample.run(n_items=1, budget_s=5.0, first_item=s)
+    tot_f, tot_t = 0.0, 0.0
+    desc = ""
+    for s in range(args.steps):
+        f, t, desc = sample.run(n_items=1, budget_s=5.0, first_item=s)
+        tot_f += f
+        tot_t += t
+    value = tot_f / tot_t / 1e12
+    k = cfg.k_for() if not cfg.dense else cfg.nkv()
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot_t / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": args.config, "description": cfg.description, "B": cfg.B, "H": cfg.H, "G": cfg.G,
+                   "D": cfg.D, "Lc": cfg.Lc, "W": cfg.W, "blk": cfg.blk, "k": k, "density": cfg.density},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+                         "sample": "per step: " + desc},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+# ------------------------------------------------------------ distributed ---
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def all_max(x, world, device):
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--config", default="1k_sr", choices=sorted(CONFIGS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing leg")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    cfg = CONFIGS[args.config]
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        print(json.dumps(run_reference(args, cfg)), flush=True)
+        return 0
+
+    if world > 1:
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=180),
+                                             device_id=torch.device("cuda", local_rank))
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    try:
+        result = run_ours(args, cfg, rank, world, device)
+        if rank == 0:
+            if world == 1 and not args.no_cpu_baseline:
+                result["cpu_baseline"] = cpu_baseline(cfg, args.seed)
+            else:
+                result["cpu_baseline"] = None
+            print(json.dumps(result), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())
