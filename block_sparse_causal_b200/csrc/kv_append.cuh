@@ -6,14 +6,19 @@
 // key design 4: reuse of the last denoising step's KV (here: overwrite the
 // newest chunk) and adaptive cropping of the SR KV window (here: keep_chunks).
 //
-// One thread block per (block r of the chunk, KV head g, batch b).  256
-// threads = 16 token lanes x 16 sixteen-byte column chunks of a 256-byte token
-// row, so every warp moves two whole rows per instruction on both sides.  The
-// block also reduces its tokens' K into the slot's pooled-K row (fp32 mean over
-// the block's true tokens), which the block-mask call reads instead of
-// re-reading the window.  The last thread block to finish commits the new
-// window state to meta; every block read the old state before counting in, so
-// no block can observe a half-updated window.
+// One thread block per (block r of the chunk, KV head g, batch b), 256
+// threads.  K is copied row for row (16 token lanes x 16 sixteen-byte column
+// chunks of a 256-byte token row: every warp moves two whole rows per
+// instruction on both sides) and reduced into the slot's pooled-K row (fp32
+// mean over the block's true tokens), which the block-mask call reads instead
+// of re-reading the window.  V is stored transposed (head dim outermost,
+// tokens contiguous) so that the attention's PV product reads it as a K-major
+// operand: each thread loads an 8-token x 8-channel bf16 tile, transposes it
+// in registers with byte permutes and writes 8 sixteen-byte token runs, so
+// each warp writes two contiguous 256-byte runs per instruction.  The last
+// thread block to finish commits the new window state to meta; every block
+// read the old state before counting in, so no block can observe a
+// half-updated window.
 #pragma once
 
 #include "uf_device.cuh"
@@ -24,7 +29,7 @@ struct AppendParams {
   const __nv_bfloat16 *k_new;  // [B, Lc, G, D]
   const __nv_bfloat16 *v_new;
   __nv_bfloat16 *k;            // [B, G, W*Lslot, D]
-  __nv_bfloat16 *v;
+  __nv_bfloat16 *v;            // [B, G, D, W*Lslot] (transposed)
   float *kpool;                // [B, G, W*nb, D]
   int32_t *meta;               // {start, n_valid, counter, reserved}
   int32_t G, W, Lc, nb, lslot, keep, replace;
@@ -47,6 +52,50 @@ __device__ __forceinline__ void append_plan(int32_t start, int32_t n, int32_t W,
     start2 = (start2 + (n2 - keep)) % W;
     n2 = keep;
   }
+}
+
+// In-register transpose of an 8x8 tile of 16-bit values: in[r] holds row r
+// (8 values, lowest address first); out[c] receives column c.
+__device__ __forceinline__ void transpose8x8_b16(const uint4 (&in)[8], uint4 (&out)[8]) {
+  uint32_t w[8][4];
+#pragma unroll
+  for (int r = 0; r < 8; ++r) {
+    w[r][0] = in[r].x;
+    w[r][1] = in[r].y;
+    w[r][2] = in[r].z;
+    w[r][3] = in[r].w;
+  }
+  // stage 1: 2x2 blocks of 16-bit values between row pairs (r, r+1)
+#pragma unroll
+  for (int r = 0; r < 8; r += 2)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const uint32_t a = w[r][c], b = w[r + 1][c];
+      w[r][c] = __byte_perm(a, b, 0x5410);       // (a.lo, b.lo)
+      w[r + 1][c] = __byte_perm(a, b, 0x7632);   // (a.hi, b.hi)
+    }
+  // stage 2: 2x2 blocks of 32-bit words between rows (r, r+2)
+#pragma unroll
+  for (int r0 = 0; r0 < 8; r0 += 4)
+#pragma unroll
+    for (int r = r0; r < r0 + 2; ++r)
+#pragma unroll
+      for (int c = 0; c < 4; c += 2) {
+        const uint32_t t = w[r][c + 1];
+        w[r][c + 1] = w[r + 2][c];
+        w[r + 2][c] = t;
+      }
+  // stage 3: 2x2 blocks of 64-bit pairs between rows (r, r+4)
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    uint32_t t0 = w[r][2], t1 = w[r][3];
+    w[r][2] = w[r + 4][0];
+    w[r][3] = w[r + 4][1];
+    w[r + 4][0] = t0;
+    w[r + 4][1] = t1;
+  }
+#pragma unroll
+  for (int c = 0; c < 8; ++c) out[c] = make_uint4(w[c][0], w[c][1], w[c][2], w[c][3]);
 }
 
 template <int BLK>
@@ -79,21 +128,32 @@ __global__ void __launch_bounds__(256) kv_append_kernel(const AppendParams p) {
   const int cnt = min(BLK, p.Lc - t0);
   const size_t src_stride = static_cast<size_t>(p.G) * D;                       // elements per token
   const __nv_bfloat16 *ksrc = p.k_new + (static_cast<size_t>(b) * p.Lc + t0) * src_stride + g * D + dc * 8;
-  const __nv_bfloat16 *vsrc = p.v_new + (static_cast<size_t>(b) * p.Lc + t0) * src_stride + g * D + dc * 8;
   const size_t dst_row0 = (static_cast<size_t>(b) * p.G + g) * p.W * p.lslot + static_cast<size_t>(slot) * p.lslot + t0;
   __nv_bfloat16 *kdst = p.k + dst_row0 * D + dc * 8;
-  __nv_bfloat16 *vdst = p.v + dst_row0 * D + dc * 8;
 
-  uint4 kr[PASSES], vr[PASSES];
+  uint4 kr[PASSES];
 #pragma unroll
   for (int m = 0; m < PASSES; ++m) {
     const int t = tl + 16 * m;
-    if (t < cnt) {
-      kr[m] = __ldg(reinterpret_cast<const uint4 *>(ksrc + t * src_stride));
-      vr[m] = __ldg(reinterpret_cast<const uint4 *>(vsrc + t * src_stride));
-    } else {
-      kr[m] = make_uint4(0, 0, 0, 0);   // padding rows of the chunk's last block
-      vr[m] = make_uint4(0, 0, 0, 0);
+    kr[m] = (t < cnt) ? __ldg(reinterpret_cast<const uint4 *>(ksrc + t * src_stride))
+                      : make_uint4(0, 0, 0, 0);   // padding rows of the chunk's last block
+  }
+  // V tile of this thread: tokens 8*tg .. 8*tg+7, channels 8*cg .. 8*cg+7
+  constexpr int TG = BLK / 8;                      // token groups (16 or 8)
+  constexpr int VTILES = (BLK / 8) * 16 / 256;     // 8x8 tiles per thread (1 for BLK 128)
+  uint4 vr[VTILES > 0 ? VTILES : 1][8];
+  const int vtiles = (BLK / 8) * 16;               // 8x8 tiles in the block
+#pragma unroll
+  for (int q = 0; q < (VTILES > 0 ? VTILES : 1); ++q) {
+    const int tile = tid + 256 * q;
+    const int tg = tile % TG, cg = tile / TG;
+    if (tile < vtiles) {
+      const __nv_bfloat16 *src =
+          p.v_new + (static_cast<size_t>(b) * p.Lc + t0 + 8 * tg) * src_stride + g * D + 8 * cg;
+#pragma unroll
+      for (int e = 0; e < 8; ++e)
+        vr[q][e] = (8 * tg + e < cnt) ? __ldg(reinterpret_cast<const uint4 *>(src + e * src_stride))
+                                       : make_uint4(0, 0, 0, 0);
     }
   }
   float acc[8];
@@ -103,13 +163,29 @@ __global__ void __launch_bounds__(256) kv_append_kernel(const AppendParams p) {
   for (int m = 0; m < PASSES; ++m) {
     const int t = tl + 16 * m;
     *reinterpret_cast<uint4 *>(kdst + static_cast<size_t>(t) * D) = kr[m];
-    *reinterpret_cast<uint4 *>(vdst + static_cast<size_t>(t) * D) = vr[m];
     const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&kr[m]);
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       const float2 f = __bfloat1622float2(h2[e]);
       acc[2 * e] += f.x;
       acc[2 * e + 1] += f.y;
+    }
+  }
+  // V^T: row (b, g, channel) holds the window's tokens contiguously
+  const size_t vt_row_len = static_cast<size_t>(p.W) * p.lslot;
+  const size_t vt_col0 = static_cast<size_t>(slot) * p.lslot + t0;
+#pragma unroll
+  for (int q = 0; q < (VTILES > 0 ? VTILES : 1); ++q) {
+    const int tile = tid + 256 * q;
+    const int tg = tile % TG, cg = tile / TG;
+    if (tile < vtiles) {
+      uint4 vt[8];
+      transpose8x8_b16(vr[q], vt);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const size_t ch = (static_cast<size_t>(b) * p.G + g) * D + 8 * cg + e;
+        *reinterpret_cast<uint4 *>(p.v + ch * vt_row_len + vt_col0 + 8 * tg) = vt[e];
+      }
     }
   }
   // block mean of K over the block's true tokens (padding rows hold zeros)

@@ -288,10 +288,18 @@ int32_t uf_block_sparse_attn(const void *q, int32_t H, const uf_kv_cache *c, con
     if (!make_map(&tq, q, 4, dims, strides, box)) return UF_ECUDA;
   }
   {
+    // K: [B*G][W*Lslot][128] -> box {64 channels, blk tokens}
     const cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(c->W) * lslot, static_cast<cuuint64_t>(c->B) * c->G};
     const cuuint64_t strides[2] = {256, static_cast<cuuint64_t>(c->W) * lslot * 256};
     const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(c->blk), 1};
     if (!make_map(&tk, c->k, 3, dims, strides, box)) return UF_ECUDA;
+  }
+  {
+    // V^T: [B*G][128][W*Lslot] -> box {64 tokens, 128 channels}
+    const cuuint64_t row = static_cast<cuuint64_t>(c->W) * lslot;
+    const cuuint64_t dims[3] = {row, 128, static_cast<cuuint64_t>(c->B) * c->G};
+    const cuuint64_t strides[2] = {row * 2, row * 2 * 128};
+    const cuuint32_t box[3] = {64, 128, 1};
     if (!make_map(&tv, c->v, 3, dims, strides, box)) return UF_ECUDA;
   }
   uf::AttnParams p;

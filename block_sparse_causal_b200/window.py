@@ -18,8 +18,9 @@ class KVWindow:
         self.B, self.G, self.D, self.W, self.Lc, self.blk = B, G, D, W, Lc, blk
         self.nb = math.ceil(Lc / blk)
         self.lslot = self.nb * blk
+        # k: token rows [B, G, W*Lslot, D]; v: transposed [B, G, D, W*Lslot]
         self.k = torch.zeros(kv_bytes // 2, dtype=torch.bfloat16, device=device).view(B, G, W * self.lslot, D)
-        self.v = torch.zeros_like(self.k)
+        self.v = torch.zeros(kv_bytes // 2, dtype=torch.bfloat16, device=device).view(B, G, D, W * self.lslot)
         self.kpool = torch.zeros(kpool_bytes // 4, dtype=torch.float32, device=device).view(B, G, W * self.nb, D)
         self.meta = torch.zeros(meta_bytes // 4, dtype=torch.int32, device=device)
         self.desc = _uf.uf_kv_cache_init(self.k, self.v, self.kpool, self.meta, B, G, D, W, Lc, blk)

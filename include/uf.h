@@ -63,8 +63,12 @@ typedef enum uf_status {
  * kv block j of the window is block j % nb of logical chunk j / nb.  The
  * physical order is never visible through the API.
  *
- *   k, v   device bf16 [B, G, W * Lslot, D].  Rows past Lc inside a slot (the
- *          padding of the chunk's last block) are zeroed by uf_kv_append.
+ *   k      device bf16 [B, G, W * Lslot, D] (token rows).
+ *   v      device bf16 [B, G, D, W * Lslot] (transposed: each channel holds
+ *          the window's tokens contiguously, the layout the PV product reads
+ *          as a K-major tensor-core operand).  In both, the tokens past Lc
+ *          inside a slot (the padding of the chunk's last block) are zeroed
+ *          by uf_kv_append.
  *   kpool  device fp32 [B, G, W * nb, D]: mean of K over the true tokens of
  *          each block of each slot, written by uf_kv_append, read by
  *          uf_block_mask (pooling K once per chunk instead of once per call).
@@ -133,7 +137,8 @@ int32_t uf_kv_reset(uf_kv_cache *c, uf_stream_t s);
  *                 Rejected (UF_EINVAL) when the host mirror says the window is
  *                 empty; on the device an empty window turns it into an append.
  *
- * Writes the chunk into its ring slot of k / v (transposing BLGD -> BGLD),
+ * Writes the chunk into its ring slot of k (BLGD -> BGLD) and v (BLGD ->
+ * BGDL),
  * zeroes the slot's padding rows, writes the slot's block means into kpool and
  * advances meta (the last thread block to finish commits the new state).
  * One kernel launch.  Calls on the same cache must be stream-ordered.

@@ -45,7 +45,8 @@ def _slot_chunk(win, c, g, b=0):
     slot = (start + c) % win.W
     rows = slice(slot * win.lslot, slot * win.lslot + win.Lc)
     pad = slice(slot * win.lslot + win.Lc, (slot + 1) * win.lslot)
-    return slot, win.k[b, g, rows], win.v[b, g, rows], win.k[b, g, pad], win.v[b, g, pad]
+    # v is stored transposed: [B, G, D, W*Lslot]
+    return slot, win.k[b, g, rows], win.v[b, g, :, rows].t(), win.k[b, g, pad], win.v[b, g, :, pad].t()
 
 
 # ----------------------------------------------------------------- append ----
