@@ -370,21 +370,32 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
           }
         }
       }
-      // P = exp2(s * c - m): pairs through packed FMA / add
+      // P = exp2(s * c - m): pairs through packed FMA / add.  The full-block
+      // and the masked (partial last block of a chunk) cases are separate
+      // loops: a per-element mask test inside the unrolled loop costs two ALU
+      // instructions per element, which made the loop ALU-bound.
       const uint64_t negm2 = f2_pack(-m_use, -m_use);
       uint32_t pk[BLK / 2];
       uint64_t acc2[4] = {0, 0, 0, 0};
+      if (full) {
 #pragma unroll
-      for (int c = 0; c < BLK / 2; ++c) {
-        float x0, x1;
-        f2_unpack(f2_fma(f2_pack(__uint_as_float(s[2 * c]), __uint_as_float(s[2 * c + 1])), c2, negm2), x0, x1);
-        float e0 = ex2_approx(x0), e1 = ex2_approx(x1);
-        if (!full) {
-          if (2 * c >= valid) e0 = 0.f;
-          if (2 * c + 1 >= valid) e1 = 0.f;
+        for (int c = 0; c < BLK / 2; ++c) {
+          float x0, x1;
+          f2_unpack(f2_fma(f2_pack(__uint_as_float(s[2 * c]), __uint_as_float(s[2 * c + 1])), c2, negm2), x0, x1);
+          const float e0 = ex2_approx(x0), e1 = ex2_approx(x1);
+          acc2[c & 3] = f2_add(acc2[c & 3], f2_pack(e0, e1));
+          pk[c] = pack_bf16x2(e0, e1);
         }
-        acc2[c & 3] = f2_add(acc2[c & 3], f2_pack(e0, e1));
-        pk[c] = pack_bf16x2(e0, e1);
+      } else {
+#pragma unroll
+        for (int c = 0; c < BLK / 2; ++c) {
+          float x0, x1;
+          f2_unpack(f2_fma(f2_pack(__uint_as_float(s[2 * c]), __uint_as_float(s[2 * c + 1])), c2, negm2), x0, x1);
+          const float e0 = 2 * c < valid ? ex2_approx(x0) : 0.f;
+          const float e1 = 2 * c + 1 < valid ? ex2_approx(x1) : 0.f;
+          acc2[c & 3] = f2_add(acc2[c & 3], f2_pack(e0, e1));
+          pk[c] = pack_bf16x2(e0, e1);
+        }
       }
       {
         float a0, a1;
