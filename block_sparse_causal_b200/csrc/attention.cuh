@@ -320,81 +320,114 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
         if (!(ok = wwait(&bar_turn[0], u & 1))) break;
       }
       tc_fence_after();
-      uint32_t s[BLK];
-#pragma unroll
-      for (int c = 0; c < BLK / 32; ++c)
-        tmem_ld32(lane_base + s_col + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&s[32 * c]));
-      tmem_wait_ld();
       const bool full = valid == BLK;
-      float mx;
-      {
+      const uint64_t negm_run2 = f2_pack(-m_run, -m_run);
+      uint32_t pk[BLK / 2];
+      uint64_t acc2[4] = {0, 0, 0, 0};
+      float m_use = m_run;
+      float mx = -INFINITY;
+      bool done = false;
+      if (full && u > 0) {
+        // common case: exponentials against the running (possibly stale)
+        // max, with the block max computed in the same pass -- the max
+        // instructions hide under the SFU-bound exponentials.  Kept unless a
+        // row's block max exceeds the reference by more than 2^8.
+        uint32_t s[BLK];
+#pragma unroll
+        for (int c = 0; c < BLK / 32; ++c)
+          tmem_ld32(lane_base + s_col + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&s[32 * c]));
+        tmem_wait_ld();
         float a[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) a[e] = -INFINITY;
-        if (full) {
-#pragma unroll
-          for (int c = 0; c < BLK; c += 16)
-#pragma unroll
-            for (int e = 0; e < 8; ++e)
-              a[e] = max3f(a[e], __uint_as_float(s[c + 2 * e]), __uint_as_float(s[c + 2 * e + 1]));
-        } else {
-#pragma unroll
-          for (int c = 0; c < BLK; ++c)
-            if (c < valid) a[c & 7] = fmaxf(a[c & 7], __uint_as_float(s[c]));
-        }
-        mx = max3f(max3f(a[0], a[1], a[2]), max3f(a[3], a[4], a[5]), fmaxf(a[6], a[7]));
-      }
-      const float m_new = fmaxf(m_run, mx * c_log2);
-      const bool need = m_new > m_run + ATTN_RESCALE_LOG2;
-      float m_use = m_run;
-      if (__any_sync(0xffffffffu, need)) {
-        m_use = m_new;
-        const float factor = ex2_approx(m_run - m_new);
-        l_run *= factor;
-        if (u > 0) {
-          // PV_{t-2} into O_x completed before S_x for block t was computed
-          const uint64_t f2 = f2_pack(factor, factor);
-#pragma unroll 1
-          for (int c = 0; c < 4; ++c) {
-            uint32_t o[32];
-            tmem_ld32(lane_base + o_col + 32 * c, o);
-            tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              float lo, hi;
-              f2_unpack(f2_mul(f2_pack(__uint_as_float(o[2 * e]), __uint_as_float(o[2 * e + 1])), f2), lo, hi);
-              o[2 * e] = __float_as_uint(lo);
-              o[2 * e + 1] = __float_as_uint(hi);
-            }
-            tmem_st32(lane_base + o_col + 32 * c, o);
-          }
-        }
-      }
-      // P = exp2(s * c - m): pairs through packed FMA / add.  The full-block
-      // and the masked (partial last block of a chunk) cases are separate
-      // loops: a per-element mask test inside the unrolled loop costs two ALU
-      // instructions per element, which made the loop ALU-bound.
-      const uint64_t negm2 = f2_pack(-m_use, -m_use);
-      uint32_t pk[BLK / 2];
-      uint64_t acc2[4] = {0, 0, 0, 0};
-      if (full) {
 #pragma unroll
         for (int c = 0; c < BLK / 2; ++c) {
+          const float s0 = __uint_as_float(s[2 * c]), s1 = __uint_as_float(s[2 * c + 1]);
+          a[c & 7] = max3f(a[c & 7], s0, s1);
           float x0, x1;
-          f2_unpack(f2_fma(f2_pack(__uint_as_float(s[2 * c]), __uint_as_float(s[2 * c + 1])), c2, negm2), x0, x1);
+          f2_unpack(f2_fma(f2_pack(s0, s1), c2, negm_run2), x0, x1);
           const float e0 = ex2_approx(x0), e1 = ex2_approx(x1);
           acc2[c & 3] = f2_add(acc2[c & 3], f2_pack(e0, e1));
           pk[c] = pack_bf16x2(e0, e1);
         }
-      } else {
+        mx = max3f(max3f(a[0], a[1], a[2]), max3f(a[3], a[4], a[5]), fmaxf(a[6], a[7]));
+        done = !__any_sync(0xffffffffu, mx * c_log2 > m_run + ATTN_RESCALE_LOG2);
+      }
+      if (!done) {
+        // S is still intact in tensor memory: P is stored only below
+        uint32_t s[BLK];
 #pragma unroll
-        for (int c = 0; c < BLK / 2; ++c) {
-          float x0, x1;
-          f2_unpack(f2_fma(f2_pack(__uint_as_float(s[2 * c]), __uint_as_float(s[2 * c + 1])), c2, negm2), x0, x1);
-          const float e0 = 2 * c < valid ? ex2_approx(x0) : 0.f;
-          const float e1 = 2 * c + 1 < valid ? ex2_approx(x1) : 0.f;
-          acc2[c & 3] = f2_add(acc2[c & 3], f2_pack(e0, e1));
-          pk[c] = pack_bf16x2(e0, e1);
+        for (int c = 0; c < BLK / 32; ++c)
+          tmem_ld32(lane_base + s_col + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&s[32 * c]));
+        tmem_wait_ld();
+        if (!(full && u > 0)) {
+          // first block of the row or a partial block: the max first
+          float a[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) a[e] = -INFINITY;
+          if (full) {
+#pragma unroll
+            for (int c = 0; c < BLK; c += 16)
+#pragma unroll
+              for (int e = 0; e < 8; ++e)
+                a[e] = max3f(a[e], __uint_as_float(s[c + 2 * e]), __uint_as_float(s[c + 2 * e + 1]));
+          } else {
+#pragma unroll
+            for (int c = 0; c < BLK; ++c)
+              if (c < valid) a[c & 7] = fmaxf(a[c & 7], __uint_as_float(s[c]));
+          }
+          mx = max3f(max3f(a[0], a[1], a[2]), max3f(a[3], a[4], a[5]), fmaxf(a[6], a[7]));
+        }
+        const float m_new = fmaxf(m_run, mx * c_log2);
+        const bool need = m_new > m_run + ATTN_RESCALE_LOG2;
+        if (__any_sync(0xffffffffu, need)) {
+          m_use = m_new;
+          const float factor = ex2_approx(m_run - m_new);
+          l_run *= factor;
+          if (u > 0) {
+            // PV_{t-2} into O_x completed before S_x for block t was computed
+            const uint64_t f2 = f2_pack(factor, factor);
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
+              uint32_t o[32];
+              tmem_ld32(lane_base + o_col + 32 * c, o);
+              tmem_wait_ld();
+#pragma unroll
+              for (int e = 0; e < 16; ++e) {
+                float lo, hi;
+                f2_unpack(f2_mul(f2_pack(__uint_as_float(o[2 * e]), __uint_as_float(o[2 * e + 1])), f2), lo, hi);
+                o[2 * e] = __float_as_uint(lo);
+                o[2 * e + 1] = __float_as_uint(hi);
+              }
+              tmem_st32(lane_base + o_col + 32 * c, o);
+            }
+          }
+        }
+        // P = exp2(s * c - m): full-block and masked (partial last block of a
+        // chunk) cases are separate loops: a per-element mask test inside the
+        // unrolled loop costs two ALU instructions per element
+        const uint64_t negm2 = f2_pack(-m_use, -m_use);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc2[e] = 0;
+        if (full) {
+#pragma unroll
+          for (int c = 0; c < BLK / 2; ++c) {
+            float x0, x1;
+            f2_unpack(f2_fma(f2_pack(__uint_as_float(s[2 * c]), __uint_as_float(s[2 * c + 1])), c2, negm2), x0, x1);
+            const float e0 = ex2_approx(x0), e1 = ex2_approx(x1);
+            acc2[c & 3] = f2_add(acc2[c & 3], f2_pack(e0, e1));
+            pk[c] = pack_bf16x2(e0, e1);
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < BLK / 2; ++c) {
+            float x0, x1;
+            f2_unpack(f2_fma(f2_pack(__uint_as_float(s[2 * c]), __uint_as_float(s[2 * c + 1])), c2, negm2), x0, x1);
+            const float e0 = 2 * c < valid ? ex2_approx(x0) : 0.f;
+            const float e1 = 2 * c + 1 < valid ? ex2_approx(x1) : 0.f;
+            acc2[c & 3] = f2_add(acc2[c & 3], f2_pack(e0, e1));
+            pk[c] = pack_bf16x2(e0, e1);
+          }
         }
       }
       {
