@@ -21,7 +21,7 @@ namespace {
 
 constexpr int32_t UF_VERSION = 100;   // 0.1.0
 constexpr int32_t kMaxW = 64;
-constexpr int32_t kMaxMaskNKV = 5000; // pooled-score row kept in shared memory
+constexpr int32_t kMaxMaskNKV = 1024; // window blocks: 32 selection keys per lane
 constexpr int32_t kMaxDevices = 64;
 std::atomic<long long> g_wait_limit{1LL << 31};
 
@@ -68,13 +68,13 @@ EncodeTiledFn encode_fn() {
 
 // bf16 tensor map, 128-byte swizzle, box {64, box[1..]} (64 bf16 = 128 bytes inner).
 bool make_map(CUtensorMap *m, const void *base, int rank, const cuuint64_t *dims, const cuuint64_t *strides,
-              const cuuint32_t *box) {
+              const cuuint32_t *box, CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint32_t es[5] = {1, 1, 1, 1, 1};
   const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void *>(base), dims, strides, box, es,
-                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
@@ -104,7 +104,7 @@ int32_t ensure_smem(K kernel, int bytes, std::atomic<int> (&done)[kMaxDevices]) 
 int32_t launch_status() { return cuda_status(cudaGetLastError()); }
 
 std::atomic<int> g_attn128_smem[kMaxDevices], g_attn64_smem[kMaxDevices], g_mask128_smem[kMaxDevices],
-    g_mask64_smem[kMaxDevices];
+    g_mask64_smem[kMaxDevices], g_mask128b_smem[kMaxDevices], g_mask64b_smem[kMaxDevices];
 
 }  // namespace
 
@@ -227,6 +227,7 @@ int32_t uf_block_mask(const void *q, int32_t H, const uf_kv_cache *c, int32_t k,
   if (k < 1 || k > nkv_max) return UF_EINVAL;
   if (c->host_n_valid < 1) return UF_EINVAL;
   if (nkv_max > kMaxMaskNKV) return UF_EUNSUPPORTED;
+  if (reinterpret_cast<uintptr_t>(q) & 15u) return UF_EINVAL;
 
   uf::MaskParams p;
   p.q = static_cast<const __nv_bfloat16 *>(q);
@@ -242,18 +243,39 @@ int32_t uf_block_mask(const void *q, int32_t H, const uf_kv_cache *c, int32_t k,
   p.nb = nb;
   p.k = k;
   p.scale = 1.0f / sqrtf(static_cast<float>(c->D));
-  const int smem = (uf::MASK_TQ * 128 + 16 * 128 + uf::MASK_KT * uf::MASK_KSTRIDE + uf::MASK_TQ * nkv_max) * 4;
-  const dim3 grid(ceil_div(nb, uf::MASK_TQ), H, c->B);
-  cudaGetLastError();
-  if (c->blk == 128) {
-    const int32_t e = ensure_smem(uf::block_mask_kernel<128>, smem, g_mask128_smem);
-    if (e != UF_OK) return e;
-    uf::block_mask_kernel<128><<<grid, 256, smem, reinterpret_cast<cudaStream_t>(s)>>>(p);
-  } else {
-    const int32_t e = ensure_smem(uf::block_mask_kernel<64>, smem, g_mask64_smem);
-    if (e != UF_OK) return e;
-    uf::block_mask_kernel<64><<<grid, 256, smem, reinterpret_cast<cudaStream_t>(s)>>>(p);
+  const int smem = uf::mask_smem_bytes(c->blk, nkv_max);
+  // Q slices for the pooling: {channels, heads, tokens, batch}, box {64, 1, blk, 1}, no swizzle
+  CUtensorMap tq;
+  {
+    const cuuint64_t dims[4] = {128, static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(c->Lc),
+                                static_cast<cuuint64_t>(c->B)};
+    const cuuint64_t strides[3] = {256, static_cast<cuuint64_t>(H) * 256, static_cast<cuuint64_t>(c->Lc) * H * 256};
+    const cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(c->blk), 1};
+    if (!make_map(&tq, q, 4, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE)) return UF_ECUDA;
   }
+  const dim3 grid(ceil_div(nb, uf::MASK_TQ), H, c->B);
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(s);
+  cudaGetLastError();
+  // keys per lane of the selection: ceil(W*nb / 32) <= MAXPER
+  int32_t e = UF_OK;
+  if (c->blk == 128) {
+    if (nkv_max <= 512) {
+      e = ensure_smem(uf::block_mask_kernel<128, 16>, smem, g_mask128_smem);
+      if (e == UF_OK) uf::block_mask_kernel<128, 16><<<grid, 256, smem, st>>>(tq, p);
+    } else {
+      e = ensure_smem(uf::block_mask_kernel<128, 32>, smem, g_mask128b_smem);
+      if (e == UF_OK) uf::block_mask_kernel<128, 32><<<grid, 256, smem, st>>>(tq, p);
+    }
+  } else {
+    if (nkv_max <= 512) {
+      e = ensure_smem(uf::block_mask_kernel<64, 16>, smem, g_mask64_smem);
+      if (e == UF_OK) uf::block_mask_kernel<64, 16><<<grid, 256, smem, st>>>(tq, p);
+    } else {
+      e = ensure_smem(uf::block_mask_kernel<64, 32>, smem, g_mask64b_smem);
+      if (e == UF_OK) uf::block_mask_kernel<64, 32><<<grid, 256, smem, st>>>(tq, p);
+    }
+  }
+  if (e != UF_OK) return e;
   return launch_status();
 }
 

@@ -168,7 +168,7 @@ int32_t uf_kv_append(uf_kv_cache *c, const void *k_new, const void *v_new,
  * always kept; the other blocks are ranked by (score descending, logical id
  * ascending) and the first k - 1 are kept.  Pooling means divide by the true
  * token count of each block (the chunk's last block may be partial).  Scores
- * are computed in fp32.  One kernel launch.
+ * are computed in fp32.  UF_EUNSUPPORTED when W * nb > 1024.  One kernel launch.
  */
 int32_t uf_block_mask(const void *q, int32_t H, const uf_kv_cache *c, int32_t k,
                       int32_t *idx, int32_t *cnt, float *scores, uf_stream_t s);
