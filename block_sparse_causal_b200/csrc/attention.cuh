@@ -89,7 +89,7 @@ __device__ __forceinline__ void kv_block_coords(int j, int start, int W, int nb,
 template <int BLK>
 __global__ void __launch_bounds__(ATTN_THREADS, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
+                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO, const AttnParams p) {
   using L = AttnSmem<BLK>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -99,7 +99,7 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
   __shared__ uint64_t bar_q, bar_l;
   __shared__ uint64_t bar_fin[2];
   __shared__ uint64_t bar_full[ATTN_NSTAGE], bar_empty[ATTN_NSTAGE];
-  __shared__ uint64_t bar_s[2], bar_p[2], bar_o[2], bar_turn[2];
+  __shared__ uint64_t bar_s[2], bar_p[2], bar_o[2], bar_turn[2], bar_st[2];
   __shared__ uint32_t s_tbase;
   __shared__ int32_t s_abort;
 
@@ -138,6 +138,7 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
       mbar_init(&bar_p[s], ATTN_SOFTMAX_THREADS / 2);
       mbar_init(&bar_o[s], 1);
       mbar_init(&bar_turn[s], ATTN_SOFTMAX_THREADS / 2);
+      mbar_init(&bar_st[s], ATTN_SOFTMAX_THREADS / 2);
     }
     s_abort = 0;
     fence_mbar_init();
@@ -454,6 +455,15 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
     float *s_ml_mine = reinterpret_cast<float *>(sKV + x * ATTN_PSTAGE * L::STAGE);
     float *s_ml_other = reinterpret_cast<float *>(sKV + (x ^ 1) * ATTN_PSTAGE * L::STAGE);
     if (ok && !skip && n_x > 0) ok = wwait(&bar_o[x], (n_x - 1) & 1);
+    // this warpgroup writes output columns [64x, 64x + 64): its own pipeline's
+    // part of them is final already, the other pipeline's after bar_l
+    uint32_t own[64];
+    if (ok && !skip && n_x > 0) {
+      tc_fence_after();
+      tmem_ld32(lane_base + tm_o(x) + x * 64, *reinterpret_cast<uint32_t(*)[32]>(&own[0]));
+      tmem_ld32(lane_base + tm_o(x) + x * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&own[32]));
+      tmem_wait_ld();
+    }
     if (ok && !skip) {
       s_ml_mine[row] = m_run;
       s_ml_mine[128 + row] = l_run;
@@ -463,7 +473,6 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
     }
     const float *s_ml0 = x == 0 ? s_ml_mine : s_ml_other;
     const float *s_ml1 = x == 0 ? s_ml_other : s_ml_mine;
-    const size_t o_off = ((static_cast<size_t>(b) * p.Lc + q_tok) * p.H + h) * 128 + x * 64;
     if (ok && !skip) {
       tc_fence_after();
       const float m0 = s_ml0[row], m1 = s_ml1[row];
@@ -473,33 +482,50 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
       const float a1 = n1 > 0 ? ex2_approx(m1 - m) : 0.f;
       const float l_tot = l0 * a0 + l1 * a1;
       const float inv_l = 1.f / l_tot;
-      const float w0 = a0 * inv_l, w1 = a1 * inv_l;
-#pragma unroll 1
-      for (int c = 0; c < 2; ++c) {
-        const uint32_t col = x * 64 + 32 * c;             // this warpgroup's half of the columns
-        uint32_t o0[32], o1[32];
-        tmem_ld32(lane_base + tm_o(0) + col, o0);
-        if (n1 > 0) tmem_ld32(lane_base + tm_o(1) + col, o1);
+      const float w_own = (x == 0 ? a0 : a1) * inv_l, w_oth = (x == 0 ? a1 : a0) * inv_l;
+      const int n_oth = x == 0 ? n1 : n0;
+      uint32_t oth[64];
+      if (n_oth > 0) {
+        tmem_ld32(lane_base + tm_o(x ^ 1) + x * 64, *reinterpret_cast<uint32_t(*)[32]>(&oth[0]));
+        tmem_ld32(lane_base + tm_o(x ^ 1) + x * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&oth[32]));
         tmem_wait_ld();
-        if (row_out) {
-          uint32_t w[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            float v0 = __uint_as_float(o0[2 * e]) * w0, v1 = __uint_as_float(o0[2 * e + 1]) * w0;
-            if (n1 > 0) {
-              v0 = fmaf(__uint_as_float(o1[2 * e]), w1, v0);
-              v1 = fmaf(__uint_as_float(o1[2 * e + 1]), w1, v1);
-            }
-            w[e] = pack_bf16x2(v0, v1);
-          }
-          uint4 *dst = reinterpret_cast<uint4 *>(p.o + o_off + 32 * c);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) dst[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
-        }
       }
+      // stage the bf16 row half in the (now idle) Q tile, 128-byte swizzled
+      // like a TMA tile: 16-byte chunk c of row r sits at chunk c ^ (r mod 8)
+      uint8_t *panel = sQ + x * (L::Q_BYTES / 2) + row * 128;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        uint32_t w[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int k0 = 8 * c + 2 * e;
+          float v0 = 0.f, v1 = 0.f;
+          if (n_x > 0) {
+            v0 = __uint_as_float(own[k0]) * w_own;
+            v1 = __uint_as_float(own[k0 + 1]) * w_own;
+          }
+          if (n_oth > 0) {
+            v0 = fmaf(__uint_as_float(oth[k0]), w_oth, v0);
+            v1 = fmaf(__uint_as_float(oth[k0 + 1]), w_oth, v1);
+          }
+          w[e] = pack_bf16x2(v0, v1);
+        }
+        *reinterpret_cast<uint4 *>(panel + ((c ^ (row & 7)) * 16)) = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+      fence_proxy_async_smem();
       if (row_out && p.lse && x == 0)
         p.lse[(static_cast<size_t>(b) * p.H + h) * p.Lc + q_tok] = (m + log2f(l_tot)) * 0.69314718055994531f;
+      mbar_arrive(&bar_st[x]);
+      ok = wwait(&bar_st[x], 0);
+      if (ok && threadIdx.x == (4 + 4 * x) * 32) {
+        // one TMA store of this warpgroup's 64-column panel; rows past the
+        // q-block or past Lc are not written
+        tma_store_4d(&tmO, sQ + x * (L::Q_BYTES / 2), x * 64, h, i * BLK, b);
+        bulk_commit();
+        bulk_wait_read();
+      }
     } else if (skip && row_out) {
+      const size_t o_off = ((static_cast<size_t>(b) * p.Lc + q_tok) * p.H + h) * 128 + x * 64;
       uint4 *dst = reinterpret_cast<uint4 *>(p.o + o_off);
 #pragma unroll
       for (int e = 0; e < 8; ++e) dst[e] = make_uint4(0, 0, 0, 0);
