@@ -6,41 +6,40 @@
 // order); Eq. 4: grouped-query KV heads.
 //
 // One thread block = one work item (batch b, query head h, q-block i): a
-// 128-row Q tile against the item's list of n kept kv blocks, split inside the
-// block into two interleaved halves -- the even-numbered kept blocks (t = 0,
-// 2, 4, ...) and the odd-numbered ones -- processed by two independent
-// pipelines that share only the Q tile.  Pipeline x has its own TMA producer
-// warp, ring of K / V shared-memory stages, MMA-issuing warp, S and O
-// accumulators in tensor memory and softmax warpgroup; the two partial
-// results are merged once at the end with their running maxima and sums (the
-// merge rule of online softmax).  Two issuing warps keep two independent
-// instruction streams in front of the tensor core, which overlaps them.
+// 128-row Q tile against the item's list of n kept kv blocks t = 0 .. n-1,
+// accumulated into one O tile with an online softmax.  Both products run on
+// the tensor core with the A operand in tensor memory and a K-major B operand
+// in shared memory:
+//   S_t = Q K_t^T   (Q copied into tensor memory once per item)
+//   O  += P_t V_t   (P_t written to tensor memory by the softmax; V is stored
+//                    transposed in the window, so V_t^T is K-major too)
+// Tensor memory (512 columns): S buffers 0 and 1 [0,128) [128,256), O
+// [256,384), Q [384,448), P [448,512).  Block t uses S buffer t mod 2, so
+// S_{t+1} is computed while the softmax works on S_t, and S_{t+2} is issued as
+// soon as the softmax has read S_t into registers (P has its own columns).
 // Twelve warps:
-//   warps 0, 1   TMA producers of pipelines 0 and 1: the pipeline's K / V
-//                tiles gathered by the block list, in the order its MMA warp
-//                consumes them (K_x, then V_t, K_{t+2} for t = x, x+2, ...);
-//                warp 0 also loads the Q tile;
-//   warps 2, 3   MMA issuers (one thread each): S_x = Q K_t^T (SS, K-major
-//                operands, 128-byte swizzle) and O_x += P_x V_t (TS: P from
-//                tensor memory, V stored transposed in the window so it is a
-//                K-major operand too).  P_x is written over the first columns
-//                of S_x, so S_x is reused for block t + 2 only after PV_t has
-//                completed (MMAs into different accumulators are not ordered
-//                by the hardware); warp 2 owns the tensor-memory allocation;
-//   warps 4-7    softmax of pipeline 0, warps 8-11 of pipeline 1: each thread
-//                owns one row, reads it from S_x (32x32b loads), applies the
-//                block's token mask, keeps a running max / sum in the exp2
-//                domain, writes P as packed bf16 and rescales its row of O_x
-//                only when the running max grew by more than 2^8 (a stale max
-//                is exact: O_x and the sum share the same reference).  When
-//                S_x for block t arrives, PV_{t-2} into O_x has completed, so
-//                the softmax never waits for anything but its S.  The two
-//                softmax warpgroups take turns in global block order (t,
-//                t + 1, ...), so one always computes exponentials while the
-//                other pipeline's MMAs run (two pipelines left alone fall into
-//                lockstep and contend for the same units).
-// Tensor memory (512 columns): S0 [0,128) O0 [128,256) S1 [256,384)
-// O1 [384,512); P_x occupies the first BLK/2 columns of S_x.
+//   warps 0, 3   TMA producers of the K ring and of the V ring: the tiles
+//                gathered by the block list, in block order;
+//   warps 1, 2   one issuing thread each (an issuing thread waits for every
+//                MMA it issues to be accepted, so two of them keep the tensor
+//                core busy): warp 1 issues QK_{t+2} once S_t has been read and
+//                owns the tensor-memory allocation, warp 2 issues PV_t once
+//                P_t is in tensor memory;
+//   warps 4-7    softmax of the even-numbered kept blocks, warps 8-11 of the
+//                odd ones: each thread owns one row (32x32b loads), applies
+//                the block's token mask, computes exponentials in the exp2
+//                domain against a reference max and writes P as packed bf16.
+//                The reference max of each row lives in shared memory and is
+//                raised only when a block's max exceeds it by more than 2^8 (a
+//                stale max is exact: O and the sums share it); raising it
+//                rescales O in tensor memory.  Per block: S to registers, the
+//                block max, then the turn -- block t waits for block t - 1's
+//                decision on the reference, so decisions are taken in block
+//                order -- then S's buffer is released and the exponentials
+//                run from registers, overlapping those of the other
+//                warpgroup's block.  Each warpgroup keeps its own partial row
+//                sum relative to the reference it last saw; the two are
+//                combined at the end.
 #pragma once
 
 #include "uf_device.cuh"
@@ -49,32 +48,33 @@ namespace uf {
 
 constexpr int ATTN_THREADS = 384;
 constexpr int ATTN_SOFTMAX_THREADS = 256;
-constexpr int ATTN_NSTAGE = 6;                   // shared-memory stages, ATTN_NSTAGE / 2 per pipeline
-constexpr int ATTN_PSTAGE = ATTN_NSTAGE / 2;
-// tensor-memory column of S_x and of O_x
-__host__ __device__ constexpr uint32_t tm_s(int x) { return static_cast<uint32_t>(x) * 256u; }
-__host__ __device__ constexpr uint32_t tm_o(int x) { return 128u + static_cast<uint32_t>(x) * 256u; }
+constexpr int ATTN_KSTAGE = 4;                   // shared-memory stages of the K ring
+constexpr int ATTN_VSTAGE = 3;                   // and of the V ring
+// tensor-memory columns
+__host__ __device__ constexpr uint32_t tm_s(int x) { return static_cast<uint32_t>(x) * 128u; }
+constexpr uint32_t TM_O = 256, TM_Q = 384, TM_P = 448;
 constexpr float ATTN_RESCALE_LOG2 = 8.0f;
 
 struct AttnParams {
   const int32_t *meta;
-  const int32_t *idx;   // [B, H, nb, k] or NULL (dense)
-  const int32_t *cnt;   // [B, H, nb] or NULL
-  __nv_bfloat16 *o;     // [B, Lc, H, D]
-  float *lse;           // [B, H, Lc] or NULL
+  const int32_t *idx;        // [B, H, nb, k] or NULL (dense)
+  const int32_t *cnt;        // [B, H, nb] or NULL
+  const __nv_bfloat16 *q;    // [B, Lc, H, D]
+  float *lse;                // [B, H, Lc] or NULL
+  __nv_bfloat16 *o;          // [B, Lc, H, D] (skipped items are written directly)
   int32_t H, G, W, Lc, nb, lslot, k;
-  float scale_log2;     // softmax scale * log2(e)
+  float scale_log2;          // softmax scale * log2(e)
   long long wait_limit;
 };
 
 template <int BLK>
 struct AttnSmem {
-  static constexpr int Q_BYTES = 128 * 256;          // 128 rows x 128 d x bf16, two 64-column panels
   static constexpr int PANEL = BLK * 128;            // one 64-channel panel of a K tile
   static constexpr int VPANEL = 128 * 128;           // one 64-token panel of a V^T tile (128 channels)
   static constexpr int STAGE = BLK * 256;
-  static constexpr int DYN = 1024 + Q_BYTES + ATTN_NSTAGE * STAGE;
+  static constexpr int DYN = 1024 + (ATTN_KSTAGE + ATTN_VSTAGE) * STAGE;
 };
+static_assert(AttnSmem<128>::STAGE >= 2 * 128 * 128, "the epilogue stages a 128x128 bf16 O tile in one stage");
 
 // Logical kv block j of the window -> first row of its tile in the cache and
 // its number of true tokens.
@@ -88,18 +88,19 @@ __device__ __forceinline__ void kv_block_coords(int j, int start, int W, int nb,
 
 template <int BLK>
 __global__ void __launch_bounds__(ATTN_THREADS, 1)
-    attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO, const AttnParams p) {
+    attn_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                const __grid_constant__ CUtensorMap tmO, const AttnParams p) {
   using L = AttnSmem<BLK>;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t *sQ = smem;
-  uint8_t *sKV = smem + L::Q_BYTES;
+  uint8_t *sK = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t *sV = sK + ATTN_KSTAGE * L::STAGE;
 
-  __shared__ uint64_t bar_q, bar_l;
+  __shared__ uint64_t bar_q, bar_l, bar_p;
   __shared__ uint64_t bar_fin[2];
-  __shared__ uint64_t bar_full[ATTN_NSTAGE], bar_empty[ATTN_NSTAGE];
-  __shared__ uint64_t bar_s[2], bar_p[2], bar_o[2], bar_turn[2], bar_st[2];
+  __shared__ uint64_t bar_kfull[ATTN_KSTAGE], bar_kempty[ATTN_KSTAGE];
+  __shared__ uint64_t bar_vfull[ATTN_VSTAGE], bar_vempty[ATTN_VSTAGE];
+  __shared__ uint64_t bar_s[2], bar_sfree[2], bar_o[2], bar_turn[2], bar_st[2];
+  __shared__ float s_mref[128];   // reference max of each row (exp2 domain), published block by block
   __shared__ uint32_t s_tbase;
   __shared__ int32_t s_abort;
 
@@ -125,17 +126,22 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
   const bool skip = bad_meta || n < 1;
 
   if (threadIdx.x == 0) {
-    mbar_init(&bar_q, 1);
+    mbar_init(&bar_q, ATTN_SOFTMAX_THREADS);
+    mbar_init(&bar_l, ATTN_SOFTMAX_THREADS);
+    mbar_init(&bar_p, ATTN_SOFTMAX_THREADS / 2);
     mbar_init(&bar_fin[0], 1);
     mbar_init(&bar_fin[1], 1);
-    mbar_init(&bar_l, ATTN_SOFTMAX_THREADS);
-    for (int s = 0; s < ATTN_NSTAGE; ++s) {
-      mbar_init(&bar_full[s], 1);
-      mbar_init(&bar_empty[s], 1);
+    for (int s = 0; s < ATTN_KSTAGE; ++s) {
+      mbar_init(&bar_kfull[s], 1);
+      mbar_init(&bar_kempty[s], 1);
+    }
+    for (int s = 0; s < ATTN_VSTAGE; ++s) {
+      mbar_init(&bar_vfull[s], 1);
+      mbar_init(&bar_vempty[s], 1);
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bar_s[s], 1);
-      mbar_init(&bar_p[s], ATTN_SOFTMAX_THREADS / 2);
+      mbar_init(&bar_sfree[s], ATTN_SOFTMAX_THREADS / 2);
       mbar_init(&bar_o[s], 1);
       mbar_init(&bar_turn[s], ATTN_SOFTMAX_THREADS / 2);
       mbar_init(&bar_st[s], ATTN_SOFTMAX_THREADS / 2);
@@ -144,7 +150,7 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
     fence_mbar_init();
     if (skip) record_error(UF_EBOUNDS);
   }
-  if (warp == 2) {
+  if (warp == 1) {
     tmem_alloc(&s_tbase, 512);
     tmem_relinquish();
   }
@@ -154,27 +160,22 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
   const uint32_t tb = s_tbase;
   volatile int32_t *abort_flag = &s_abort;
 
-  if (warp < 2) {
-    // ------------------------------------------------------------ producer --
-    const int x = warp;                         // pipeline of this producer
-    const int n_mine = skip ? 0 : (n - x + 1) / 2;
+  if (warp == 0 || warp == 3) {
+    // ------------------------------------------------------------ producers -
+    const bool is_v = warp == 3;
+    const int nst = is_v ? ATTN_VSTAGE : ATTN_KSTAGE;
+    uint64_t *full_bars = is_v ? bar_vfull : bar_kfull;
+    uint64_t *empty_bars = is_v ? bar_vempty : bar_kempty;
+    uint8_t *ring = is_v ? sV : sK;
     if (lane == 0 && !skip) {
-      tma_prefetch_desc(&tmK);
-      tma_prefetch_desc(&tmV);
-      if (x == 0) {
-        tma_prefetch_desc(&tmQ);
-        mbar_arrive_expect_tx(&bar_q, L::Q_BYTES);
-        tma_load_4d(sQ, &tmQ, &bar_q, 0, h, i * BLK, b);
-        tma_load_4d(sQ + L::Q_BYTES / 2, &tmQ, &bar_q, 64, h, i * BLK, b);
-      }
+      tma_prefetch_desc(is_v ? &tmV : &tmK);
       const int zc = b * p.G + g;
-      const int stage0 = x * ATTN_PSTAGE;
       int stage = 0;
       uint32_t phase = 0;
       int issued = 0;
-      // same order as this pipeline's MMA warp consumes: K_x, then V_t, K_{t+2} for t = x, x+2, ...
-      auto load = [&](int t, bool is_v) -> bool {
-        if (!wait_bounded(&bar_empty[stage0 + stage], phase ^ 1u, abort_flag, p.wait_limit)) return false;
+      bool ok = true;
+      for (int t = 0; t < n && ok; ++t) {
+        if (!(ok = wait_bounded(&empty_bars[stage], phase ^ 1u, abort_flag, p.wait_limit))) break;
         int jb = row_idx ? __ldg(row_idx + t) : t;
         if (jb < 0 || jb >= NKV) {
           record_error(UF_EBOUNDS);
@@ -182,9 +183,9 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
         }
         int row, valid;
         kv_block_coords(jb, start, p.W, p.nb, p.lslot, BLK, p.Lc, row, valid);
-        uint64_t *full = &bar_full[stage0 + stage];
+        uint64_t *full = &full_bars[stage];
         mbar_arrive_expect_tx(full, L::STAGE);
-        uint8_t *dst = sKV + (stage0 + stage) * L::STAGE;
+        uint8_t *dst = ring + stage * L::STAGE;
         if (is_v) {
           // V^T tile: 128 channel rows x BLK tokens, in 64-token panels
 #pragma unroll
@@ -196,116 +197,137 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
           tma_load_3d(dst + L::PANEL, &tmK, full, 64, row, zc);
         }
         ++issued;
-        if (++stage == ATTN_PSTAGE) {
+        if (++stage == nst) {
           stage = 0;
           phase ^= 1u;
         }
-        return true;
-      };
-      bool ok = n_mine > 0 ? load(x, false) : true;
-      for (int u = 0; u < n_mine && ok; ++u) {
-        const int t = x + 2 * u;
-        ok = load(t, true);
-        if (ok && t + 2 < n) ok = load(t + 2, false);
       }
       if (!ok) {
         // unwind: let every load still in flight land before the block exits
         int s = stage;
         uint32_t ph = phase;
-        for (int q = 0; q < ATTN_PSTAGE && q < issued; ++q) {
+        for (int q = 0; q < nst && q < issued; ++q) {
           if (--s < 0) {
-            s = ATTN_PSTAGE - 1;
+            s = nst - 1;
             ph ^= 1u;
           }
           int32_t never = 0;
-          wait_bounded(&bar_full[stage0 + s], ph, &never, p.wait_limit);
+          wait_bounded(&full_bars[s], ph, &never, p.wait_limit);
         }
       }
     }
-  } else if (warp < 4) {
-    // ------------------------------------------------------------ MMA -------
-    const int x = warp - 2;                     // pipeline of this issuer
-    const int n_mine = skip ? 0 : (n - x + 1) / 2;
-    if (lane == 0 && n_mine > 0) {
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ QK issuer -
+    if (lane == 0 && !skip) {
       const uint32_t idesc_qk = idesc_bf16_f32(128, BLK, 0);
-      const uint32_t idesc_pv = idesc_bf16_f32(128, 128, 0);
-      const uint32_t q_addr = smem_u32(sQ);
-      const uint32_t kv_addr = smem_u32(sKV);
-      const int stage0 = x * ATTN_PSTAGE;
-      const uint32_t s_tmem = tb + tm_s(x), o_tmem = tb + tm_o(x);
+      const uint32_t k_base = smem_u32(sK);
       int stage = 0;
       uint32_t phase = 0;
-      bool ok = wait_bounded(&bar_q, 0, abort_flag, p.wait_limit);
-      if (ok) tc_fence_after();
-      auto advance = [&]() {
-        if (++stage == ATTN_PSTAGE) {
+      auto issue_qk = [&](int t) -> bool {
+        if (!wait_bounded(&bar_kfull[stage], phase, abort_flag, p.wait_limit)) return false;
+        tc_fence_after();
+        const uint32_t k_addr = k_base + stage * L::STAGE;
+        const uint32_t s_tmem = tb + tm_s(t & 1);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint64_t bd = sdesc_sw128(k_addr + (kk >> 2) * L::PANEL + (kk & 3) * 32, 16, 1024);
+          mma_ts(s_tmem, tb + TM_Q + kk * 8, bd, idesc_qk, kk > 0);
+        }
+        mma_commit(&bar_kempty[stage]);
+        mma_commit(&bar_s[t & 1]);
+        if (++stage == ATTN_KSTAGE) {
           stage = 0;
           phase ^= 1u;
         }
-      };
-      auto issue_qk = [&]() -> bool {
-        if (!wait_bounded(&bar_full[stage0 + stage], phase, abort_flag, p.wait_limit)) return false;
-        tc_fence_after();
-        const uint32_t k_addr = kv_addr + (stage0 + stage) * L::STAGE;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t off = (kk & 3) * 32;
-          const uint64_t ad = sdesc_sw128(q_addr + (kk >> 2) * (L::Q_BYTES / 2) + off, 16, 1024);
-          const uint64_t bd = sdesc_sw128(k_addr + (kk >> 2) * L::PANEL + off, 16, 1024);
-          mma_ss(s_tmem, ad, bd, idesc_qk, kk > 0);
-        }
-        mma_commit(&bar_empty[stage0 + stage]);
-        mma_commit(&bar_s[x]);
-        advance();
         return true;
       };
-      auto issue_pv = [&](int u) -> bool {
-        if (!wait_bounded(&bar_p[x], u & 1, abort_flag, p.wait_limit)) return false;
-        if (!wait_bounded(&bar_full[stage0 + stage], phase, abort_flag, p.wait_limit)) return false;
+      bool ok = wait_bounded(&bar_q, 0, abort_flag, p.wait_limit);
+      if (ok) tc_fence_after();
+      if (ok) ok = issue_qk(0);
+      if (ok && n > 1) ok = issue_qk(1);
+      for (int t = 0; t + 2 < n && ok; ++t) {
+        // S buffer t mod 2 is free once the softmax has read S_t
+        if (!(ok = wait_bounded(&bar_sfree[t & 1], (t >> 1) & 1, abort_flag, p.wait_limit))) break;
         tc_fence_after();
-        const uint32_t v_addr = kv_addr + (stage0 + stage) * L::STAGE;
+        ok = issue_qk(t + 2);
+      }
+      // every MMA issued by this thread has completed once bar_fin flips
+      mma_commit(&bar_fin[0]);
+      int32_t never = 0;
+      wait_bounded(&bar_fin[0], 0, &never, p.wait_limit);
+    }
+  } else if (warp == 2) {
+    // ------------------------------------------------------------ PV issuer -
+    if (lane == 0 && !skip) {
+      const uint32_t idesc_pv = idesc_bf16_f32(128, 128, 0);
+      const uint32_t v_base = smem_u32(sV);
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int t = 0; t < n && ok; ++t) {
+        if (!(ok = wait_bounded(&bar_p, t & 1, abort_flag, p.wait_limit))) break;
+        if (!(ok = wait_bounded(&bar_vfull[stage], phase, abort_flag, p.wait_limit))) break;
+        tc_fence_after();
+        const uint32_t v_addr = v_base + stage * L::STAGE;
 #pragma unroll
         for (int kk = 0; kk < BLK / 16; ++kk) {
           const uint64_t bd = sdesc_sw128(v_addr + (kk >> 2) * L::VPANEL + (kk & 3) * 32, 16, 1024);
-          mma_ts(o_tmem, s_tmem + kk * 8, bd, idesc_pv, (u > 0 || kk > 0) ? 1u : 0u);
+          mma_ts(tb + TM_O, tb + TM_P + kk * 8, bd, idesc_pv, (t > 0 || kk > 0) ? 1u : 0u);
         }
-        mma_commit(&bar_empty[stage0 + stage]);
-        mma_commit(&bar_o[x]);
-        advance();
-        return true;
-      };
-      if (ok) ok = issue_qk();
-      for (int u = 0; u < n_mine && ok; ++u) {
-        if (!(ok = issue_pv(u))) break;
-        if (u + 1 < n_mine) {
-          // S_x / P_x is reused for the next block once this PV has read P_x
-          if (!(ok = wait_bounded(&bar_o[x], u & 1, abort_flag, p.wait_limit))) break;
-          tc_fence_after();
-          if (!(ok = issue_qk())) break;
+        mma_commit(&bar_vempty[stage]);
+        mma_commit(&bar_o[t & 1]);
+        if (++stage == ATTN_VSTAGE) {
+          stage = 0;
+          phase ^= 1u;
         }
       }
-      // every MMA issued by this thread has completed once bar_fin flips
-      mma_commit(&bar_fin[x]);
+      mma_commit(&bar_fin[1]);
       int32_t never = 0;
-      wait_bounded(&bar_fin[x], 0, &never, p.wait_limit);
+      wait_bounded(&bar_fin[1], 0, &never, p.wait_limit);
     }
   } else {
     // ------------------------------------------------------------ softmax ---
-    const int x = (warp - 4) >> 2;              // pipeline: 0 = even kept blocks, 1 = odd kept blocks
+    const int x = (warp - 4) >> 2;              // 0 = even kept blocks, 1 = odd kept blocks
     const int wq = warp & 3;                    // tensor-memory lane quarter of this warp
     const int row = wq * 32 + lane;             // row of the Q tile
     const uint32_t lane_base = tb + (static_cast<uint32_t>(wq * 32) << 16);
-    const uint32_t s_col = tm_s(x), o_col = tm_o(x);
+    const uint32_t s_col = tm_s(x);
     const int q_tok = i * BLK + row;
     const bool row_out = row < BLK && q_tok < p.Lc;
     const float c_log2 = p.scale_log2;
     const uint64_t c2 = f2_pack(c_log2, c_log2);
-    float m_run = -INFINITY, l_run = 0.f;
     // tcgen05.ld / st are warp-collective: every wait result is made warp-uniform
     auto wwait = [&](uint64_t *bar, uint32_t parity) {
       return __all_sync(0xffffffffu, wait_bounded(bar, parity, abort_flag, p.wait_limit));
     };
     bool ok = !skip;
+    if (ok) {
+      // Q row -> tensor memory: this warpgroup copies channels [64x, 64x + 64)
+      // (32 columns of packed bf16 pairs, the A-operand layout of the QK MMA);
+      // rows past the q-block or past Lc are zero
+      uint32_t qw[32];
+      if (row_out) {
+        const uint4 *src = reinterpret_cast<const uint4 *>(
+            p.q + ((static_cast<size_t>(b) * p.Lc + q_tok) * p.H + h) * 128 + x * 64);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const uint4 v = __ldg(src + e);
+          qw[4 * e] = v.x;
+          qw[4 * e + 1] = v.y;
+          qw[4 * e + 2] = v.z;
+          qw[4 * e + 3] = v.w;
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) qw[e] = 0u;
+      }
+      tmem_st32(lane_base + TM_Q + 32 * x, qw);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&bar_q);
+    }
+    float m_run = -INFINITY;   // reference max this warpgroup last saw
+    float l_run = 0.f;         // this warpgroup's partial row sum, relative to m_run
     const int n_mine = skip ? 0 : (n - x + 1) / 2;   // kept blocks of this warpgroup
     for (int u = 0; u < n_mine && ok; ++u) {
       const int t = x + 2 * u;
@@ -314,121 +336,102 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
       int krow, valid;
       kv_block_coords(jb, start, p.W, p.nb, p.lslot, BLK, p.Lc, krow, valid);
       if (!(ok = wwait(&bar_s[x], u & 1))) break;
-      // turn: block t - 1 (the other warpgroup) has finished its exponentials
-      if (x == 0 && u > 0) {
-        if (!(ok = wwait(&bar_turn[1], (u - 1) & 1))) break;
-      } else if (x == 1) {
-        if (!(ok = wwait(&bar_turn[0], u & 1))) break;
-      }
       tc_fence_after();
       const bool full = valid == BLK;
-      const uint64_t negm_run2 = f2_pack(-m_run, -m_run);
-      uint32_t pk[BLK / 2];
-      uint64_t acc2[4] = {0, 0, 0, 0};
-      float m_use = m_run;
-      float mx = -INFINITY;
-      bool done = false;
-      if (full && u > 0) {
-        // common case: exponentials against the running (possibly stale)
-        // max, with the block max computed in the same pass -- the max
-        // instructions hide under the SFU-bound exponentials.  Kept unless a
-        // row's block max exceeds the reference by more than 2^8.
-        uint32_t s[BLK];
+      uint32_t s[BLK];
 #pragma unroll
-        for (int c = 0; c < BLK / 32; ++c)
-          tmem_ld32(lane_base + s_col + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&s[32 * c]));
-        tmem_wait_ld();
+      for (int c = 0; c < BLK / 32; ++c)
+        tmem_ld32(lane_base + s_col + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&s[32 * c]));
+      tmem_wait_ld();
+      // block max over the block's true tokens
+      float mx;
+      {
         float a[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) a[e] = -INFINITY;
+        if (full) {
+#pragma unroll
+          for (int c = 0; c < BLK; c += 16)
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              a[e] = max3f(a[e], __uint_as_float(s[c + 2 * e]), __uint_as_float(s[c + 2 * e + 1]));
+        } else {
+#pragma unroll
+          for (int c = 0; c < BLK; ++c)
+            if (c < valid) a[c & 7] = fmaxf(a[c & 7], __uint_as_float(s[c]));
+        }
+        mx = max3f(max3f(a[0], a[1], a[2]), max3f(a[3], a[4], a[5]), fmaxf(a[6], a[7]));
+      }
+      // block t - 1 (the other warpgroup) has settled the reference max:
+      // adopt it, bringing this warpgroup's partial sum to the same reference
+      if (t > 0) {
+        if (!(ok = wwait(&bar_turn[x ^ 1], x == 0 ? ((u - 1) & 1) : (u & 1)))) break;
+        const float m_ref = s_mref[row];
+        if (m_ref != m_run) {
+          l_run *= ex2_approx(m_run - m_ref);
+          m_run = m_ref;
+        }
+      }
+      // raise the reference only when the block max exceeds it by more than 2^8
+      bool o_ready = false;    // PV_{t-1} known to have completed
+      const float m_new = fmaxf(m_run, mx * c_log2);
+      if (__any_sync(0xffffffffu, m_new > m_run + ATTN_RESCALE_LOG2)) {
+        const float factor = ex2_approx(m_run - m_new);
+        l_run *= factor;
+        if (t > 0) {
+          // O holds PV_0 .. PV_{t-1}: wait for the last of them, then rescale
+          if (!(ok = wwait(&bar_o[(t - 1) & 1], ((t - 1) >> 1) & 1))) break;
+          o_ready = true;
+          tc_fence_after();
+          const uint64_t f2 = f2_pack(factor, factor);
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c) {
+            uint32_t o[32];
+            tmem_ld32(lane_base + TM_O + 32 * c, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              float lo, hi;
+              f2_unpack(f2_mul(f2_pack(__uint_as_float(o[2 * e]), __uint_as_float(o[2 * e + 1])), f2), lo, hi);
+              o[2 * e] = __float_as_uint(lo);
+              o[2 * e + 1] = __float_as_uint(hi);
+            }
+            tmem_st32(lane_base + TM_O + 32 * c, o);
+          }
+          tmem_wait_st();
+        }
+        m_run = m_new;
+      }
+      // publish the reference for block t + 1, hand over the turn and release
+      // S buffer t mod 2 (held in registers from here on)
+      s_mref[row] = m_run;
+      tc_fence_before();
+      mbar_arrive(&bar_turn[x]);
+      mbar_arrive(&bar_sfree[x]);
+      // P = exp2(s * c - m): full-block and masked (partial last block of a
+      // chunk) cases are separate loops: a per-element mask test inside the
+      // unrolled loop costs two ALU instructions per element
+      const uint64_t negm2 = f2_pack(-m_run, -m_run);
+      uint32_t pk[BLK / 2];
+      uint64_t acc2[4] = {0, 0, 0, 0};
+      if (full) {
 #pragma unroll
         for (int c = 0; c < BLK / 2; ++c) {
-          const float s0 = __uint_as_float(s[2 * c]), s1 = __uint_as_float(s[2 * c + 1]);
-          a[c & 7] = max3f(a[c & 7], s0, s1);
           float x0, x1;
-          f2_unpack(f2_fma(f2_pack(s0, s1), c2, negm_run2), x0, x1);
+          f2_unpack(f2_fma(f2_pack(__uint_as_float(s[2 * c]), __uint_as_float(s[2 * c + 1])), c2, negm2), x0, x1);
           const float e0 = ex2_approx(x0), e1 = ex2_approx(x1);
           acc2[c & 3] = f2_add(acc2[c & 3], f2_pack(e0, e1));
           pk[c] = pack_bf16x2(e0, e1);
         }
-        mx = max3f(max3f(a[0], a[1], a[2]), max3f(a[3], a[4], a[5]), fmaxf(a[6], a[7]));
-        done = !__any_sync(0xffffffffu, mx * c_log2 > m_run + ATTN_RESCALE_LOG2);
-      }
-      if (!done) {
-        // S is still intact in tensor memory: P is stored only below
-        uint32_t s[BLK];
+      } else {
 #pragma unroll
-        for (int c = 0; c < BLK / 32; ++c)
-          tmem_ld32(lane_base + s_col + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&s[32 * c]));
-        tmem_wait_ld();
-        if (!(full && u > 0)) {
-          // first block of the row or a partial block: the max first
-          float a[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) a[e] = -INFINITY;
-          if (full) {
-#pragma unroll
-            for (int c = 0; c < BLK; c += 16)
-#pragma unroll
-              for (int e = 0; e < 8; ++e)
-                a[e] = max3f(a[e], __uint_as_float(s[c + 2 * e]), __uint_as_float(s[c + 2 * e + 1]));
-          } else {
-#pragma unroll
-            for (int c = 0; c < BLK; ++c)
-              if (c < valid) a[c & 7] = fmaxf(a[c & 7], __uint_as_float(s[c]));
-          }
-          mx = max3f(max3f(a[0], a[1], a[2]), max3f(a[3], a[4], a[5]), fmaxf(a[6], a[7]));
-        }
-        const float m_new = fmaxf(m_run, mx * c_log2);
-        const bool need = m_new > m_run + ATTN_RESCALE_LOG2;
-        if (__any_sync(0xffffffffu, need)) {
-          m_use = m_new;
-          const float factor = ex2_approx(m_run - m_new);
-          l_run *= factor;
-          if (u > 0) {
-            // PV_{t-2} into O_x completed before S_x for block t was computed
-            const uint64_t f2 = f2_pack(factor, factor);
-#pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
-              uint32_t o[32];
-              tmem_ld32(lane_base + o_col + 32 * c, o);
-              tmem_wait_ld();
-#pragma unroll
-              for (int e = 0; e < 16; ++e) {
-                float lo, hi;
-                f2_unpack(f2_mul(f2_pack(__uint_as_float(o[2 * e]), __uint_as_float(o[2 * e + 1])), f2), lo, hi);
-                o[2 * e] = __float_as_uint(lo);
-                o[2 * e + 1] = __float_as_uint(hi);
-              }
-              tmem_st32(lane_base + o_col + 32 * c, o);
-            }
-          }
-        }
-        // P = exp2(s * c - m): full-block and masked (partial last block of a
-        // chunk) cases are separate loops: a per-element mask test inside the
-        // unrolled loop costs two ALU instructions per element
-        const uint64_t negm2 = f2_pack(-m_use, -m_use);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) acc2[e] = 0;
-        if (full) {
-#pragma unroll
-          for (int c = 0; c < BLK / 2; ++c) {
-            float x0, x1;
-            f2_unpack(f2_fma(f2_pack(__uint_as_float(s[2 * c]), __uint_as_float(s[2 * c + 1])), c2, negm2), x0, x1);
-            const float e0 = ex2_approx(x0), e1 = ex2_approx(x1);
-            acc2[c & 3] = f2_add(acc2[c & 3], f2_pack(e0, e1));
-            pk[c] = pack_bf16x2(e0, e1);
-          }
-        } else {
-#pragma unroll
-          for (int c = 0; c < BLK / 2; ++c) {
-            float x0, x1;
-            f2_unpack(f2_fma(f2_pack(__uint_as_float(s[2 * c]), __uint_as_float(s[2 * c + 1])), c2, negm2), x0, x1);
-            const float e0 = 2 * c < valid ? ex2_approx(x0) : 0.f;
-            const float e1 = 2 * c + 1 < valid ? ex2_approx(x1) : 0.f;
-            acc2[c & 3] = f2_add(acc2[c & 3], f2_pack(e0, e1));
-            pk[c] = pack_bf16x2(e0, e1);
-          }
+        for (int c = 0; c < BLK / 2; ++c) {
+          float x0, x1;
+          f2_unpack(f2_fma(f2_pack(__uint_as_float(s[2 * c]), __uint_as_float(s[2 * c + 1])), c2, negm2), x0, x1);
+          const float e0 = 2 * c < valid ? ex2_approx(x0) : 0.f;
+          const float e1 = 2 * c + 1 < valid ? ex2_approx(x1) : 0.f;
+          acc2[c & 3] = f2_add(acc2[c & 3], f2_pack(e0, e1));
+          pk[c] = pack_bf16x2(e0, e1);
         }
       }
       {
@@ -436,79 +439,56 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
         f2_unpack(f2_add(f2_add(acc2[0], acc2[1]), f2_add(acc2[2], acc2[3])), a0, a1);
         l_run += a0 + a1;
       }
-      m_run = m_use;
-      mbar_arrive(&bar_turn[x]);
+      // P's columns are free once PV_{t-1} has read them
+      if (t > 0 && !o_ready) {
+        if (!(ok = wwait(&bar_o[(t - 1) & 1], ((t - 1) >> 1) & 1))) break;
+        tc_fence_after();
+      }
 #pragma unroll
       for (int c = 0; c < BLK / 64; ++c)
-        tmem_st32(lane_base + s_col + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&pk[32 * c]));
+        tmem_st32(lane_base + TM_P + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&pk[32 * c]));
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&bar_p[x]);
+      mbar_arrive(&bar_p);
     }
     // ---------------------------------------------------------- epilogue ----
-    // merge the two pipelines: (m_x, l_x, O_x) -> O, LSE.  Each warpgroup waits
-    // for its own pipeline's last PV only (the other pipeline may lag by any
-    // number of blocks), then publishes (m, l) in its pipeline's first ring
-    // stage, idle once that last PV has completed; bar_l orders both.
+    // Every PV has completed once PV_{n-1} has (one issuing thread, completions
+    // in order), and every QK before it.  The rings are idle then: the first K
+    // stage carries the (m, l) exchange, the first V stage the bf16 O tile for
+    // the TMA store.
     const int n0 = skip ? 0 : (n + 1) / 2, n1 = skip ? 0 : n / 2;
-    const int n_x = x == 0 ? n0 : n1;
-    float *s_ml_mine = reinterpret_cast<float *>(sKV + x * ATTN_PSTAGE * L::STAGE);
-    float *s_ml_other = reinterpret_cast<float *>(sKV + (x ^ 1) * ATTN_PSTAGE * L::STAGE);
-    if (ok && !skip && n_x > 0) ok = wwait(&bar_o[x], (n_x - 1) & 1);
-    // this warpgroup writes output columns [64x, 64x + 64): its own pipeline's
-    // part of them is final already, the other pipeline's after bar_l
-    uint32_t own[64];
-    if (ok && !skip && n_x > 0) {
-      tc_fence_after();
-      tmem_ld32(lane_base + tm_o(x) + x * 64, *reinterpret_cast<uint32_t(*)[32]>(&own[0]));
-      tmem_ld32(lane_base + tm_o(x) + x * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&own[32]));
-      tmem_wait_ld();
-    }
+    float *s_ml = reinterpret_cast<float *>(sK);
+    uint8_t *s_out = sV;
+    if (ok && !skip) ok = wwait(&bar_o[(n - 1) & 1], ((n - 1) >> 1) & 1);
     if (ok && !skip) {
-      s_ml_mine[row] = m_run;
-      s_ml_mine[128 + row] = l_run;
-      tc_fence_before();
+      s_ml[x * 256 + row] = m_run;
+      s_ml[x * 256 + 128 + row] = l_run;
       mbar_arrive(&bar_l);
       ok = wwait(&bar_l, 0);
     }
-    const float *s_ml0 = x == 0 ? s_ml_mine : s_ml_other;
-    const float *s_ml1 = x == 0 ? s_ml_other : s_ml_mine;
     if (ok && !skip) {
       tc_fence_after();
-      const float m0 = s_ml0[row], m1 = s_ml1[row];
-      const float l0 = s_ml0[128 + row], l1 = s_ml1[128 + row];
-      const float m = fmaxf(m0, m1);
-      const float a0 = n0 > 0 ? ex2_approx(m0 - m) : 0.f;
-      const float a1 = n1 > 0 ? ex2_approx(m1 - m) : 0.f;
-      const float l_tot = l0 * a0 + l1 * a1;
+      const float m0 = s_ml[row], m1 = s_ml[256 + row];
+      const float l0 = s_ml[128 + row], l1 = s_ml[384 + row];
+      // the reference max only grows, so O is relative to the larger one
+      const float m = n1 > 0 ? fmaxf(m0, m1) : m0;
+      float l_tot = n0 > 0 ? l0 * ex2_approx(m0 - m) : 0.f;
+      if (n1 > 0) l_tot += l1 * ex2_approx(m1 - m);
       const float inv_l = 1.f / l_tot;
-      const float w_own = (x == 0 ? a0 : a1) * inv_l, w_oth = (x == 0 ? a1 : a0) * inv_l;
-      const int n_oth = x == 0 ? n1 : n0;
-      uint32_t oth[64];
-      if (n_oth > 0) {
-        tmem_ld32(lane_base + tm_o(x ^ 1) + x * 64, *reinterpret_cast<uint32_t(*)[32]>(&oth[0]));
-        tmem_ld32(lane_base + tm_o(x ^ 1) + x * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&oth[32]));
-        tmem_wait_ld();
-      }
-      // stage the bf16 row half in the (now idle) Q tile, 128-byte swizzled
-      // like a TMA tile: 16-byte chunk c of row r sits at chunk c ^ (r mod 8)
-      uint8_t *panel = sQ + x * (L::Q_BYTES / 2) + row * 128;
+      uint32_t o[64];
+      tmem_ld32(lane_base + TM_O + x * 64, *reinterpret_cast<uint32_t(*)[32]>(&o[0]));
+      tmem_ld32(lane_base + TM_O + x * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&o[32]));
+      tmem_wait_ld();
+      // stage this warpgroup's 64-column half of the bf16 row, 128-byte
+      // swizzled like a TMA tile: 16-byte chunk c of row r at chunk c ^ (r mod 8)
+      uint8_t *panel = s_out + x * (128 * 128) + row * 128;
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
         uint32_t w[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int k0 = 8 * c + 2 * e;
-          float v0 = 0.f, v1 = 0.f;
-          if (n_x > 0) {
-            v0 = __uint_as_float(own[k0]) * w_own;
-            v1 = __uint_as_float(own[k0 + 1]) * w_own;
-          }
-          if (n_oth > 0) {
-            v0 = fmaf(__uint_as_float(oth[k0]), w_oth, v0);
-            v1 = fmaf(__uint_as_float(oth[k0 + 1]), w_oth, v1);
-          }
-          w[e] = pack_bf16x2(v0, v1);
+          w[e] = pack_bf16x2(__uint_as_float(o[k0]) * inv_l, __uint_as_float(o[k0 + 1]) * inv_l);
         }
         *reinterpret_cast<uint4 *>(panel + ((c ^ (row & 7)) * 16)) = make_uint4(w[0], w[1], w[2], w[3]);
       }
@@ -520,7 +500,7 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
       if (ok && threadIdx.x == (4 + 4 * x) * 32) {
         // one TMA store of this warpgroup's 64-column panel; rows past the
         // q-block or past Lc are not written
-        tma_store_4d(&tmO, sQ + x * (L::Q_BYTES / 2), x * 64, h, i * BLK, b);
+        tma_store_4d(&tmO, s_out + x * (128 * 128), x * 64, h, i * BLK, b);
         bulk_commit();
         bulk_wait_read();
       }
@@ -535,7 +515,7 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 2) {
+  if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tb, 512);
   }

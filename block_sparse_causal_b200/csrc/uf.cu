@@ -300,15 +300,14 @@ int32_t uf_block_sparse_attn(const void *q, int32_t H, const uf_kv_cache *c, con
   if (items >= (1LL << 31)) return UF_EINVAL;
 
   const int32_t lslot = nb * c->blk;
-  CUtensorMap tq, tk, tv, to;
+  CUtensorMap tk, tv, to;
   {
+    // O: [B, Lc, H, D] as {channels, heads, tokens, batch}; one q-block
+    // (blk rows) of one head per 64-channel store
     const cuuint64_t dims[4] = {128, static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(c->Lc),
                                 static_cast<cuuint64_t>(c->B)};
     // byte strides of dims 1..3 (head, token, batch)
     const cuuint64_t strides[3] = {256, static_cast<cuuint64_t>(H) * 256, static_cast<cuuint64_t>(c->Lc) * H * 256};
-    const cuuint32_t box[4] = {64, 1, 128, 1};
-    if (!make_map(&tq, q, 4, dims, strides, box)) return UF_ECUDA;
-    // O: same layout as Q; one q-block (blk rows) per store
     const cuuint32_t obox[4] = {64, 1, static_cast<cuuint32_t>(c->blk), 1};
     if (!make_map(&to, o, 4, dims, strides, obox)) return UF_ECUDA;
   }
@@ -331,6 +330,7 @@ int32_t uf_block_sparse_attn(const void *q, int32_t H, const uf_kv_cache *c, con
   p.meta = c->meta;
   p.idx = idx;
   p.cnt = cnt;
+  p.q = static_cast<const __nv_bfloat16 *>(q);
   p.o = static_cast<__nv_bfloat16 *>(o);
   p.lse = lse;
   p.H = H;
@@ -348,12 +348,12 @@ int32_t uf_block_sparse_attn(const void *q, int32_t H, const uf_kv_cache *c, con
     constexpr int smem = uf::AttnSmem<128>::DYN;
     const int32_t e = ensure_smem(uf::attn_kernel<128>, smem, g_attn128_smem);
     if (e != UF_OK) return e;
-    uf::attn_kernel<128><<<static_cast<unsigned>(items), uf::ATTN_THREADS, smem, st>>>(tq, tk, tv, to, p);
+    uf::attn_kernel<128><<<static_cast<unsigned>(items), uf::ATTN_THREADS, smem, st>>>(tk, tv, to, p);
   } else {
     constexpr int smem = uf::AttnSmem<64>::DYN;
     const int32_t e = ensure_smem(uf::attn_kernel<64>, smem, g_attn64_smem);
     if (e != UF_OK) return e;
-    uf::attn_kernel<64><<<static_cast<unsigned>(items), uf::ATTN_THREADS, smem, st>>>(tq, tk, tv, to, p);
+    uf::attn_kernel<64><<<static_cast<unsigned>(items), uf::ATTN_THREADS, smem, st>>>(tk, tv, to, p);
   }
   return launch_status();
 }
