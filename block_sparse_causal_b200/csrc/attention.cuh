@@ -63,6 +63,7 @@ struct AttnParams {
   float *lse;                // [B, H, Lc] or NULL
   __nv_bfloat16 *o;          // [B, Lc, H, D] (skipped items are written directly)
   int32_t H, G, W, Lc, nb, lslot, k;
+  uint32_t nb_mul;           // floor(2^32 / nb) (2^32 - 1 for nb = 1): j / nb without a divide
   float scale_log2;          // softmax scale * log2(e)
   long long wait_limit;
 };
@@ -76,12 +77,21 @@ struct AttnSmem {
 };
 static_assert(AttnSmem<128>::STAGE >= 2 * 128 * 128, "the epilogue stages a 128x128 bf16 O tile in one stage");
 
-// Logical kv block j of the window -> first row of its tile in the cache and
-// its number of true tokens.
-__device__ __forceinline__ void kv_block_coords(int j, int start, int W, int nb, int lslot, int blk, int Lc,
-                                                int &row, int &valid) {
-  const int c = j / nb, r = j - c * nb;
-  const int slot = (start + c) % W;
+// Logical kv block j (0 <= j < n_valid * nb) of the window -> first row of its
+// tile in the cache and its number of true tokens.  Chunk c = j / nb comes
+// from a multiply-high by floor(2^32 / nb), which is at most one below the
+// quotient, and one correction step; the ring slot start + c (both below W)
+// wraps with one subtraction.  No divide instruction on the per-block path.
+__device__ __forceinline__ void kv_block_coords(int j, int start, int W, int nb, uint32_t nb_mul, int lslot,
+                                                int blk, int Lc, int &row, int &valid) {
+  int c = static_cast<int>(__umulhi(static_cast<uint32_t>(j), nb_mul));
+  int r = j - c * nb;
+  if (r >= nb) {
+    ++c;
+    r -= nb;
+  }
+  int slot = start + c;
+  if (slot >= W) slot -= W;
   row = slot * lslot + r * blk;
   valid = (r == nb - 1) ? (Lc - (nb - 1) * blk) : blk;
 }
@@ -182,7 +192,7 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
           jb = diag;
         }
         int row, valid;
-        kv_block_coords(jb, start, p.W, p.nb, p.lslot, BLK, p.Lc, row, valid);
+        kv_block_coords(jb, start, p.W, p.nb, p.nb_mul, p.lslot, BLK, p.Lc, row, valid);
         uint64_t *full = &full_bars[stage];
         mbar_arrive_expect_tx(full, L::STAGE);
         uint8_t *dst = ring + stage * L::STAGE;
@@ -334,7 +344,7 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
       int jb = row_idx ? __ldg(row_idx + t) : t;
       if (jb < 0 || jb >= NKV) jb = diag;
       int krow, valid;
-      kv_block_coords(jb, start, p.W, p.nb, p.lslot, BLK, p.Lc, krow, valid);
+      kv_block_coords(jb, start, p.W, p.nb, p.nb_mul, p.lslot, BLK, p.Lc, krow, valid);
       if (!(ok = wwait(&bar_s[x], u & 1))) break;
       tc_fence_after();
       const bool full = valid == BLK;

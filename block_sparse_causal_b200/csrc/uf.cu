@@ -340,6 +340,7 @@ int32_t uf_block_sparse_attn(const void *q, int32_t H, const uf_kv_cache *c, con
   p.nb = nb;
   p.lslot = lslot;
   p.k = k;
+  p.nb_mul = nb == 1 ? 0xFFFFFFFFu : static_cast<uint32_t>((1ULL << 32) / static_cast<uint64_t>(nb));
   p.scale_log2 = scale * 1.4426950408889634f;
   p.wait_limit = g_wait_limit.load();
   cudaGetLastError();
