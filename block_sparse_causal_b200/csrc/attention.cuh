@@ -5,31 +5,39 @@
 // blog), Sec. 3.3: no token mask inside the window (causality by processing
 // order); Eq. 4: grouped-query KV heads.
 //
-// One thread block = one work item (batch b, query head h, q-block i): a
-// 128-row Q tile against the item's list of n kept kv blocks t = 0 .. n-1,
-// accumulated into one O tile with an online softmax.  Both products run on
-// the tensor core with the A operand in tensor memory and a K-major B operand
-// in shared memory:
-//   S_t = Q K_t^T   (Q copied into tensor memory once per item)
+// Work item = (batch b, query head h, q-block i): a 128-row Q tile against
+// the item's list of n kept kv blocks t = 0 .. n-1, accumulated into one O
+// tile with an online softmax.  The grid is persistent: thread block c takes
+// items c, c + grid, c + 2 grid, ..., and every pipeline below runs on across
+// item boundaries, so the next item's Q and K / V tiles load, and its first
+// QK products run, while the current item finishes.
+//
+// Both products run on the tensor core with the A operand in tensor memory
+// and a K-major B operand in shared memory:
+//   S_t = Q K_t^T   (Q staged by TMA in shared memory, copied into tensor
+//                    memory by the softmax threads once per item)
 //   O  += P_t V_t   (P_t written to tensor memory by the softmax; V is stored
 //                    transposed in the window, so V_t^T is K-major too)
 // Tensor memory (512 columns): S buffers 0 and 1 [0,128) [128,256), O
-// [256,384), Q [384,448), P [448,512).  Block t uses S buffer t mod 2, so
-// S_{t+1} is computed while the softmax works on S_t, and S_{t+2} is issued as
-// soon as the softmax has read S_t into registers (P has its own columns).
+// [256,384), Q [384,448), P [448,512).  Kept blocks are numbered across the
+// items of a thread block (g = blocks of earlier items + t); block g uses S
+// buffer g mod 2 and is handled by softmax warpgroup g mod 2.  S_{g+2} is
+// issued as soon as the softmax has read S_g into registers (P has its own
+// columns).
 // Twelve warps:
-//   warps 0, 3   TMA producers of the K ring and of the V ring: the tiles
-//                gathered by the block list, in block order;
+//   warps 0, 3   TMA producers of the K ring and of the V ring, in block
+//                order;
 //   warps 1, 2   one issuing thread each (an issuing thread waits for every
 //                MMA it issues to be accepted, so two of them keep the tensor
-//                core busy): warp 1 issues QK_{t+2} once S_t has been read and
-//                owns the tensor-memory allocation, warp 2 issues PV_t once
-//                P_t is in tensor memory;
-//   warps 4-7    softmax of the even-numbered kept blocks, warps 8-11 of the
-//                odd ones: each thread owns one row (32x32b loads), applies
-//                the block's token mask, computes exponentials in the exp2
-//                domain against a reference max and writes P as packed bf16.
-//                The reference max of each row lives in shared memory and is
+//                core busy): warp 1 issues the QK products, requests each
+//                item's Q tile as soon as the previous one has been copied
+//                into tensor memory, and owns the tensor-memory allocation;
+//                warp 2 issues the PV products;
+//   warps 4-7    softmax of the even-numbered blocks, warps 8-11 of the odd
+//                ones: each thread owns one row (32x32b loads), applies the
+//                block's token mask, computes exponentials in the exp2 domain
+//                against a reference max and writes P as packed bf16.  The
+//                reference max of each row lives in shared memory and is
 //                raised only when a block's max exceeds it by more than 2^8 (a
 //                stale max is exact: O and the sums share it); raising it
 //                rescales O in tensor memory.  Per block: S to registers, the
@@ -39,7 +47,8 @@
 //                run from registers, overlapping those of the other
 //                warpgroup's block.  Each warpgroup keeps its own partial row
 //                sum relative to the reference it last saw; the two are
-//                combined at the end.
+//                combined in the item's epilogue, which also hands O back to
+//                the PV issuer for the next item.
 #pragma once
 
 #include "uf_device.cuh"
@@ -48,20 +57,30 @@ namespace uf {
 
 constexpr int ATTN_THREADS = 384;
 constexpr int ATTN_SOFTMAX_THREADS = 256;
-constexpr int ATTN_KSTAGE = 4;                   // shared-memory stages of the K ring
+constexpr int ATTN_KSTAGE = 3;                   // shared-memory stages of the K ring
 constexpr int ATTN_VSTAGE = 3;                   // and of the V ring
 // tensor-memory columns
 __host__ __device__ constexpr uint32_t tm_s(int x) { return static_cast<uint32_t>(x) * 128u; }
 constexpr uint32_t TM_O = 256, TM_Q = 384, TM_P = 448;
 constexpr float ATTN_RESCALE_LOG2 = 8.0f;
+// Registers per thread: the block is launched with ATTN_LAUNCH_REGS (the
+// most 384 threads can have); the producer / issuer warpgroup then releases
+// registers to the two softmax warpgroups.  The budgets add up to the launch
+// allocation exactly (a raise beyond it would wait forever), and the host
+// refuses to launch a build whose kernel was compiled to another count.
+constexpr int ATTN_LAUNCH_REGS = 168;
+constexpr int ATTN_REGS_IO = 56;
+constexpr int ATTN_REGS_SOFTMAX = 224;
+static_assert(128 * ATTN_REGS_IO + 256 * ATTN_REGS_SOFTMAX == ATTN_THREADS * ATTN_LAUNCH_REGS,
+              "register budgets must add up to the launch allocation");
 
 struct AttnParams {
   const int32_t *meta;
   const int32_t *idx;        // [B, H, nb, k] or NULL (dense)
   const int32_t *cnt;        // [B, H, nb] or NULL
-  const __nv_bfloat16 *q;    // [B, Lc, H, D]
   float *lse;                // [B, H, Lc] or NULL
-  __nv_bfloat16 *o;          // [B, Lc, H, D] (skipped items are written directly)
+  __nv_bfloat16 *o;          // [B, Lc, H, D]
+  int32_t items;             // B * H * nb
   int32_t H, G, W, Lc, nb, lslot, k;
   uint32_t nb_mul;           // floor(2^32 / nb) (2^32 - 1 for nb = 1): j / nb without a divide
   float scale_log2;          // softmax scale * log2(e)
@@ -70,12 +89,12 @@ struct AttnParams {
 
 template <int BLK>
 struct AttnSmem {
+  static constexpr int Q_BYTES = 128 * 256;          // 128 rows x 128 channels, two 64-channel panels
   static constexpr int PANEL = BLK * 128;            // one 64-channel panel of a K tile
   static constexpr int VPANEL = 128 * 128;           // one 64-token panel of a V^T tile (128 channels)
   static constexpr int STAGE = BLK * 256;
-  static constexpr int DYN = 1024 + (ATTN_KSTAGE + ATTN_VSTAGE) * STAGE;
+  static constexpr int DYN = 1024 + Q_BYTES + (ATTN_KSTAGE + ATTN_VSTAGE) * STAGE;
 };
-static_assert(AttnSmem<128>::STAGE >= 2 * 128 * 128, "the epilogue stages a 128x128 bf16 O tile in one stage");
 
 // Logical kv block j (0 <= j < n_valid * nb) of the window -> first row of its
 // tile in the cache and its number of true tokens.  Chunk c = j / nb comes
@@ -96,51 +115,76 @@ __device__ __forceinline__ void kv_block_coords(int j, int start, int W, int nb,
   valid = (r == nb - 1) ? (Lc - (nb - 1) * blk) : blk;
 }
 
+// One work item as every role of the thread block sees it.
+struct AttnItem {
+  int i, h, b, g;             // q-block, query head, batch, kv head
+  int n;                      // kept kv blocks (< 1: nothing to compute)
+  int diag;                   // the q-block's own block in the newest chunk
+  const int32_t *row_idx;     // its block list, or NULL (dense: block t is t)
+};
+
+__device__ __forceinline__ AttnItem attn_item(const AttnParams &p, int item, int NKV, int n_valid) {
+  AttnItem it;
+  it.i = item % p.nb;
+  const int bh = item / p.nb;
+  it.h = bh % p.H;
+  it.b = bh / p.H;
+  it.g = it.h / (p.H / p.G);
+  it.diag = (n_valid - 1) * p.nb + it.i;
+  it.row_idx = p.idx ? p.idx + static_cast<size_t>(item) * p.k : nullptr;
+  it.n = NKV;
+  if (it.row_idx) {
+    it.n = p.cnt ? __ldg(p.cnt + item) : p.k;
+    if (it.n > p.k) it.n = -1;   // malformed row
+  }
+  if (NKV < 1) it.n = -1;
+  return it;
+}
+
+// Kept block t of an item -> logical kv block of the window; an out-of-range
+// entry reads the diagonal block instead (`bad` tells the producer to record
+// the error).
+__device__ __forceinline__ int attn_block(const AttnItem &it, int t, int NKV, bool &bad) {
+  const int jb = it.row_idx ? __ldg(it.row_idx + t) : t;
+  bad = jb < 0 || jb >= NKV;
+  return bad ? it.diag : jb;
+}
+
 template <int BLK>
 __global__ void __launch_bounds__(ATTN_THREADS, 1)
-    attn_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-                const __grid_constant__ CUtensorMap tmO, const AttnParams p) {
+    attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
   using L = AttnSmem<BLK>;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t *sK = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t *sQ = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t *sK = sQ + L::Q_BYTES;
   uint8_t *sV = sK + ATTN_KSTAGE * L::STAGE;
 
-  __shared__ uint64_t bar_q, bar_l, bar_p;
-  __shared__ uint64_t bar_fin[2];
+  // per-item barriers: Q landed in shared memory / free in tensor memory /
+  // copied into tensor memory; O read by the epilogue; (m, l) exchange
+  __shared__ uint64_t bar_qfull, bar_qtfree, bar_q, bar_ofree, bar_l;
+  // per-block barriers
   __shared__ uint64_t bar_kfull[ATTN_KSTAGE], bar_kempty[ATTN_KSTAGE];
   __shared__ uint64_t bar_vfull[ATTN_VSTAGE], bar_vempty[ATTN_VSTAGE];
-  __shared__ uint64_t bar_s[2], bar_sfree[2], bar_o[2], bar_turn[2], bar_st[2];
+  __shared__ uint64_t bar_s[2], bar_sfree[2], bar_o[2], bar_turn[2], bar_p;
+  __shared__ uint64_t bar_fin[2];
   __shared__ float s_mref[128];   // reference max of each row (exp2 domain), published block by block
+  __shared__ float s_l[2][128];   // epilogue: each warpgroup's partial row sums
   __shared__ uint32_t s_tbase;
   __shared__ int32_t s_abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int NQ = p.nb;
-  const int item = blockIdx.x;
-  const int i = item % NQ;
-  const int bh = item / NQ;
-  const int h = bh % p.H, b = bh / p.H;
-  const int g = h / (p.H / p.G);
-
   // window state (written by the append call earlier on the stream)
   const int start = __ldcg(p.meta + 0), n_valid = __ldcg(p.meta + 1);
   const bool bad_meta = start < 0 || start >= p.W || n_valid < 1 || n_valid > p.W;
   const int NKV = bad_meta ? 0 : n_valid * p.nb;
-  const int diag = (n_valid - 1) * p.nb + i;
-  const int32_t *row_idx = p.idx ? p.idx + static_cast<size_t>(item) * p.k : nullptr;
-  int n = NKV;
-  if (row_idx) {
-    n = p.cnt ? __ldg(p.cnt + item) : p.k;
-    if (n > p.k) n = -1;   // malformed row
-  }
-  const bool skip = bad_meta || n < 1;
 
   if (threadIdx.x == 0) {
+    mbar_init(&bar_qfull, 1);
+    mbar_init(&bar_qtfree, 1);
     mbar_init(&bar_q, ATTN_SOFTMAX_THREADS);
+    mbar_init(&bar_ofree, ATTN_SOFTMAX_THREADS);
     mbar_init(&bar_l, ATTN_SOFTMAX_THREADS);
-    mbar_init(&bar_p, ATTN_SOFTMAX_THREADS / 2);
-    mbar_init(&bar_fin[0], 1);
-    mbar_init(&bar_fin[1], 1);
     for (int s = 0; s < ATTN_KSTAGE; ++s) {
       mbar_init(&bar_kfull[s], 1);
       mbar_init(&bar_kempty[s], 1);
@@ -154,11 +198,12 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
       mbar_init(&bar_sfree[s], ATTN_SOFTMAX_THREADS / 2);
       mbar_init(&bar_o[s], 1);
       mbar_init(&bar_turn[s], ATTN_SOFTMAX_THREADS / 2);
-      mbar_init(&bar_st[s], ATTN_SOFTMAX_THREADS / 2);
+      mbar_init(&bar_fin[s], 1);
     }
+    mbar_init(&bar_p, ATTN_SOFTMAX_THREADS / 2);
     s_abort = 0;
     fence_mbar_init();
-    if (skip) record_error(UF_EBOUNDS);
+    if (bad_meta && blockIdx.x == 0) record_error(UF_EBOUNDS);
   }
   if (warp == 1) {
     tmem_alloc(&s_tbase, 512);
@@ -170,356 +215,429 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
   const uint32_t tb = s_tbase;
   volatile int32_t *abort_flag = &s_abort;
 
-  if (warp == 0 || warp == 3) {
-    // ------------------------------------------------------------ producers -
-    const bool is_v = warp == 3;
-    const int nst = is_v ? ATTN_VSTAGE : ATTN_KSTAGE;
-    uint64_t *full_bars = is_v ? bar_vfull : bar_kfull;
-    uint64_t *empty_bars = is_v ? bar_vempty : bar_kempty;
-    uint8_t *ring = is_v ? sV : sK;
-    if (lane == 0 && !skip) {
-      tma_prefetch_desc(is_v ? &tmV : &tmK);
-      const int zc = b * p.G + g;
-      int stage = 0;
-      uint32_t phase = 0;
-      int issued = 0;
-      bool ok = true;
-      for (int t = 0; t < n && ok; ++t) {
-        if (!(ok = wait_bounded(&empty_bars[stage], phase ^ 1u, abort_flag, p.wait_limit))) break;
-        int jb = row_idx ? __ldg(row_idx + t) : t;
-        if (jb < 0 || jb >= NKV) {
-          record_error(UF_EBOUNDS);
-          jb = diag;
-        }
-        int row, valid;
-        kv_block_coords(jb, start, p.W, p.nb, p.nb_mul, p.lslot, BLK, p.Lc, row, valid);
-        uint64_t *full = &full_bars[stage];
-        mbar_arrive_expect_tx(full, L::STAGE);
-        uint8_t *dst = ring + stage * L::STAGE;
-        if (is_v) {
-          // V^T tile: 128 channel rows x BLK tokens, in 64-token panels
-#pragma unroll
-          for (int pnl = 0; pnl < BLK / 64; ++pnl)
-            tma_load_3d(dst + pnl * L::VPANEL, &tmV, full, row + 64 * pnl, 0, zc);
-        } else {
-          // K tile: BLK token rows x 128 channels, in 64-channel panels
-          tma_load_3d(dst, &tmK, full, 0, row, zc);
-          tma_load_3d(dst + L::PANEL, &tmK, full, 64, row, zc);
-        }
-        ++issued;
-        if (++stage == nst) {
-          stage = 0;
-          phase ^= 1u;
-        }
-      }
-      if (!ok) {
-        // unwind: let every load still in flight land before the block exits
-        int s = stage;
-        uint32_t ph = phase;
-        for (int q = 0; q < nst && q < issued; ++q) {
-          if (--s < 0) {
-            s = nst - 1;
-            ph ^= 1u;
+  if (warp < 4) {
+    // producers and issuers need few registers: hand them to the softmax
+    warpgroup_reg_release<ATTN_REGS_IO>();
+    if (warp == 0 || warp == 3) {
+      // ------------------------------------------------------------ producers -
+      const bool is_v = warp == 3;
+      const int nst = is_v ? ATTN_VSTAGE : ATTN_KSTAGE;
+      uint64_t *full_bars = is_v ? bar_vfull : bar_kfull;
+      uint64_t *empty_bars = is_v ? bar_vempty : bar_kempty;
+      uint8_t *ring = is_v ? sV : sK;
+      if (lane == 0 && NKV > 0) {
+        tma_prefetch_desc(is_v ? &tmV : &tmK);
+        int stage = 0;
+        uint32_t phase = 0;
+        int issued = 0;
+        bool ok = true;
+        for (int item = blockIdx.x; item < p.items && ok; item += gridDim.x) {
+          const AttnItem it = attn_item(p, item, NKV, n_valid);
+          if (it.n < 1) continue;
+          const int zc = it.b * p.G + it.g;
+          for (int t = 0; t < it.n; ++t) {
+            if (!(ok = wait_bounded(&empty_bars[stage], phase ^ 1u, abort_flag, p.wait_limit))) break;
+            bool bad;
+            const int jb = attn_block(it, t, NKV, bad);
+            if (bad) record_error(UF_EBOUNDS);
+            int row, valid;
+            kv_block_coords(jb, start, p.W, p.nb, p.nb_mul, p.lslot, BLK, p.Lc, row, valid);
+            uint64_t *full = &full_bars[stage];
+            mbar_arrive_expect_tx(full, L::STAGE);
+            uint8_t *dst = ring + stage * L::STAGE;
+            if (is_v) {
+              // V^T tile: 128 channel rows x BLK tokens, in 64-token panels
+  #pragma unroll
+              for (int pnl = 0; pnl < BLK / 64; ++pnl)
+                tma_load_3d(dst + pnl * L::VPANEL, &tmV, full, row + 64 * pnl, 0, zc);
+            } else {
+              // K tile: BLK token rows x 128 channels, in 64-channel panels
+              tma_load_3d(dst, &tmK, full, 0, row, zc);
+              tma_load_3d(dst + L::PANEL, &tmK, full, 64, row, zc);
+            }
+            ++issued;
+            if (++stage == nst) {
+              stage = 0;
+              phase ^= 1u;
+            }
           }
+        }
+        if (!ok) {
+          // unwind: let every load still in flight land before the block exits
           int32_t never = 0;
-          wait_bounded(&full_bars[s], ph, &never, p.wait_limit);
+          int s = stage;
+          uint32_t ph = phase;
+          for (int q = 0; q < nst && q < issued; ++q) {
+            if (--s < 0) {
+              s = nst - 1;
+              ph ^= 1u;
+            }
+            wait_bounded(&full_bars[s], ph, &never, p.wait_limit);
+          }
         }
       }
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ QK issuer -
-    if (lane == 0 && !skip) {
-      const uint32_t idesc_qk = idesc_bf16_f32(128, BLK, 0);
-      const uint32_t k_base = smem_u32(sK);
-      int stage = 0;
-      uint32_t phase = 0;
-      auto issue_qk = [&](int t) -> bool {
-        if (!wait_bounded(&bar_kfull[stage], phase, abort_flag, p.wait_limit)) return false;
-        tc_fence_after();
-        const uint32_t k_addr = k_base + stage * L::STAGE;
-        const uint32_t s_tmem = tb + tm_s(t & 1);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t bd = sdesc_sw128(k_addr + (kk >> 2) * L::PANEL + (kk & 3) * 32, 16, 1024);
-          mma_ts(s_tmem, tb + TM_Q + kk * 8, bd, idesc_qk, kk > 0);
+    } else if (warp == 1) {
+      // ------------------------------------------------------------ QK issuer -
+      if (lane == 0 && NKV > 0) {
+        const uint32_t idesc_qk = idesc_bf16_f32(128, BLK, 0);
+        const uint32_t k_base = smem_u32(sK);
+        int stage = 0;
+        uint32_t phase = 0;
+        int uses[2] = {0, 0};   // QK products issued into each S buffer so far
+        int kq = 0, g0 = 0, q_loads = 0;
+        bool ok = true;
+        tma_prefetch_desc(&tmQ);
+        // Q tile of a live item -> shared memory (rows past Lc read as zero)
+        auto request_q = [&](const AttnItem &a) {
+          mbar_arrive_expect_tx(&bar_qfull, L::Q_BYTES);
+          tma_load_4d(sQ, &tmQ, &bar_qfull, 0, a.h, a.i * BLK, a.b);
+          tma_load_4d(sQ + L::Q_BYTES / 2, &tmQ, &bar_qfull, 64, a.h, a.i * BLK, a.b);
+          ++q_loads;
+        };
+        int item = blockIdx.x;
+        AttnItem it;
+        for (; item < p.items; item += gridDim.x) {
+          it = attn_item(p, item, NKV, n_valid);
+          if (it.n >= 1) break;
         }
-        mma_commit(&bar_kempty[stage]);
-        mma_commit(&bar_s[t & 1]);
-        if (++stage == ATTN_KSTAGE) {
-          stage = 0;
-          phase ^= 1u;
+        if (item < p.items) request_q(it);
+        while (item < p.items && ok) {
+          // the item's Q is in tensor memory, so the staging tile is free for
+          // the next live item's Q
+          if (!(ok = wait_bounded(&bar_q, kq & 1, abort_flag, p.wait_limit))) break;
+          tc_fence_after();
+          int item_next = item + gridDim.x;
+          AttnItem nxt;
+          for (; item_next < p.items; item_next += gridDim.x) {
+            nxt = attn_item(p, item_next, NKV, n_valid);
+            if (nxt.n >= 1) break;
+          }
+          if (item_next < p.items) request_q(nxt);
+          for (int t = 0; t < it.n; ++t) {
+            const int buf = (g0 + t) & 1;
+            // the buffer's previous block has been read by the softmax
+            if (uses[buf] > 0 && !(ok = wait_bounded(&bar_sfree[buf], (uses[buf] - 1) & 1, abort_flag, p.wait_limit)))
+              break;
+            if (!(ok = wait_bounded(&bar_kfull[stage], phase, abort_flag, p.wait_limit))) break;
+            tc_fence_after();
+            const uint32_t k_addr = k_base + stage * L::STAGE;
+  #pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+              const uint64_t bd = sdesc_sw128(k_addr + (kk >> 2) * L::PANEL + (kk & 3) * 32, 16, 1024);
+              mma_ts(tb + tm_s(buf), tb + TM_Q + kk * 8, bd, idesc_qk, kk > 0);
+            }
+            mma_commit(&bar_kempty[stage]);
+            mma_commit(&bar_s[buf]);
+            ++uses[buf];
+            if (++stage == ATTN_KSTAGE) {
+              stage = 0;
+              phase ^= 1u;
+            }
+          }
+          if (!ok) break;
+          // Q's columns are free once every QK product of the item has completed
+          mma_commit(&bar_qtfree);
+          g0 += it.n;
+          ++kq;
+          item = item_next;
+          it = nxt;
         }
-        return true;
-      };
-      bool ok = wait_bounded(&bar_q, 0, abort_flag, p.wait_limit);
-      if (ok) tc_fence_after();
-      if (ok) ok = issue_qk(0);
-      if (ok && n > 1) ok = issue_qk(1);
-      for (int t = 0; t + 2 < n && ok; ++t) {
-        // S buffer t mod 2 is free once the softmax has read S_t
-        if (!(ok = wait_bounded(&bar_sfree[t & 1], (t >> 1) & 1, abort_flag, p.wait_limit))) break;
-        tc_fence_after();
-        ok = issue_qk(t + 2);
+        // every MMA issued by this thread has completed once bar_fin flips, and
+        // a Q tile still in flight has landed (the next is requested only after
+        // the previous one was copied out, so at most one)
+        mma_commit(&bar_fin[0]);
+        int32_t never = 0;
+        wait_bounded(&bar_fin[0], 0, &never, p.wait_limit);
+        if (!ok && q_loads > 0) wait_bounded(&bar_qfull, (q_loads - 1) & 1, &never, p.wait_limit);
       }
-      // every MMA issued by this thread has completed once bar_fin flips
-      mma_commit(&bar_fin[0]);
-      int32_t never = 0;
-      wait_bounded(&bar_fin[0], 0, &never, p.wait_limit);
-    }
-  } else if (warp == 2) {
-    // ------------------------------------------------------------ PV issuer -
-    if (lane == 0 && !skip) {
-      const uint32_t idesc_pv = idesc_bf16_f32(128, 128, 0);
-      const uint32_t v_base = smem_u32(sV);
-      int stage = 0;
-      uint32_t phase = 0;
-      bool ok = true;
-      for (int t = 0; t < n && ok; ++t) {
-        if (!(ok = wait_bounded(&bar_p, t & 1, abort_flag, p.wait_limit))) break;
-        if (!(ok = wait_bounded(&bar_vfull[stage], phase, abort_flag, p.wait_limit))) break;
-        tc_fence_after();
-        const uint32_t v_addr = v_base + stage * L::STAGE;
-#pragma unroll
-        for (int kk = 0; kk < BLK / 16; ++kk) {
-          const uint64_t bd = sdesc_sw128(v_addr + (kk >> 2) * L::VPANEL + (kk & 3) * 32, 16, 1024);
-          mma_ts(tb + TM_O, tb + TM_P + kk * 8, bd, idesc_pv, (t > 0 || kk > 0) ? 1u : 0u);
+    } else {
+      // ------------------------------------------------------------ PV issuer -
+      if (lane == 0 && NKV > 0) {
+        const uint32_t idesc_pv = idesc_bf16_f32(128, 128, 0);
+        const uint32_t v_base = smem_u32(sV);
+        int stage = 0;
+        uint32_t phase = 0;
+        int kq = 0, g0 = 0;
+        bool ok = true;
+        for (int item = blockIdx.x; item < p.items && ok; item += gridDim.x) {
+          const AttnItem it = attn_item(p, item, NKV, n_valid);
+          if (it.n < 1) continue;
+          // the previous item's epilogue has read O
+          if (kq > 0 && !(ok = wait_bounded(&bar_ofree, (kq - 1) & 1, abort_flag, p.wait_limit))) break;
+          for (int t = 0; t < it.n; ++t) {
+            const int gb = g0 + t;
+            if (!(ok = wait_bounded(&bar_p, gb & 1, abort_flag, p.wait_limit))) break;
+            if (!(ok = wait_bounded(&bar_vfull[stage], phase, abort_flag, p.wait_limit))) break;
+            tc_fence_after();
+            const uint32_t v_addr = v_base + stage * L::STAGE;
+  #pragma unroll
+            for (int kk = 0; kk < BLK / 16; ++kk) {
+              const uint64_t bd = sdesc_sw128(v_addr + (kk >> 2) * L::VPANEL + (kk & 3) * 32, 16, 1024);
+              mma_ts(tb + TM_O, tb + TM_P + kk * 8, bd, idesc_pv, (t > 0 || kk > 0) ? 1u : 0u);
+            }
+            mma_commit(&bar_vempty[stage]);
+            mma_commit(&bar_o[gb & 1]);
+            if (++stage == ATTN_VSTAGE) {
+              stage = 0;
+              phase ^= 1u;
+            }
+          }
+          g0 += it.n;
+          ++kq;
         }
-        mma_commit(&bar_vempty[stage]);
-        mma_commit(&bar_o[t & 1]);
-        if (++stage == ATTN_VSTAGE) {
-          stage = 0;
-          phase ^= 1u;
-        }
+        mma_commit(&bar_fin[1]);
+        int32_t never = 0;
+        wait_bounded(&bar_fin[1], 0, &never, p.wait_limit);
       }
-      mma_commit(&bar_fin[1]);
-      int32_t never = 0;
-      wait_bounded(&bar_fin[1], 0, &never, p.wait_limit);
     }
   } else {
+    warpgroup_reg_raise<ATTN_REGS_SOFTMAX>();
     // ------------------------------------------------------------ softmax ---
-    const int x = (warp - 4) >> 2;              // 0 = even kept blocks, 1 = odd kept blocks
+    const int x = (warp - 4) >> 2;              // handles blocks g with g mod 2 == x
     const int wq = warp & 3;                    // tensor-memory lane quarter of this warp
     const int row = wq * 32 + lane;             // row of the Q tile
     const uint32_t lane_base = tb + (static_cast<uint32_t>(wq * 32) << 16);
     const uint32_t s_col = tm_s(x);
-    const int q_tok = i * BLK + row;
-    const bool row_out = row < BLK && q_tok < p.Lc;
     const float c_log2 = p.scale_log2;
     const uint64_t c2 = f2_pack(c_log2, c_log2);
     // tcgen05.ld / st are warp-collective: every wait result is made warp-uniform
     auto wwait = [&](uint64_t *bar, uint32_t parity) {
       return __all_sync(0xffffffffu, wait_bounded(bar, parity, abort_flag, p.wait_limit));
     };
-    bool ok = !skip;
-    if (ok) {
-      // Q row -> tensor memory: this warpgroup copies channels [64x, 64x + 64)
-      // (32 columns of packed bf16 pairs, the A-operand layout of the QK MMA);
-      // rows past the q-block or past Lc are zero
+    // an item with nothing to compute: zero output, -inf log-sum-exp
+    auto write_empty = [&](const AttnItem &a) {
+      const int q_tok = a.i * BLK + row;
+      if (row < BLK && q_tok < p.Lc) {
+        uint4 *dst = reinterpret_cast<uint4 *>(p.o + ((static_cast<size_t>(a.b) * p.Lc + q_tok) * p.H + a.h) * 128 +
+                                               x * 64);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) dst[e] = make_uint4(0, 0, 0, 0);
+        if (p.lse && x == 0) p.lse[(static_cast<size_t>(a.b) * p.H + a.h) * p.Lc + q_tok] = -INFINITY;
+      }
+      if (threadIdx.x == 128) record_error(UF_EBOUNDS);
+    };
+    // first item at or after `from` (in this block's sequence) with blocks to
+    // compute; the empty ones on the way are written here
+    auto next_live = [&](int from, AttnItem &out) -> int {
+      for (int j = from; j < p.items; j += gridDim.x) {
+        out = attn_item(p, j, NKV, n_valid);
+        if (out.n >= 1) return j;
+        write_empty(out);
+      }
+      return p.items;
+    };
+    // Q of live item number kq -> tensor memory, once it has landed and the
+    // previous item's QK products have completed: this warpgroup copies
+    // channels [64x, 64x + 64) of its row out of the 128-byte-swizzled tile
+    // (32 columns of packed bf16 pairs, the A-operand layout of the QK MMA)
+    auto load_q = [&](int kq) -> bool {
+      if (!wwait(&bar_qfull, kq & 1)) return false;
+      if (kq > 0 && !wwait(&bar_qtfree, (kq - 1) & 1)) return false;
+      tc_fence_after();
       uint32_t qw[32];
-      if (row_out) {
-        const uint4 *src = reinterpret_cast<const uint4 *>(
-            p.q + ((static_cast<size_t>(b) * p.Lc + q_tok) * p.H + h) * 128 + x * 64);
+      const uint8_t *src = sQ + x * (L::Q_BYTES / 2) + row * 128;
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const uint4 v = __ldg(src + e);
-          qw[4 * e] = v.x;
-          qw[4 * e + 1] = v.y;
-          qw[4 * e + 2] = v.z;
-          qw[4 * e + 3] = v.w;
-        }
-      } else {
-#pragma unroll
-        for (int e = 0; e < 32; ++e) qw[e] = 0u;
+      for (int c = 0; c < 8; ++c) {
+        const uint4 v = *reinterpret_cast<const uint4 *>(src + ((c ^ (row & 7)) * 16));
+        qw[4 * c] = v.x;
+        qw[4 * c + 1] = v.y;
+        qw[4 * c + 2] = v.z;
+        qw[4 * c + 3] = v.w;
       }
       tmem_st32(lane_base + TM_Q + 32 * x, qw);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&bar_q);
-    }
-    float m_run = -INFINITY;   // reference max this warpgroup last saw
-    float l_run = 0.f;         // this warpgroup's partial row sum, relative to m_run
-    const int n_mine = skip ? 0 : (n - x + 1) / 2;   // kept blocks of this warpgroup
-    for (int u = 0; u < n_mine && ok; ++u) {
-      const int t = x + 2 * u;
-      int jb = row_idx ? __ldg(row_idx + t) : t;
-      if (jb < 0 || jb >= NKV) jb = diag;
-      int krow, valid;
-      kv_block_coords(jb, start, p.W, p.nb, p.nb_mul, p.lslot, BLK, p.Lc, krow, valid);
-      if (!(ok = wwait(&bar_s[x], u & 1))) break;
-      tc_fence_after();
-      const bool full = valid == BLK;
-      uint32_t s[BLK];
+      return true;
+    };
+
+    AttnItem cur;
+    int item = next_live(blockIdx.x, cur);
+    bool ok = item >= p.items || load_q(0);
+    int kq = 0, g0 = 0;   // live items and kept blocks of this thread block so far
+    while (item < p.items && ok) {
+      const int n = cur.n;
+      float m_run = -INFINITY;   // reference max this warpgroup last saw
+      float l_run = 0.f;         // this warpgroup's partial row sum, relative to m_run
+      int n_mine = 0;
+      for (int t = x ^ (g0 & 1); t < n; t += 2) {
+        const int gb = g0 + t;   // this warpgroup's (gb >> 1)-th block
+        ++n_mine;
+        bool bad;
+        const int jb = attn_block(cur, t, NKV, bad);
+        int krow, valid;
+        kv_block_coords(jb, start, p.W, p.nb, p.nb_mul, p.lslot, BLK, p.Lc, krow, valid);
+        if (!(ok = wwait(&bar_s[x], (gb >> 1) & 1))) break;
+        tc_fence_after();
+        const bool full = valid == BLK;
+        uint32_t s[BLK];
 #pragma unroll
-      for (int c = 0; c < BLK / 32; ++c)
-        tmem_ld32(lane_base + s_col + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&s[32 * c]));
-      tmem_wait_ld();
-      // block max over the block's true tokens
-      float mx;
-      {
-        float a[8];
+        for (int c = 0; c < BLK / 32; ++c)
+          tmem_ld32(lane_base + s_col + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&s[32 * c]));
+        tmem_wait_ld();
+        // block max over the block's true tokens
+        float mx;
+        {
+          float a[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) a[e] = -INFINITY;
+          for (int e = 0; e < 8; ++e) a[e] = -INFINITY;
+          if (full) {
+#pragma unroll
+            for (int c = 0; c < BLK; c += 16)
+#pragma unroll
+              for (int e = 0; e < 8; ++e)
+                a[e] = max3f(a[e], __uint_as_float(s[c + 2 * e]), __uint_as_float(s[c + 2 * e + 1]));
+          } else {
+#pragma unroll
+            for (int c = 0; c < BLK; ++c)
+              if (c < valid) a[c & 7] = fmaxf(a[c & 7], __uint_as_float(s[c]));
+          }
+          mx = max3f(max3f(a[0], a[1], a[2]), max3f(a[3], a[4], a[5]), fmaxf(a[6], a[7]));
+        }
+        // block t - 1 (the other warpgroup) has settled the reference max:
+        // adopt it, bringing this warpgroup's partial sum to the same reference
+        if (t > 0) {
+          if (!(ok = wwait(&bar_turn[x ^ 1], ((gb - 1) >> 1) & 1))) break;
+          const float m_ref = s_mref[row];
+          if (m_ref != m_run) {
+            l_run *= ex2_approx(m_run - m_ref);
+            m_run = m_ref;
+          }
+        }
+        // raise the reference only when the block max exceeds it by more than 2^8
+        bool o_ready = false;    // PV of block gb - 1 known to have completed
+        const float m_new = fmaxf(m_run, mx * c_log2);
+        if (__any_sync(0xffffffffu, m_new > m_run + ATTN_RESCALE_LOG2)) {
+          const float factor = ex2_approx(m_run - m_new);
+          l_run *= factor;
+          if (t > 0) {
+            // O holds the item's PV products up to block gb - 1: wait for the
+            // last of them, then rescale
+            if (!(ok = wwait(&bar_o[(gb - 1) & 1], ((gb - 1) >> 1) & 1))) break;
+            o_ready = true;
+            tc_fence_after();
+            const uint64_t f2 = f2_pack(factor, factor);
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
+              uint32_t o[32];
+              tmem_ld32(lane_base + TM_O + 32 * c, o);
+              tmem_wait_ld();
+#pragma unroll
+              for (int e = 0; e < 16; ++e) {
+                float lo, hi;
+                f2_unpack(f2_mul(f2_pack(__uint_as_float(o[2 * e]), __uint_as_float(o[2 * e + 1])), f2), lo, hi);
+                o[2 * e] = __float_as_uint(lo);
+                o[2 * e + 1] = __float_as_uint(hi);
+              }
+              tmem_st32(lane_base + TM_O + 32 * c, o);
+            }
+            tmem_wait_st();
+          }
+          m_run = m_new;
+        }
+        // publish the reference for block t + 1, hand over the turn and release
+        // the S buffer (held in registers from here on)
+        s_mref[row] = m_run;
+        tc_fence_before();
+        mbar_arrive(&bar_turn[x]);
+        mbar_arrive(&bar_sfree[x]);
+        // P = exp2(s * c - m): full-block and masked (partial last block of a
+        // chunk) cases are separate loops: a per-element mask test inside the
+        // unrolled loop costs two ALU instructions per element
+        const uint64_t negm2 = f2_pack(-m_run, -m_run);
+        uint32_t pk[BLK / 2];
+        uint64_t acc2[4] = {0, 0, 0, 0};
         if (full) {
 #pragma unroll
-          for (int c = 0; c < BLK; c += 16)
-#pragma unroll
-            for (int e = 0; e < 8; ++e)
-              a[e] = max3f(a[e], __uint_as_float(s[c + 2 * e]), __uint_as_float(s[c + 2 * e + 1]));
+          for (int c = 0; c < BLK / 2; ++c) {
+            float x0, x1;
+            f2_unpack(f2_fma(f2_pack(__uint_as_float(s[2 * c]), __uint_as_float(s[2 * c + 1])), c2, negm2), x0, x1);
+            const float e0 = ex2_approx(x0), e1 = ex2_approx(x1);
+            acc2[c & 3] = f2_add(acc2[c & 3], f2_pack(e0, e1));
+            pk[c] = pack_bf16x2(e0, e1);
+          }
         } else {
 #pragma unroll
-          for (int c = 0; c < BLK; ++c)
-            if (c < valid) a[c & 7] = fmaxf(a[c & 7], __uint_as_float(s[c]));
-        }
-        mx = max3f(max3f(a[0], a[1], a[2]), max3f(a[3], a[4], a[5]), fmaxf(a[6], a[7]));
-      }
-      // block t - 1 (the other warpgroup) has settled the reference max:
-      // adopt it, bringing this warpgroup's partial sum to the same reference
-      if (t > 0) {
-        if (!(ok = wwait(&bar_turn[x ^ 1], x == 0 ? ((u - 1) & 1) : (u & 1)))) break;
-        const float m_ref = s_mref[row];
-        if (m_ref != m_run) {
-          l_run *= ex2_approx(m_run - m_ref);
-          m_run = m_ref;
-        }
-      }
-      // raise the reference only when the block max exceeds it by more than 2^8
-      bool o_ready = false;    // PV_{t-1} known to have completed
-      const float m_new = fmaxf(m_run, mx * c_log2);
-      if (__any_sync(0xffffffffu, m_new > m_run + ATTN_RESCALE_LOG2)) {
-        const float factor = ex2_approx(m_run - m_new);
-        l_run *= factor;
-        if (t > 0) {
-          // O holds PV_0 .. PV_{t-1}: wait for the last of them, then rescale
-          if (!(ok = wwait(&bar_o[(t - 1) & 1], ((t - 1) >> 1) & 1))) break;
-          o_ready = true;
-          tc_fence_after();
-          const uint64_t f2 = f2_pack(factor, factor);
-#pragma unroll 1
-          for (int c = 0; c < 4; ++c) {
-            uint32_t o[32];
-            tmem_ld32(lane_base + TM_O + 32 * c, o);
-            tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              float lo, hi;
-              f2_unpack(f2_mul(f2_pack(__uint_as_float(o[2 * e]), __uint_as_float(o[2 * e + 1])), f2), lo, hi);
-              o[2 * e] = __float_as_uint(lo);
-              o[2 * e + 1] = __float_as_uint(hi);
-            }
-            tmem_st32(lane_base + TM_O + 32 * c, o);
+          for (int c = 0; c < BLK / 2; ++c) {
+            float x0, x1;
+            f2_unpack(f2_fma(f2_pack(__uint_as_float(s[2 * c]), __uint_as_float(s[2 * c + 1])), c2, negm2), x0, x1);
+            const float e0 = 2 * c < valid ? ex2_approx(x0) : 0.f;
+            const float e1 = 2 * c + 1 < valid ? ex2_approx(x1) : 0.f;
+            acc2[c & 3] = f2_add(acc2[c & 3], f2_pack(e0, e1));
+            pk[c] = pack_bf16x2(e0, e1);
           }
-          tmem_wait_st();
         }
-        m_run = m_new;
-      }
-      // publish the reference for block t + 1, hand over the turn and release
-      // S buffer t mod 2 (held in registers from here on)
-      s_mref[row] = m_run;
-      tc_fence_before();
-      mbar_arrive(&bar_turn[x]);
-      mbar_arrive(&bar_sfree[x]);
-      // P = exp2(s * c - m): full-block and masked (partial last block of a
-      // chunk) cases are separate loops: a per-element mask test inside the
-      // unrolled loop costs two ALU instructions per element
-      const uint64_t negm2 = f2_pack(-m_run, -m_run);
-      uint32_t pk[BLK / 2];
-      uint64_t acc2[4] = {0, 0, 0, 0};
-      if (full) {
-#pragma unroll
-        for (int c = 0; c < BLK / 2; ++c) {
-          float x0, x1;
-          f2_unpack(f2_fma(f2_pack(__uint_as_float(s[2 * c]), __uint_as_float(s[2 * c + 1])), c2, negm2), x0, x1);
-          const float e0 = ex2_approx(x0), e1 = ex2_approx(x1);
-          acc2[c & 3] = f2_add(acc2[c & 3], f2_pack(e0, e1));
-          pk[c] = pack_bf16x2(e0, e1);
+        {
+          float a0, a1;
+          f2_unpack(f2_add(f2_add(acc2[0], acc2[1]), f2_add(acc2[2], acc2[3])), a0, a1);
+          l_run += a0 + a1;
         }
-      } else {
-#pragma unroll
-        for (int c = 0; c < BLK / 2; ++c) {
-          float x0, x1;
-          f2_unpack(f2_fma(f2_pack(__uint_as_float(s[2 * c]), __uint_as_float(s[2 * c + 1])), c2, negm2), x0, x1);
-          const float e0 = 2 * c < valid ? ex2_approx(x0) : 0.f;
-          const float e1 = 2 * c + 1 < valid ? ex2_approx(x1) : 0.f;
-          acc2[c & 3] = f2_add(acc2[c & 3], f2_pack(e0, e1));
-          pk[c] = pack_bf16x2(e0, e1);
+        // P's columns are free once the PV of block gb - 1 has read them (for
+        // the item's first block, the previous item's epilogue waited for it)
+        if (t > 0 && !o_ready) {
+          if (!(ok = wwait(&bar_o[(gb - 1) & 1], ((gb - 1) >> 1) & 1))) break;
+          tc_fence_after();
         }
-      }
-      {
-        float a0, a1;
-        f2_unpack(f2_add(f2_add(acc2[0], acc2[1]), f2_add(acc2[2], acc2[3])), a0, a1);
-        l_run += a0 + a1;
-      }
-      // P's columns are free once PV_{t-1} has read them
-      if (t > 0 && !o_ready) {
-        if (!(ok = wwait(&bar_o[(t - 1) & 1], ((t - 1) >> 1) & 1))) break;
-        tc_fence_after();
-      }
 #pragma unroll
-      for (int c = 0; c < BLK / 64; ++c)
-        tmem_st32(lane_base + TM_P + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&pk[32 * c]));
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(&bar_p);
-    }
-    // ---------------------------------------------------------- epilogue ----
-    // Every PV has completed once PV_{n-1} has (one issuing thread, completions
-    // in order), and every QK before it.  The rings are idle then: the first K
-    // stage carries the (m, l) exchange, the first V stage the bf16 O tile for
-    // the TMA store.
-    const int n0 = skip ? 0 : (n + 1) / 2, n1 = skip ? 0 : n / 2;
-    float *s_ml = reinterpret_cast<float *>(sK);
-    uint8_t *s_out = sV;
-    if (ok && !skip) ok = wwait(&bar_o[(n - 1) & 1], ((n - 1) >> 1) & 1);
-    if (ok && !skip) {
-      s_ml[x * 256 + row] = m_run;
-      s_ml[x * 256 + 128 + row] = l_run;
+        for (int c = 0; c < BLK / 64; ++c)
+          tmem_st32(lane_base + TM_P + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&pk[32 * c]));
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&bar_p);
+      }
+      if (!ok) break;
+      // the next live item's Q goes into tensor memory now, so that its first
+      // QK products run during this item's epilogue
+      AttnItem nxt;
+      const int item_next = next_live(item + gridDim.x, nxt);
+      if (item_next < p.items && !(ok = load_q(kq + 1))) break;
+      // ---------------------------------------------------------- epilogue --
+      // every PV of the item has completed once its last one has (one issuing
+      // thread, completions in order)
+      const int gl = g0 + n - 1;
+      if (!(ok = wwait(&bar_o[gl & 1], (gl >> 1) & 1))) break;
+      // the reference after the item's last decision; each warpgroup's sum
+      // brought to it
       mbar_arrive(&bar_l);
-      ok = wwait(&bar_l, 0);
-    }
-    if (ok && !skip) {
+      if (!(ok = wwait(&bar_l, 0))) break;
+      const float m_fin = s_mref[row];
+      s_l[x][row] = n_mine > 0 ? l_run * ex2_approx(m_run - m_fin) : 0.f;
+      mbar_arrive(&bar_l);
+      if (!(ok = wwait(&bar_l, 1))) break;
+      const float l_tot = s_l[0][row] + s_l[1][row];
       tc_fence_after();
-      const float m0 = s_ml[row], m1 = s_ml[256 + row];
-      const float l0 = s_ml[128 + row], l1 = s_ml[384 + row];
-      // the reference max only grows, so O is relative to the larger one
-      const float m = n1 > 0 ? fmaxf(m0, m1) : m0;
-      float l_tot = n0 > 0 ? l0 * ex2_approx(m0 - m) : 0.f;
-      if (n1 > 0) l_tot += l1 * ex2_approx(m1 - m);
-      const float inv_l = 1.f / l_tot;
+      // this warpgroup's half of the O row; O then goes back to the PV issuer
       uint32_t o[64];
       tmem_ld32(lane_base + TM_O + x * 64, *reinterpret_cast<uint32_t(*)[32]>(&o[0]));
       tmem_ld32(lane_base + TM_O + x * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&o[32]));
       tmem_wait_ld();
-      // stage this warpgroup's 64-column half of the bf16 row, 128-byte
-      // swizzled like a TMA tile: 16-byte chunk c of row r at chunk c ^ (r mod 8)
-      uint8_t *panel = s_out + x * (128 * 128) + row * 128;
+      tc_fence_before();
+      mbar_arrive(&bar_ofree);
+      const int q_tok = cur.i * BLK + row;
+      if (row < BLK && q_tok < p.Lc) {
+        const float inv_l = 1.f / l_tot;
+        uint32_t w[32];
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        uint32_t w[4];
+        for (int e = 0; e < 32; ++e)
+          w[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv_l, __uint_as_float(o[2 * e + 1]) * inv_l);
+        __nv_bfloat16 *dst = p.o + ((static_cast<size_t>(cur.b) * p.Lc + q_tok) * p.H + cur.h) * 128 + x * 64;
+        // whole 32-byte sectors per store when O allows it
+        if ((reinterpret_cast<uintptr_t>(p.o) & 31u) == 0) {
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int k0 = 8 * c + 2 * e;
-          w[e] = pack_bf16x2(__uint_as_float(o[k0]) * inv_l, __uint_as_float(o[k0 + 1]) * inv_l);
+          for (int c = 0; c < 4; ++c) st_global_32B(dst + 16 * c, &w[8 * c]);
+        } else {
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            reinterpret_cast<uint4 *>(dst)[c] = make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
         }
-        *reinterpret_cast<uint4 *>(panel + ((c ^ (row & 7)) * 16)) = make_uint4(w[0], w[1], w[2], w[3]);
+        if (p.lse && x == 0)
+          p.lse[(static_cast<size_t>(cur.b) * p.H + cur.h) * p.Lc + q_tok] =
+              (m_fin + log2f(l_tot)) * 0.69314718055994531f;
       }
-      fence_proxy_async_smem();
-      if (row_out && p.lse && x == 0)
-        p.lse[(static_cast<size_t>(b) * p.H + h) * p.Lc + q_tok] = (m + log2f(l_tot)) * 0.69314718055994531f;
-      mbar_arrive(&bar_st[x]);
-      ok = wwait(&bar_st[x], 0);
-      if (ok && threadIdx.x == (4 + 4 * x) * 32) {
-        // one TMA store of this warpgroup's 64-column panel; rows past the
-        // q-block or past Lc are not written
-        tma_store_4d(&tmO, s_out + x * (128 * 128), x * 64, h, i * BLK, b);
-        bulk_commit();
-        bulk_wait_read();
-      }
-    } else if (skip && row_out) {
-      const size_t o_off = ((static_cast<size_t>(b) * p.Lc + q_tok) * p.H + h) * 128 + x * 64;
-      uint4 *dst = reinterpret_cast<uint4 *>(p.o + o_off);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) dst[e] = make_uint4(0, 0, 0, 0);
-      if (p.lse && x == 0) p.lse[(static_cast<size_t>(b) * p.H + h) * p.Lc + q_tok] = -INFINITY;
+      g0 += n;
+      ++kq;
+      item = item_next;
+      cur = nxt;
     }
   }
 

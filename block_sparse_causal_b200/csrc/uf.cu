@@ -103,6 +103,44 @@ int32_t ensure_smem(K kernel, int bytes, std::atomic<int> (&done)[kMaxDevices]) 
 
 int32_t launch_status() { return cuda_status(cudaGetLastError()); }
 
+// The attention kernel splits its launch register allocation between
+// warpgroups (setmaxnreg); the split is only valid for the per-thread count
+// it was written for, so a build compiled to another count is refused.
+template <typename K>
+int32_t check_launch_regs(K kernel, std::atomic<int> (&done)[kMaxDevices]) {
+  int dev = 0;
+  const int32_t st = cuda_status(cudaGetDevice(&dev));
+  if (st != UF_OK) return st;
+  if (dev < 0 || dev >= kMaxDevices) return UF_EUNSUPPORTED;
+  if (done[dev].load() == 1) return UF_OK;
+  cudaFuncAttributes attr;
+  const int32_t st2 = cuda_status(cudaFuncGetAttributes(&attr, kernel));
+  if (st2 != UF_OK) return st2;
+  if (attr.numRegs != uf::ATTN_LAUNCH_REGS) return UF_EUNSUPPORTED;
+  done[dev].store(1);
+  return UF_OK;
+}
+std::atomic<int> g_attn128_regs[kMaxDevices], g_attn64_regs[kMaxDevices];
+
+// Streaming multiprocessors of the current device (cached per device): the
+// persistent attention grid has one thread block per SM.
+std::atomic<int> g_sm_count[kMaxDevices];
+int32_t sm_count(int *out) {
+  int dev = 0;
+  const int32_t st = cuda_status(cudaGetDevice(&dev));
+  if (st != UF_OK) return st;
+  if (dev < 0 || dev >= kMaxDevices) return UF_EUNSUPPORTED;
+  int v = g_sm_count[dev].load();
+  if (v <= 0) {
+    const int32_t st2 = cuda_status(cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev));
+    if (st2 != UF_OK) return st2;
+    if (v <= 0) return UF_EUNSUPPORTED;
+    g_sm_count[dev].store(v);
+  }
+  *out = v;
+  return UF_OK;
+}
+
 std::atomic<int> g_attn128_smem[kMaxDevices], g_attn64_smem[kMaxDevices], g_mask128_smem[kMaxDevices],
     g_mask64_smem[kMaxDevices], g_mask128b_smem[kMaxDevices], g_mask64b_smem[kMaxDevices];
 
@@ -300,16 +338,16 @@ int32_t uf_block_sparse_attn(const void *q, int32_t H, const uf_kv_cache *c, con
   if (items >= (1LL << 31)) return UF_EINVAL;
 
   const int32_t lslot = nb * c->blk;
-  CUtensorMap tk, tv, to;
+  CUtensorMap tq, tk, tv;
   {
-    // O: [B, Lc, H, D] as {channels, heads, tokens, batch}; one q-block
-    // (blk rows) of one head per 64-channel store
+    // Q: [B, Lc, H, D] as {channels, heads, tokens, batch}; a 128-row tile of
+    // one head per 64-channel load (rows past Lc read as zero)
     const cuuint64_t dims[4] = {128, static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(c->Lc),
                                 static_cast<cuuint64_t>(c->B)};
     // byte strides of dims 1..3 (head, token, batch)
     const cuuint64_t strides[3] = {256, static_cast<cuuint64_t>(H) * 256, static_cast<cuuint64_t>(c->Lc) * H * 256};
-    const cuuint32_t obox[4] = {64, 1, static_cast<cuuint32_t>(c->blk), 1};
-    if (!make_map(&to, o, 4, dims, strides, obox)) return UF_ECUDA;
+    const cuuint32_t box[4] = {64, 1, 128, 1};
+    if (!make_map(&tq, q, 4, dims, strides, box)) return UF_ECUDA;
   }
   {
     // K: [B*G][W*Lslot][128] -> box {64 channels, blk tokens}
@@ -330,8 +368,8 @@ int32_t uf_block_sparse_attn(const void *q, int32_t H, const uf_kv_cache *c, con
   p.meta = c->meta;
   p.idx = idx;
   p.cnt = cnt;
-  p.q = static_cast<const __nv_bfloat16 *>(q);
   p.o = static_cast<__nv_bfloat16 *>(o);
+  p.items = static_cast<int32_t>(items);
   p.lse = lse;
   p.H = H;
   p.G = c->G;
@@ -343,18 +381,24 @@ int32_t uf_block_sparse_attn(const void *q, int32_t H, const uf_kv_cache *c, con
   p.nb_mul = nb == 1 ? 0xFFFFFFFFu : static_cast<uint32_t>((1ULL << 32) / static_cast<uint64_t>(nb));
   p.scale_log2 = scale * 1.4426950408889634f;
   p.wait_limit = g_wait_limit.load();
+  int sms = 0;
+  const int32_t se = sm_count(&sms);
+  if (se != UF_OK) return se;
+  const unsigned grid = static_cast<unsigned>(items < sms ? items : sms);
   cudaGetLastError();
   const cudaStream_t st = reinterpret_cast<cudaStream_t>(s);
   if (c->blk == 128) {
     constexpr int smem = uf::AttnSmem<128>::DYN;
-    const int32_t e = ensure_smem(uf::attn_kernel<128>, smem, g_attn128_smem);
+    int32_t e = check_launch_regs(uf::attn_kernel<128>, g_attn128_regs);
+    if (e == UF_OK) e = ensure_smem(uf::attn_kernel<128>, smem, g_attn128_smem);
     if (e != UF_OK) return e;
-    uf::attn_kernel<128><<<static_cast<unsigned>(items), uf::ATTN_THREADS, smem, st>>>(tk, tv, to, p);
+    uf::attn_kernel<128><<<grid, uf::ATTN_THREADS, smem, st>>>(tq, tk, tv, p);
   } else {
     constexpr int smem = uf::AttnSmem<64>::DYN;
-    const int32_t e = ensure_smem(uf::attn_kernel<64>, smem, g_attn64_smem);
+    int32_t e = check_launch_regs(uf::attn_kernel<64>, g_attn64_regs);
+    if (e == UF_OK) e = ensure_smem(uf::attn_kernel<64>, smem, g_attn64_smem);
     if (e != UF_OK) return e;
-    uf::attn_kernel<64><<<static_cast<unsigned>(items), uf::ATTN_THREADS, smem, st>>>(tk, tv, to, p);
+    uf::attn_kernel<64><<<grid, uf::ATTN_THREADS, smem, st>>>(tq, tk, tv, p);
   }
   return launch_status();
 }
