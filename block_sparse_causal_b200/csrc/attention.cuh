@@ -30,9 +30,8 @@
 //   warps 1, 2   one issuing thread each (an issuing thread waits for every
 //                MMA it issues to be accepted, so two of them keep the tensor
 //                core busy): warp 1 issues the QK products, requests each
-//                item's Q tile as soon as the previous one has been copied
-//                into tensor memory, and owns the tensor-memory allocation;
-//                warp 2 issues the PV products;
+//                item's Q tile once the staging tile is free, and owns the
+//                tensor-memory allocation; warp 2 issues the PV products;
 //   warps 4-7    softmax of the even-numbered blocks, warps 8-11 of the odd
 //                ones: each thread owns one row (32x32b loads), applies the
 //                block's token mask, computes exponentials in the exp2 domain
@@ -48,7 +47,10 @@
 //                warpgroup's block.  Each warpgroup keeps its own partial row
 //                sum relative to the reference it last saw; the two are
 //                combined in the item's epilogue, which also hands O back to
-//                the PV issuer for the next item.
+//                the PV issuer for the next item and stages the bf16 output
+//                in the Q staging tile (free between the copy of the next
+//                item's Q and the request for the one after), from which the
+//                PV issuer writes it with TMA stores.
 #pragma once
 
 #include "uf_device.cuh"
@@ -153,7 +155,8 @@ __device__ __forceinline__ int attn_block(const AttnItem &it, int t, int NKV, bo
 template <int BLK>
 __global__ void __launch_bounds__(ATTN_THREADS, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
+                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                const AttnParams p) {
   using L = AttnSmem<BLK>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *sQ = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -161,8 +164,9 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
   uint8_t *sV = sK + ATTN_KSTAGE * L::STAGE;
 
   // per-item barriers: Q landed in shared memory / free in tensor memory /
-  // copied into tensor memory; O read by the epilogue; (m, l) exchange
-  __shared__ uint64_t bar_qfull, bar_qtfree, bar_q, bar_ofree, bar_l;
+  // copied into tensor memory; O read by the epilogue; (m, l) exchange; O
+  // staged by each warpgroup; staging tile read by the output stores
+  __shared__ uint64_t bar_qfull, bar_qtfree, bar_q, bar_ofree, bar_l, bar_st[2], bar_ostore;
   // per-block barriers
   __shared__ uint64_t bar_kfull[ATTN_KSTAGE], bar_kempty[ATTN_KSTAGE];
   __shared__ uint64_t bar_vfull[ATTN_VSTAGE], bar_vempty[ATTN_VSTAGE];
@@ -185,6 +189,9 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
     mbar_init(&bar_q, ATTN_SOFTMAX_THREADS);
     mbar_init(&bar_ofree, ATTN_SOFTMAX_THREADS);
     mbar_init(&bar_l, ATTN_SOFTMAX_THREADS);
+    mbar_init(&bar_st[0], ATTN_SOFTMAX_THREADS / 2);
+    mbar_init(&bar_st[1], ATTN_SOFTMAX_THREADS / 2);
+    mbar_init(&bar_ostore, 1);
     for (int s = 0; s < ATTN_KSTAGE; ++s) {
       mbar_init(&bar_kfull[s], 1);
       mbar_init(&bar_kempty[s], 1);
@@ -247,7 +254,7 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
             uint8_t *dst = ring + stage * L::STAGE;
             if (is_v) {
               // V^T tile: 128 channel rows x BLK tokens, in 64-token panels
-  #pragma unroll
+#pragma unroll
               for (int pnl = 0; pnl < BLK / 64; ++pnl)
                 tma_load_3d(dst + pnl * L::VPANEL, &tmV, full, row + 64 * pnl, 0, zc);
             } else {
@@ -302,17 +309,12 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
         }
         if (item < p.items) request_q(it);
         while (item < p.items && ok) {
-          // the item's Q is in tensor memory, so the staging tile is free for
-          // the next live item's Q
+          // the item's Q is in tensor memory
           if (!(ok = wait_bounded(&bar_q, kq & 1, abort_flag, p.wait_limit))) break;
           tc_fence_after();
-          int item_next = item + gridDim.x;
+          int item_next = p.items;
           AttnItem nxt;
-          for (; item_next < p.items; item_next += gridDim.x) {
-            nxt = attn_item(p, item_next, NKV, n_valid);
-            if (nxt.n >= 1) break;
-          }
-          if (item_next < p.items) request_q(nxt);
+          const int t_request = it.n > 1 ? 1 : 0;
           for (int t = 0; t < it.n; ++t) {
             const int buf = (g0 + t) & 1;
             // the buffer's previous block has been read by the softmax
@@ -321,7 +323,7 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
             if (!(ok = wait_bounded(&bar_kfull[stage], phase, abort_flag, p.wait_limit))) break;
             tc_fence_after();
             const uint32_t k_addr = k_base + stage * L::STAGE;
-  #pragma unroll
+#pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
               const uint64_t bd = sdesc_sw128(k_addr + (kk >> 2) * L::PANEL + (kk & 3) * 32, 16, 1024);
               mma_ts(tb + tm_s(buf), tb + TM_Q + kk * 8, bd, idesc_qk, kk > 0);
@@ -332,6 +334,19 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
             if (++stage == ATTN_KSTAGE) {
               stage = 0;
               phase ^= 1u;
+            }
+            if (t == t_request) {
+              // with the item's first products on their way: the next live
+              // item's Q, once the previous item's output stores have read
+              // the staging tile
+              for (item_next = item + gridDim.x; item_next < p.items; item_next += gridDim.x) {
+                nxt = attn_item(p, item_next, NKV, n_valid);
+                if (nxt.n >= 1) break;
+              }
+              if (item_next < p.items) {
+                if (kq > 0 && !(ok = wait_bounded(&bar_ostore, (kq - 1) & 1, abort_flag, p.wait_limit))) break;
+                request_q(nxt);
+              }
             }
           }
           if (!ok) break;
@@ -359,18 +374,34 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
         uint32_t phase = 0;
         int kq = 0, g0 = 0;
         bool ok = true;
+        // output of live item number k: once its epilogue has read O and both
+        // warpgroups have staged their halves, one TMA store per 64-column
+        // panel (rows past the q-block or past Lc are not written); the
+        // staging tile is released once the stores have read it
+        auto store_output = [&](const AttnItem &a, int k) -> bool {
+          if (!wait_bounded(&bar_ofree, k & 1, abort_flag, p.wait_limit)) return false;
+          if (!wait_bounded(&bar_st[0], k & 1, abort_flag, p.wait_limit)) return false;
+          if (!wait_bounded(&bar_st[1], k & 1, abort_flag, p.wait_limit)) return false;
+          tma_store_4d(&tmO, sQ, 0, a.h, a.i * BLK, a.b);
+          tma_store_4d(&tmO, sQ + L::Q_BYTES / 2, 64, a.h, a.i * BLK, a.b);
+          bulk_commit();
+          bulk_wait_read();
+          mbar_arrive(&bar_ostore);
+          return true;
+        };
+        AttnItem prev;
         for (int item = blockIdx.x; item < p.items && ok; item += gridDim.x) {
           const AttnItem it = attn_item(p, item, NKV, n_valid);
           if (it.n < 1) continue;
-          // the previous item's epilogue has read O
-          if (kq > 0 && !(ok = wait_bounded(&bar_ofree, (kq - 1) & 1, abort_flag, p.wait_limit))) break;
+          // the previous item's output leaves (and its epilogue has read O)
+          if (kq > 0 && !(ok = store_output(prev, kq - 1))) break;
           for (int t = 0; t < it.n; ++t) {
             const int gb = g0 + t;
             if (!(ok = wait_bounded(&bar_p, gb & 1, abort_flag, p.wait_limit))) break;
             if (!(ok = wait_bounded(&bar_vfull[stage], phase, abort_flag, p.wait_limit))) break;
             tc_fence_after();
             const uint32_t v_addr = v_base + stage * L::STAGE;
-  #pragma unroll
+#pragma unroll
             for (int kk = 0; kk < BLK / 16; ++kk) {
               const uint64_t bd = sdesc_sw128(v_addr + (kk >> 2) * L::VPANEL + (kk & 3) * 32, 16, 1024);
               mma_ts(tb + TM_O, tb + TM_P + kk * 8, bd, idesc_pv, (t > 0 || kk > 0) ? 1u : 0u);
@@ -382,9 +413,11 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
               phase ^= 1u;
             }
           }
+          prev = it;
           g0 += it.n;
           ++kq;
         }
+        if (ok && kq > 0) ok = store_output(prev, kq - 1);
         mma_commit(&bar_fin[1]);
         int32_t never = 0;
         wait_bounded(&bar_fin[1], 0, &never, p.wait_limit);
@@ -613,27 +646,27 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(&bar_ofree);
-      const int q_tok = cur.i * BLK + row;
-      if (row < BLK && q_tok < p.Lc) {
-        const float inv_l = 1.f / l_tot;
-        uint32_t w[32];
+      // this warpgroup's 64-column half of the bf16 row -> the staging tile
+      // (the next item's Q has left it), 128-byte swizzled like a TMA tile:
+      // 16-byte chunk c of row r at chunk c ^ (r mod 8)
+      const float inv_l = 1.f / l_tot;
+      uint8_t *panel = sQ + x * (L::Q_BYTES / 2) + row * 128;
 #pragma unroll
-        for (int e = 0; e < 32; ++e)
-          w[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv_l, __uint_as_float(o[2 * e + 1]) * inv_l);
-        __nv_bfloat16 *dst = p.o + ((static_cast<size_t>(cur.b) * p.Lc + q_tok) * p.H + cur.h) * 128 + x * 64;
-        // whole 32-byte sectors per store when O allows it
-        if ((reinterpret_cast<uintptr_t>(p.o) & 31u) == 0) {
+      for (int c = 0; c < 8; ++c) {
+        uint32_t w[4];
 #pragma unroll
-          for (int c = 0; c < 4; ++c) st_global_32B(dst + 16 * c, &w[8 * c]);
-        } else {
-#pragma unroll
-          for (int c = 0; c < 8; ++c)
-            reinterpret_cast<uint4 *>(dst)[c] = make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+        for (int e = 0; e < 4; ++e) {
+          const int k0 = 8 * c + 2 * e;
+          w[e] = pack_bf16x2(__uint_as_float(o[k0]) * inv_l, __uint_as_float(o[k0 + 1]) * inv_l);
         }
-        if (p.lse && x == 0)
-          p.lse[(static_cast<size_t>(cur.b) * p.H + cur.h) * p.Lc + q_tok] =
-              (m_fin + log2f(l_tot)) * 0.69314718055994531f;
+        *reinterpret_cast<uint4 *>(panel + ((c ^ (row & 7)) * 16)) = make_uint4(w[0], w[1], w[2], w[3]);
       }
+      // (the PV issuer writes the tile out)
+      fence_proxy_async_smem();
+      mbar_arrive(&bar_st[x]);
+      const int q_tok = cur.i * BLK + row;
+      if (row < BLK && q_tok < p.Lc && p.lse && x == 0)
+        p.lse[(static_cast<size_t>(cur.b) * p.H + cur.h) * p.Lc + q_tok] = (m_fin + log2f(l_tot)) * 0.69314718055994531f;
       g0 += n;
       ++kq;
       item = item_next;

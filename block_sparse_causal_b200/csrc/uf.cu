@@ -338,16 +338,19 @@ int32_t uf_block_sparse_attn(const void *q, int32_t H, const uf_kv_cache *c, con
   if (items >= (1LL << 31)) return UF_EINVAL;
 
   const int32_t lslot = nb * c->blk;
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, to;
   {
-    // Q: [B, Lc, H, D] as {channels, heads, tokens, batch}; a 128-row tile of
-    // one head per 64-channel load (rows past Lc read as zero)
+    // Q and O: [B, Lc, H, D] as {channels, heads, tokens, batch}.  Q: a
+    // 128-row tile of one head per 64-channel load (rows past Lc read as
+    // zero); O: one q-block (blk rows) of one head per 64-channel store
     const cuuint64_t dims[4] = {128, static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(c->Lc),
                                 static_cast<cuuint64_t>(c->B)};
     // byte strides of dims 1..3 (head, token, batch)
     const cuuint64_t strides[3] = {256, static_cast<cuuint64_t>(H) * 256, static_cast<cuuint64_t>(c->Lc) * H * 256};
     const cuuint32_t box[4] = {64, 1, 128, 1};
     if (!make_map(&tq, q, 4, dims, strides, box)) return UF_ECUDA;
+    const cuuint32_t obox[4] = {64, 1, static_cast<cuuint32_t>(c->blk), 1};
+    if (!make_map(&to, o, 4, dims, strides, obox)) return UF_ECUDA;
   }
   {
     // K: [B*G][W*Lslot][128] -> box {64 channels, blk tokens}
@@ -392,13 +395,13 @@ int32_t uf_block_sparse_attn(const void *q, int32_t H, const uf_kv_cache *c, con
     int32_t e = check_launch_regs(uf::attn_kernel<128>, g_attn128_regs);
     if (e == UF_OK) e = ensure_smem(uf::attn_kernel<128>, smem, g_attn128_smem);
     if (e != UF_OK) return e;
-    uf::attn_kernel<128><<<grid, uf::ATTN_THREADS, smem, st>>>(tq, tk, tv, p);
+    uf::attn_kernel<128><<<grid, uf::ATTN_THREADS, smem, st>>>(tq, tk, tv, to, p);
   } else {
     constexpr int smem = uf::AttnSmem<64>::DYN;
     int32_t e = check_launch_regs(uf::attn_kernel<64>, g_attn64_regs);
     if (e == UF_OK) e = ensure_smem(uf::attn_kernel<64>, smem, g_attn64_smem);
     if (e != UF_OK) return e;
-    uf::attn_kernel<64><<<grid, uf::ATTN_THREADS, smem, st>>>(tq, tk, tv, p);
+    uf::attn_kernel<64><<<grid, uf::ATTN_THREADS, smem, st>>>(tq, tk, tv, to, p);
   }
   return launch_status();
 }

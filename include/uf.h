@@ -197,8 +197,7 @@ int32_t uf_block_mask(const void *q, int32_t H, const uf_kv_cache *c, int32_t k,
  * diagonal block and UF_EBOUNDS is recorded; a row with cnt < 1 gets O = 0,
  * LSE = -inf and UF_EBOUNDS.  One kernel launch (tcgen05 tensor cores, TMA)
  * with at most one thread block per SM, each looping over (b, h, q-block)
- * items.  q and o must be 16-byte aligned (o is written in 32-byte pieces
- * when it is 32-byte aligned).  UF_EUNSUPPORTED when the library's kernel
+ * items.  q and o must be 16-byte aligned.  UF_EUNSUPPORTED when the library's kernel
  * was compiled to a register count its warp specialisation does not expect.
  */
 int32_t uf_block_sparse_attn(const void *q, int32_t H, const uf_kv_cache *c,
