@@ -161,44 +161,60 @@ def block_scores(qpool: np.ndarray, kpool: np.ndarray, scale: float) -> np.ndarr
     return out
 
 
-def select_blocks(scores: np.ndarray, k: int, diag: Sequence[int]):
-    """Per-row top-k block selection with a forced diagonal block.
+def select_blocks(scores: np.ndarray, k: int, diag: Sequence[int], local: int = 0, local_only: bool = False):
+    """Per-row top-k block selection with forced blocks.
+
+    Ultra Flash (papernotes notes), Method, key design 3: each head keeps its
+    top-k blocks by pooled score; the layer's mask also combines a local
+    sliding-window mask (and the ablation table's "fixed local window instead
+    of adaptive top-k" keeps that window alone).  Forced blocks: the band of
+    logical blocks within ``local`` of the diagonal, clipped to the window
+    (local = 0: the diagonal alone).  The rest of the row's k blocks are the
+    others ranked by (score descending, logical index ascending); with
+    ``local_only`` the row is the band alone.
 
     scores [B, H, NQ, NKV]; diag[i] = logical index of q-block i's own block.
-    Returns (idx [B, H, NQ, k_eff] ascending int32, cnt [B, H, NQ] int32,
-    boundary [B, H, NQ, 2] float64).  ``boundary`` holds the score of the last
-    kept non-diagonal block and of the first dropped one (NaN when there is
-    none); rows where the two are closer than the near-tie tolerance may
-    legitimately differ between two correct implementations.
+    Returns (idx [B, H, NQ, k_eff] int32, ascending, padded with -1 past cnt;
+    cnt [B, H, NQ] int32; boundary [B, H, NQ, 2] float64).  ``boundary`` holds
+    the score of the last kept scored block and of the first dropped one (NaN
+    when there is none); rows where the two are closer than the near-tie
+    tolerance may legitimately differ between two correct implementations.
     """
     B, H, NQ, NKV = scores.shape
     k_eff = min(k, NKV)
     if k_eff < 1:
         raise ValueError("k must be >= 1")
-    idx = np.empty((B, H, NQ, k_eff), dtype=np.int32)
-    cnt = np.full((B, H, NQ), k_eff, dtype=np.int32)
+    if local < 0 or 2 * local + 1 > k:
+        raise ValueError("the band (2 local + 1 blocks) must fit in k")
+    idx = np.full((B, H, NQ, k_eff), -1, dtype=np.int32)
+    cnt = np.zeros((B, H, NQ), dtype=np.int32)
     boundary = np.full((B, H, NQ, 2), np.nan)
     all_j = np.arange(NKV)
     for b in range(B):
         for h in range(H):
             for i in range(NQ):
                 d = diag[i]
-                cand = all_j[all_j != d]
+                band = all_j[np.abs(all_j - d) <= local]
+                take = 0 if local_only else k_eff - len(band)
+                cand = all_j[np.abs(all_j - d) > local]
                 s = scores[b, h, i, cand]
                 # rank: score descending, then logical index ascending
                 order = cand[np.lexsort((cand, -s))]
-                chosen = order[: k_eff - 1]
-                idx[b, h, i] = np.sort(np.append(chosen, d))
-                if k_eff - 1 >= 1:
-                    boundary[b, h, i, 0] = scores[b, h, i, order[k_eff - 2]]
-                if k_eff - 1 < len(order):
-                    boundary[b, h, i, 1] = scores[b, h, i, order[k_eff - 1]]
+                chosen = order[:take]
+                row = np.sort(np.concatenate([band, chosen]))
+                idx[b, h, i, : len(row)] = row
+                cnt[b, h, i] = len(row)
+                if take >= 1:
+                    boundary[b, h, i, 0] = scores[b, h, i, order[take - 1]]
+                if not local_only and take < len(order):
+                    boundary[b, h, i, 1] = scores[b, h, i, order[take]]
     return idx, cnt, boundary
 
 
 def block_mask(q: np.ndarray, window: RollingWindow, blk: int, k: int,
-               scale: Optional[float] = None):
-    """The whole mask step for the newest chunk's queries.
+               scale: Optional[float] = None, local: int = 0, local_only: bool = False):
+    """The whole mask step for the newest chunk's queries (``local`` and
+    ``local_only`` as in select_blocks).
 
     q [B, Lc, H, D]; the window holds n_valid chunks of K [B, Lc, G, D].
     Returns dict(idx, cnt, scores, boundary, qpool, kpool).
@@ -214,7 +230,7 @@ def block_mask(q: np.ndarray, window: RollingWindow, blk: int, k: int,
     kpool = np.concatenate([pool_blocks(kc, blk) for kc in window.k], axis=2)  # [B,G,NKV,D]
     scores = block_scores(qpool, kpool, scale)
     diag = [(n_valid - 1) * nb + i for i in range(nb)]
-    idx, cnt, boundary = select_blocks(scores, k, diag)
+    idx, cnt, boundary = select_blocks(scores, k, diag, local, local_only)
     return dict(idx=idx, cnt=cnt, scores=scores, boundary=boundary, qpool=qpool, kpool=kpool)
 
 

@@ -148,6 +148,65 @@ def test_density_one_keeps_all_blocks():
     assert np.array_equal(idx, idx2) and np.all(cnt2 == 10)
 
 
+# ------------------------------------------------ local-band pins ----------
+def _bruteforce_select_forced(row, k, forced):
+    """Among all k-subsets containing every forced block, the one with the
+    largest score sum, ties broken by the smallest index sum."""
+    others = [j for j in range(len(row)) if j not in forced]
+    best, best_key = (), None
+    for sub in itertools.combinations(others, k - len(forced)):
+        key = (math.fsum(row[j] for j in sub), -sum(sub))
+        if best_key is None or key > best_key:
+            best, best_key = sub, key
+    return sorted(list(best) + list(forced))
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_local_band_bruteforce(seed):
+    # band [d - local, d + local] clipped to the window, then the best others
+    r = np.random.default_rng(200 + seed)
+    NQ, NKV = 4, 10
+    scores = r.standard_normal((1, 2, NQ, NKV))
+    diag = [6 + i for i in range(NQ)]
+    for local in (1, 2):
+        for k in (2 * local + 1, 2 * local + 2, 2 * local + 3, 8):
+            idx, cnt, _ = select_blocks(scores, k, diag, local=local)
+            assert np.all(cnt == k)
+            for h in range(2):
+                for i in range(NQ):
+                    band = [j for j in range(NKV) if abs(j - diag[i]) <= local]
+                    want = _bruteforce_select_forced(scores[0, h, i], k, band)
+                    assert idx[0, h, i].tolist() == want, (local, k, i)
+
+
+def test_local_only_is_the_clipped_band():
+    scores = np.random.default_rng(5).standard_normal((1, 1, 4, 10))
+    idx, cnt, bnd = select_blocks(scores, 7, [6, 7, 8, 9], local=2, local_only=True)
+    assert cnt[0, 0].tolist() == [5, 5, 4, 3]            # the last rows run past the window
+    assert idx[0, 0, 0].tolist() == [4, 5, 6, 7, 8, -1, -1]
+    assert idx[0, 0, 3].tolist() == [7, 8, 9, -1, -1, -1, -1]
+    assert np.all(np.isnan(bnd))                          # no scored block, no boundary
+
+
+def test_local_band_wider_than_window_keeps_everything():
+    scores = np.random.default_rng(6).standard_normal((1, 1, 2, 6))
+    idx, cnt, _ = select_blocks(scores, 11, [4, 5], local=5)
+    assert np.all(cnt == 6) and np.all(idx == np.arange(6))
+
+
+def test_local_band_must_fit_in_k():
+    scores = np.zeros((1, 1, 1, 8))
+    with pytest.raises(ValueError):
+        select_blocks(scores, 4, [7], local=2)
+
+
+def test_local_band_with_ties_prefers_low_index():
+    # all scores equal: after the band, the lowest-index blocks are taken
+    scores = np.zeros((1, 1, 1, 12))
+    idx, _, _ = select_blocks(scores, 5, [9], local=1)
+    assert idx[0, 0, 0].tolist() == [0, 1, 8, 9, 10]
+
+
 def test_mask_known_argmax_one_hot_offsets():
     # every key block of the older chunk points along its own axis e_j, the query
     # block i points along e_{(3*i) % 8}; the best non-diagonal block is therefore
