@@ -104,6 +104,10 @@ def append_bytes(cfg):
     return 2 * chunk + 2 * slot + cfg.B * cfg.G * cfg.nb * cfg.D * 4
 
 
+def mask_call_name(args):
+    return "uf_block_mask_local + " if (args.mask_local or args.mask_local_only) else "uf_block_mask + "
+
+
 def mask_bytes(cfg, k):
     # read Q once; pooled K of the window once per KV head; write idx and cnt
     return (cfg.B * cfg.Lc * cfg.H * cfg.D * 2 + cfg.B * cfg.G * cfg.nkv() * cfg.D * 4
@@ -176,10 +180,17 @@ class ClockSampler:
 
 
 # --------------------------------------------------------------- GPU arm ----
+def mask_k(args, cfg):
+    """Kept blocks per q-block: the workload's k, widened to hold a forced local band."""
+    k = cfg.k_for() if not cfg.dense else cfg.nkv()
+    return max(k, 2 * args.mask_local + 1) if not cfg.dense else k
+
+
 def run_ours(args, cfg, rank, world, device):
     import block_sparse_causal_b200 as uf
     stream = torch.cuda.current_stream()
-    k = cfg.k_for() if not cfg.dense else cfg.nkv()
+    k = mask_k(args, cfg)
+    local_flags = uf.UF_MASK_LOCAL_ONLY if args.mask_local_only else 0
     scale = 1.0 / math.sqrt(cfg.D)
 
     # seeded chunks, generated on the host, resident in HBM before timing
@@ -207,7 +218,10 @@ def run_ours(args, cfg, rank, world, device):
                 ev[2].record(stream)
             uf.uf_block_sparse_attn(chunk["q"], cfg.H, win.desc, None, None, 0, scale, o, lse)
         else:
-            uf.uf_block_mask(chunk["q"], cfg.H, win.desc, k, idx[s], cnt[s])
+            if args.mask_local or args.mask_local_only:
+                uf.uf_block_mask_local(chunk["q"], cfg.H, win.desc, k, args.mask_local, local_flags, idx[s], cnt[s])
+            else:
+                uf.uf_block_mask(chunk["q"], cfg.H, win.desc, k, idx[s], cnt[s])
             if ev is not None:
                 ev[2].record(stream)
             uf.uf_block_sparse_attn(chunk["q"], cfg.H, win.desc, idx[s], cnt[s], k, scale, o, lse)
@@ -316,7 +330,8 @@ def run_ours(args, cfg, rank, world, device):
             "workload": args.config, "description": cfg.description, "B": cfg.B, "H": cfg.H, "G": cfg.G,
             "D": cfg.D, "Lc": cfg.Lc, "W": cfg.W, "blk": cfg.blk, "k": k,
             "density": cfg.density, "kept_flops_per_step": flops_per_step,
-            "step": "uf_kv_append + " + ("" if cfg.dense else "uf_block_mask + ") + "uf_block_sparse_attn",
+            "mask_local": args.mask_local, "mask_local_only": bool(args.mask_local_only),
+            "step": "uf_kv_append + " + ("" if cfg.dense else mask_call_name(args)) + "uf_block_sparse_attn",
             "l2": "no flush: every step's working set (%.0f MB) exceeds the 126 MB L2" % (
                 (cfg.B * cfg.Lc * (cfg.H * 2 + cfg.G * 2) * cfg.D * 2
                  + 2 * cfg.B * cfg.G * cfg.nkv() * cfg.blk * cfg.D * 2) / 1e6),
@@ -348,17 +363,20 @@ class OracleSample:
     mask of one query head over the full window, then attention for up to
     ``n_items`` work items of that head.  Inputs are prepared once."""
 
-    def __init__(self, cfg, seed):
+    def __init__(self, cfg, seed, local=0, local_only=False):
         import oracle
         from workloads import to_f64
         self.oracle = oracle
         self.cfg = cfg
+        self.local, self.local_only = local, local_only
         chunks = [chunk_inputs(cfg, seed, t) for t in range(cfg.W)]
         self.win = oracle.RollingWindow(cfg.W)
         for c in chunks:
             self.win.append(to_f64(c["k"][:, :, 0:1]), to_f64(c["v"][:, :, 0:1]))
         self.q = to_f64(chunks[-1]["q"][:, :, 0:1])
         self.k = cfg.k_for() if not cfg.dense else cfg.nkv()
+        if not cfg.dense:
+            self.k = max(self.k, 2 * local + 1)
         self.vq = [cfg.blk] * (cfg.nb - 1) + [cfg.last_block_tokens]
         self.vkv = self.vq * cfg.W
 
@@ -366,13 +384,13 @@ class OracleSample:
         """Returns (kept FLOPs computed, seconds, description)."""
         cfg = self.cfg
         t0 = time.perf_counter()
-        m = self.oracle.block_mask(self.q, self.win, cfg.blk, self.k)
+        m = self.oracle.block_mask(self.q, self.win, cfg.blk, self.k, local=self.local, local_only=self.local_only)
         flops = 0.0
         done = 0
         while done < n_items and time.perf_counter() - t0 < budget_s:
             i = (first_item + done) % cfg.nb
             self.oracle.block_sparse_attention(self.q, self.win, cfg.blk, m["idx"], m["cnt"], items=[(0, 0, i)])
-            flops += 4.0 * cfg.D * self.vq[i] * sum(self.vkv[j] for j in m["idx"][0, 0, i])
+            flops += 4.0 * cfg.D * self.vq[i] * sum(self.vkv[j] for j in m["idx"][0, 0, i, :m["cnt"][0, 0, i]])
             done += 1
         dt = time.perf_counter() - t0
         return flops, dt, (f"mask of 1 head ({cfg.nb} q-blocks over {cfg.nkv()} kv blocks) "
@@ -390,15 +408,15 @@ def blas_threads():
     return os.cpu_count()
 
 
-def cpu_baseline(cfg, seed):
-    flops, dt, desc = OracleSample(cfg, seed).run(n_items=10_000, budget_s=12.0)
+def cpu_baseline(cfg, seed, local=0, local_only=False):
+    flops, dt, desc = OracleSample(cfg, seed, local, local_only).run(n_items=10_000, budget_s=12.0)
     return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
             "sample": desc + f", {dt:.1f} s of fp64 numpy", "seconds": dt}
 
 
 def run_reference(args, cfg):
     # each step: the oracle on a bounded sample (one head's mask + 1 work item)
-    sample = OracleSample(cfg, args.seed)
+    sample = OracleSample(cfg, args.seed, args.mask_local, args.mask_local_only)
     for s in range(args.warmup):
         sample.run(n_items=1, budget_s=5.0, first_item=s)
     tot_f, tot_t = 0.0, 0.0
@@ -408,13 +426,14 @@ def run_reference(args, cfg):
         tot_f += f
         tot_t += t
     value = tot_f / tot_t / 1e12
-    k = cfg.k_for() if not cfg.dense else cfg.nkv()
+    k = mask_k(args, cfg)
     return {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": 1,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot_t / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": args.config, "description": cfg.description, "B": cfg.B, "H": cfg.H, "G": cfg.G,
-                   "D": cfg.D, "Lc": cfg.Lc, "W": cfg.W, "blk": cfg.blk, "k": k, "density": cfg.density},
+                   "D": cfg.D, "Lc": cfg.Lc, "W": cfg.W, "blk": cfg.blk, "k": k, "density": cfg.density,
+                   "mask_local": args.mask_local, "mask_local_only": bool(args.mask_local_only)},
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
                          "sample": "per step: " + desc},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -444,6 +463,10 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing leg")
+    ap.add_argument("--mask-local", type=int, default=0,
+                    help="radius of the forced local band of blocks around the diagonal (uf_block_mask_local)")
+    ap.add_argument("--mask-local-only", action="store_true",
+                    help="keep the local band only (the fixed-local-window mask)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -468,7 +491,7 @@ def main():
         result = run_ours(args, cfg, rank, world, device)
         if rank == 0:
             if world == 1 and not args.no_cpu_baseline:
-                result["cpu_baseline"] = cpu_baseline(cfg, args.seed)
+                result["cpu_baseline"] = cpu_baseline(cfg, args.seed, args.mask_local, args.mask_local_only)
             else:
                 result["cpu_baseline"] = None
             print(json.dumps(result), flush=True)

@@ -14,6 +14,7 @@ _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libuf.so")
 
 UF_OK, UF_EINVAL, UF_ECUDA, UF_ETIMEOUT, UF_EBOUNDS, UF_EUNSUPPORTED = range(6)
 UF_APPEND_REPLACE_NEWEST = 1
+UF_MASK_LOCAL_ONLY = 1
 
 
 class UfKvCache(ctypes.Structure):
@@ -54,6 +55,7 @@ def _load() -> ctypes.CDLL:
         "uf_kv_reset": ([pc, vp], i32),
         "uf_kv_append": ([pc, vp, vp, i32, i32, vp], i32),
         "uf_block_mask": ([vp, i32, pc, i32, vp, vp, vp, vp], i32),
+        "uf_block_mask_local": ([vp, i32, pc, i32, i32, i32, vp, vp, vp, vp], i32),
         "uf_block_sparse_attn": ([vp, i32, pc, vp, vp, i32, ctypes.c_float, vp, vp, vp], i32),
         "uf_get_error": ([ctypes.POINTER(i32), i32], i32),
         "uf_last_cuda_error": ([], ctypes.c_char_p),
@@ -117,6 +119,12 @@ def uf_kv_append(cache: UfKvCache, k_new, v_new, keep_chunks: int, flags: int = 
 def uf_block_mask(q, H: int, cache: UfKvCache, k: int, idx, cnt, scores=None, stream=None) -> None:
     _check(lib.uf_block_mask(_ptr(q), H, ctypes.byref(cache), k, _ptr(idx), _ptr(cnt), _ptr(scores),
                              _stream(stream)), "uf_block_mask")
+
+
+def uf_block_mask_local(q, H: int, cache: UfKvCache, k: int, local: int, flags: int, idx, cnt, scores=None,
+                        stream=None) -> None:
+    _check(lib.uf_block_mask_local(_ptr(q), H, ctypes.byref(cache), k, local, flags, _ptr(idx), _ptr(cnt),
+                                   _ptr(scores), _stream(stream)), "uf_block_mask_local")
 
 
 def uf_block_sparse_attn(q, H: int, cache: UfKvCache, idx, cnt, k: int, scale: float, o, lse=None,

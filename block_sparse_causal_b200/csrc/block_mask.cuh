@@ -43,6 +43,8 @@ struct MaskParams {
   int32_t *cnt;             // [B, H, nb]
   float *scores;            // optional [B, H, nb, W*nb]
   int32_t H, G, W, Lc, nb, k;
+  int32_t local;            // radius of the forced band of blocks around the diagonal
+  int32_t local_only;       // keep the band only (no scored blocks)
   float scale;
 };
 
@@ -217,17 +219,21 @@ __global__ void __launch_bounds__(256, 2) block_mask_kernel(const __grid_constan
       for (int j = lane; j < NKV; j += 32) p.scores[row * nkv_max + j] = sc[j];
     }
     const int diag = (n_valid - 1) * p.nb + i;
-    const int k_eff = min(p.k, NKV);
-    const int need = k_eff - 1;            // non-diagonal blocks to keep
+    // forced blocks: the band [diag - local, diag + local] of the window
+    // (local = 0: the diagonal alone); the host guarantees 2 local + 1 <= k
+    const int lo = max(0, diag - p.local), hi = min(NKV - 1, diag + p.local);
+    const int n_forced = hi - lo + 1;
+    const int k_eff = p.local_only ? n_forced : min(p.k, NKV);
+    const int need = k_eff - n_forced;     // scored blocks to keep
     const int per = (NKV + 31) / 32;       // keys of this lane: j in [lane*per, lane*per + per)
     const int jb = lane * per;
-    // order-preserving integer keys in registers; the diagonal and padding get 0
-    // (below every real key: a float's key is never 0) and are never counted
+    // order-preserving integer keys in registers; forced blocks and padding get
+    // 0 (below every real key: a float's key is never 0) and are never counted
     uint32_t key[MAXPER];
 #pragma unroll
     for (int m = 0; m < MAXPER; ++m) {
       const int j = jb + m;
-      key[m] = (m < per && j < NKV && j != diag) ? order_key(sc[j]) : 0u;
+      key[m] = (m < per && j < NKV && (j < lo || j > hi)) ? order_key(sc[j]) : 0u;
     }
     uint32_t T = 0xFFFFFFFFu;              // threshold key (need == 0: nothing passes)
     int take_eq = 0;
@@ -259,7 +265,7 @@ __global__ void __launch_bounds__(256, 2) block_mask_kernel(const __grid_constan
 #pragma unroll
       for (int m = 0; m < MAXPER; ++m) {
         const int j = jb + m;
-        bool keep = (m < per && j == diag);
+        bool keep = (m < per && j >= lo && j <= hi);
         if (need > 0 && key[m] != 0u) {
           if (key[m] > T) keep = true;
           else if (key[m] == T && eq_run < take_eq) keep = true;

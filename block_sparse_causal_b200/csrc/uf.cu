@@ -256,7 +256,14 @@ int32_t uf_kv_append(uf_kv_cache *c, const void *k_new, const void *v_new, int32
 
 int32_t uf_block_mask(const void *q, int32_t H, const uf_kv_cache *c, int32_t k, int32_t *idx, int32_t *cnt,
                       float *scores, uf_stream_t s) {
+  return uf_block_mask_local(q, H, c, k, 0, 0, idx, cnt, scores, s);
+}
+
+int32_t uf_block_mask_local(const void *q, int32_t H, const uf_kv_cache *c, int32_t k, int32_t local,
+                            int32_t flags, int32_t *idx, int32_t *cnt, float *scores, uf_stream_t s) {
   if (!cache_ok(c)) return UF_EINVAL;
+  if (local < 0 || local > (1 << 20) || (flags & ~UF_MASK_LOCAL_ONLY) != 0) return UF_EINVAL;
+  if (2 * local + 1 > k) return UF_EINVAL;
   if (!q || !idx || !cnt || !aligned16(q)) return UF_EINVAL;
   if (!aligned16(idx) || !aligned16(cnt) || (scores && !aligned16(scores))) return UF_EINVAL;
   if (H < 1 || H % c->G != 0) return UF_EINVAL;
@@ -280,6 +287,8 @@ int32_t uf_block_mask(const void *q, int32_t H, const uf_kv_cache *c, int32_t k,
   p.Lc = c->Lc;
   p.nb = nb;
   p.k = k;
+  p.local = local;
+  p.local_only = (flags & UF_MASK_LOCAL_ONLY) ? 1 : 0;
   p.scale = 1.0f / sqrtf(static_cast<float>(c->D));
   const int smem = uf::mask_smem_bytes(c->blk, nkv_max);
   // Q slices for the pooling: {channels, heads, tokens, batch}, box {64, 1, blk, 1}, no swizzle

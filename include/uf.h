@@ -6,6 +6,8 @@
  *   uf_kv_append         rolling-window append / evict of the new chunk's K and V
  *   uf_block_mask        per-head block mean-pooling of Q and K, pooled block
  *                        scores, top-k block selection with the diagonal kept
+ *                        (uf_block_mask_local: with a forced local band of
+ *                        blocks around the diagonal, or the band alone)
  *   uf_block_sparse_attn softmax attention of the chunk's queries over the kept
  *                        blocks of the window (bf16 in, fp32 softmax, bf16 O and
  *                        fp32 LSE), grouped-query aware
@@ -172,6 +174,29 @@ int32_t uf_kv_append(uf_kv_cache *c, const void *k_new, const void *v_new,
  */
 int32_t uf_block_mask(const void *q, int32_t H, const uf_kv_cache *c, int32_t k,
                       int32_t *idx, int32_t *cnt, float *scores, uf_stream_t s);
+
+/* uf_block_mask_local flag: keep the local band only (no scored blocks). */
+#define UF_MASK_LOCAL_ONLY 1
+
+/*
+ * Block mask with a local sliding-window band (Ultra Flash notes, Method, key
+ * design 3: each attention layer combines a local sliding-window mask with the
+ * temporal causal mask, then keeps each head's top-k blocks; the ablation
+ * table's "fixed local window instead of adaptive top-k" is the band alone).
+ * The pages do not define the band's shape; here it is the run of logical
+ * kv blocks within `local` of the diagonal, [d_i - local, d_i + local]
+ * clipped to [0, NKV).
+ *
+ *   local   band radius in blocks, >= 0, with 2 * local + 1 <= k;
+ *           uf_block_mask(...) is uf_block_mask_local(..., local = 0, flags = 0).
+ *   flags   0: keep the band, then the other blocks ranked by (score
+ *           descending, logical id ascending) until the row has min(k, NKV)
+ *           blocks; UF_MASK_LOCAL_ONLY: keep the band only (cnt = its size).
+ *   other arguments, outputs and errors as uf_block_mask.
+ */
+int32_t uf_block_mask_local(const void *q, int32_t H, const uf_kv_cache *c, int32_t k,
+                            int32_t local, int32_t flags, int32_t *idx, int32_t *cnt,
+                            float *scores, uf_stream_t s);
 
 /*
  * Block-sparse chunk-causal attention (Ultra Flash notes, key design 3:

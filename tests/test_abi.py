@@ -111,6 +111,11 @@ def test_calls_reject_bad_arguments_before_launch(uf):
         with pytest.raises(uf.UfError) as e:
             uf.uf_block_mask(q, H, c, k, idx, cnt, None, stream=0)
         assert e.value.status == uf.UF_EINVAL
+    # local band: wider than k, negative radius, unknown flag (every case is invalid: nothing launches)
+    for k, local, flags in [(2, 1, 0), (5, -1, 0), (5, 1, 2), (6, 3, 0), (3, 1, uf.UF_MASK_LOCAL_ONLY | 4)]:
+        with pytest.raises(uf.UfError) as e:
+            uf.uf_block_mask_local(q, 2, c, k, local, flags, idx, cnt, None, stream=0)
+        assert e.value.status == uf.UF_EINVAL
     for scale in (0.0, -1.0, float("inf"), float("nan")):
         with pytest.raises(uf.UfError) as e:
             uf.uf_block_sparse_attn(q, 2, c, None, None, 0, scale, FakeTensor(0xA00000), None, stream=0)

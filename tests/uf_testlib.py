@@ -42,7 +42,7 @@ class GpuStream:
         v = inp["v"].to(self.device)
         self.win.append(k, v, keep_chunks=keep, replace_newest=replace)
 
-    def mask(self, q_cpu, k: int, want_scores=True):
+    def mask(self, q_cpu, k: int, want_scores=True, local: int = 0, local_only: bool = False):
         cfg = self.cfg
         q = q_cpu.to(self.device)
         nb = cfg.nb
@@ -50,7 +50,11 @@ class GpuStream:
         cnt = torch.full((cfg.B, cfg.H, nb), -7, dtype=torch.int32, device=self.device)
         scores = (torch.full((cfg.B, cfg.H, nb, cfg.W * nb), float("nan"), device=self.device)
                   if want_scores else None)
-        self.uf.uf_block_mask(q, cfg.H, self.win.desc, k, idx, cnt, scores)
+        if local == 0 and not local_only:
+            self.uf.uf_block_mask(q, cfg.H, self.win.desc, k, idx, cnt, scores)
+        else:
+            flags = self.uf.UF_MASK_LOCAL_ONLY if local_only else 0
+            self.uf.uf_block_mask_local(q, cfg.H, self.win.desc, k, local, flags, idx, cnt, scores)
         return idx, cnt, scores
 
     def attention(self, q_cpu, idx=None, cnt=None, k=0, scale=None):
@@ -84,12 +88,13 @@ class OracleStream:
     def head_window(self, h):
         return self.windows[h // (self.cfg.H // self.cfg.G)]
 
-    def mask(self, q_cpu, k: int, heads: Optional[Sequence[int]] = None):
+    def mask(self, q_cpu, k: int, heads: Optional[Sequence[int]] = None, local: int = 0, local_only: bool = False):
         cfg = self.cfg
         heads = range(cfg.H) if heads is None else heads
         out = {}
         for h in heads:
-            r = oracle.block_mask(to_f64(q_cpu[:, :, h:h + 1]), self.head_window(h), cfg.blk, k)
+            r = oracle.block_mask(to_f64(q_cpu[:, :, h:h + 1]), self.head_window(h), cfg.blk, k,
+                                  local=local, local_only=local_only)
             out[h] = r
         return out
 
