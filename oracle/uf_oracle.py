@@ -60,6 +60,8 @@ __all__ = [
     "select_blocks",
     "block_mask",
     "block_sparse_attention",
+    "rope",
+    "window_rope",
 ]
 
 
@@ -289,3 +291,48 @@ def block_sparse_attention(q: np.ndarray, window: RollingWindow, blk: int,
         O[b, s0:e0, h, :] = (p @ vv) / l[:, None]
         LSE[b, h, s0:e0] = m[:, 0] + np.log(l)
     return O, LSE
+
+
+# --------------------------------------------------------------------------
+# Rotary position embedding with window-relative positions
+# --------------------------------------------------------------------------
+def rope(x: np.ndarray, pos: np.ndarray, base: float = 10000.0) -> np.ndarray:
+    """Rotary position embedding of the last axis (RoFormer, Su et al. 2021:
+    channel pairs (x_2i, x_2i+1) rotated by the angle pos * theta_i with
+    theta_i = base^(-2i / D)).  The pages name RoPE but not its form
+    (FlashDecoder, "long video decoding": positions relative to the current
+    window; Algorithm 1: "RoPE offset t * L_frm"); this is the published form.
+
+    x [..., L, heads, D]; pos [L] integer positions of the L tokens.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    D = x.shape[-1]
+    if D % 2:
+        raise ValueError("D must be even")
+    theta = base ** (-2.0 * np.arange(D // 2) / D)                      # [D/2]
+    ang = np.asarray(pos, dtype=np.float64)[:, None] * theta[None, :]   # [L, D/2]
+    c = np.cos(ang)[:, None, :]                                         # [L, 1, D/2]
+    s = np.sin(ang)[:, None, :]
+    x0, x1 = x[..., 0::2], x[..., 1::2]
+    out = np.empty_like(x)
+    out[..., 0::2] = x0 * c - x1 * s
+    out[..., 1::2] = x0 * s + x1 * c
+    return out
+
+
+def window_rope(q: np.ndarray, window: RollingWindow, base: float = 10000.0):
+    """The window and the newest chunk's queries with RoPE at window-relative
+    positions (FlashDecoder, "long video decoding": RoPE positions are assigned
+    relative to the current window, not by absolute frame index): token r of
+    the window's chunk c (c = 0 the oldest) sits at c * Lc + r, so the query
+    chunk (the newest) sits at (n_valid - 1) * Lc + r.  Returns (q_rot, a new
+    RollingWindow holding the rotated K and the unchanged V), ready for
+    block_mask and block_sparse_attention.
+    """
+    Lc = q.shape[1]
+    n = window.n_valid
+    out = RollingWindow(window.W)
+    for c in range(n):
+        out.append(rope(window.k[c], c * Lc + np.arange(Lc), base), window.v[c])
+    q_rot = rope(q, (n - 1) * Lc + np.arange(Lc), base)
+    return q_rot, out

@@ -10,8 +10,8 @@ import os
 import numpy as np
 import pytest
 
-from oracle import (RollingWindow, block_mask, block_ranges, block_scores,
-                    block_sparse_attention, pool_blocks, select_blocks, window_blocks)
+from oracle import (RollingWindow, block_mask, block_ranges, block_scores, block_sparse_attention,
+                    pool_blocks, rope, select_blocks, window_blocks, window_rope)
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 rng = np.random.default_rng(1234)
@@ -481,3 +481,89 @@ def test_first_chunk_window_is_own_chunk_only():
     m = block_mask(q, w, blk, 5)
     assert m["idx"].shape[-1] == 2 and np.all(m["cnt"] == 2)
     assert m["scores"].shape[-1] == 2
+
+
+# ------------------------------------------------------------ RoPE pins ------
+
+def test_rope_position_zero_is_identity():
+    x = np.random.default_rng(1).standard_normal((2, 3, 4, 16))
+    assert np.array_equal(rope(x, np.zeros(3, dtype=np.int64)), x)
+
+
+def test_rope_is_complex_multiplication_per_pair():
+    # RoFormer's complex form: (x_2i + i x_2i+1) * exp(i * pos * theta_i)
+    r = np.random.default_rng(2)
+    D, L = 8, 6
+    x = r.standard_normal((1, L, 1, D))
+    pos = np.array([0, 1, 7, 100, 12345, 987654])
+    y = rope(x, pos, base=500.0)
+    z = x[..., 0::2] + 1j * x[..., 1::2]
+    ang = np.outer(pos, [math.pow(500.0, -2.0 * i / D) for i in range(D // 2)])
+    w = z * np.exp(1j * ang)[None, :, None, :]
+    assert np.allclose(y[..., 0::2], w.real, atol=1e-9) and np.allclose(y[..., 1::2], w.imag, atol=1e-9)
+
+
+def test_rope_frequencies_form_the_roformer_ladder():
+    # rotate unit vectors by position 1 and read each pair's angle back
+    D, base = 16, 10000.0
+    x = np.zeros((1, 1, D // 2, D))
+    for i in range(D // 2):
+        x[0, 0, i, 2 * i] = 1.0
+    y = rope(x, np.array([1]), base)
+    ang = np.array([math.atan2(y[0, 0, i, 2 * i + 1], y[0, 0, i, 2 * i]) for i in range(D // 2)])
+    assert abs(ang[0] - 1.0) < 1e-15                                  # theta_0 = 1 rad per position
+    ratio = ang[1:] / ang[:-1]
+    assert np.allclose(ratio, base ** (-2.0 / D), rtol=1e-12)         # geometric in the pair index
+    assert abs(ang[-1] - base ** (-(D - 2) / D)) < 1e-15
+
+
+def test_rope_scores_depend_on_position_difference_only():
+    r = np.random.default_rng(3)
+    q, k = r.standard_normal((1, 1, 1, 32)), r.standard_normal((1, 1, 1, 32))
+    for m, n, c in [(5, 2, 100), (0, 17, 4096), (300, 300, 7)]:
+        a = float(np.sum(rope(q, [m]) * rope(k, [n])))
+        b = float(np.sum(rope(q, [m + c]) * rope(k, [n + c])))
+        d = float(np.sum(q * rope(k, [n - m])))                       # only the difference rotates
+        assert abs(a - b) < 1e-9 and abs(a - d) < 1e-9
+
+
+def _shifted_window(q, w, Lc, shift, base=10000.0):
+    out = RollingWindow(w.W)
+    for c in range(w.n_valid):
+        out.append(rope(w.k[c], shift + c * Lc + np.arange(Lc), base), w.v[c])
+    return rope(q, shift + (w.n_valid - 1) * Lc + np.arange(Lc), base), out
+
+
+def test_window_relative_rope_equals_any_common_shift():
+    # window-relative positions give the same pooled scores, masks and attention
+    # as positions shifted by any constant (e.g. absolute stream positions)
+    r = np.random.default_rng(4)
+    Lc, blk, D = 40, 8, 16
+    w = RollingWindow(3)
+    for _ in range(3):
+        w.append(r.standard_normal((1, Lc, 1, D)), r.standard_normal((1, Lc, 1, D)))
+    q = r.standard_normal((1, Lc, 2, D))
+    qa, wa = window_rope(q, w)
+    qb, wb = _shifted_window(q, w, Lc, shift=3 * 10 ** 6 + 17)
+    ma, mb = block_mask(qa, wa, blk, 4), block_mask(qb, wb, blk, 4)
+    assert np.allclose(ma["scores"], mb["scores"], atol=1e-9)
+    assert np.array_equal(ma["idx"], mb["idx"])
+    Oa, La = block_sparse_attention(qa, wa, blk, ma["idx"], ma["cnt"])
+    Ob, Lb = block_sparse_attention(qb, wb, blk, ma["idx"], ma["cnt"])
+    assert np.allclose(Oa, Ob, atol=1e-9) and np.allclose(La, Lb, atol=1e-9)
+
+
+def test_window_rope_positions_follow_the_window():
+    # after the window slides, chunk c of the window is rotated by c * Lc + r
+    r = np.random.default_rng(5)
+    Lc, D = 6, 4
+    w = RollingWindow(2)
+    chunks = [r.standard_normal((1, Lc, 1, D)) for _ in range(3)]
+    for ch in chunks:
+        w.append(ch, ch)
+    q = r.standard_normal((1, Lc, 1, D))
+    qr, wr = window_rope(q, w)
+    assert np.allclose(wr.k[0], rope(chunks[1], np.arange(Lc)))
+    assert np.allclose(wr.k[1], rope(chunks[2], Lc + np.arange(Lc)))
+    assert np.allclose(qr, rope(q, Lc + np.arange(Lc)))
+    assert np.array_equal(wr.v[1], chunks[2])
