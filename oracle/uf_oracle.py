@@ -62,6 +62,7 @@ __all__ = [
     "block_sparse_attention",
     "rope",
     "window_rope",
+    "round_bf16",
 ]
 
 
@@ -320,7 +321,20 @@ def rope(x: np.ndarray, pos: np.ndarray, base: float = 10000.0) -> np.ndarray:
     return out
 
 
-def window_rope(q: np.ndarray, window: RollingWindow, base: float = 10000.0):
+def round_bf16(x: np.ndarray) -> np.ndarray:
+    """float64 -> nearest bfloat16 value (ties to even), returned as float64:
+    the rounding a bf16 store applies.  bf16 keeps 8 significant bits, so the
+    grid spacing at x is 2^(floor(log2|x|) - 7); np.round rounds halves to
+    even.  (Inputs here are far from the bf16 range limits.)"""
+    x = np.asarray(x, dtype=np.float64)
+    ax = np.abs(x)
+    e = np.floor(np.log2(np.where(ax > 0, ax, 1.0)))
+    ulp = np.exp2(e - 7)
+    return np.where(ax > 0, np.round(x / ulp) * ulp, 0.0)
+
+
+def window_rope(q: np.ndarray, window: RollingWindow, base: float = 10000.0, shift: int = 0,
+                to_bf16: bool = False):
     """The window and the newest chunk's queries with RoPE at window-relative
     positions (FlashDecoder, "long video decoding": RoPE positions are assigned
     relative to the current window, not by absolute frame index): token r of
@@ -328,11 +342,17 @@ def window_rope(q: np.ndarray, window: RollingWindow, base: float = 10000.0):
     chunk (the newest) sits at (n_valid - 1) * Lc + r.  Returns (q_rot, a new
     RollingWindow holding the rotated K and the unchanged V), ready for
     block_mask and block_sparse_attention.
+
+    ``shift`` adds a common offset to every position (rotary scores depend
+    only on position differences, so exact results do not change); with
+    ``to_bf16`` the rotated values are rounded to bf16 as a bf16 cache stores
+    them.  Together they give the rotated values a stream-position cache holds.
     """
     Lc = q.shape[1]
     n = window.n_valid
     out = RollingWindow(window.W)
+    fin = round_bf16 if to_bf16 else (lambda a: a)
     for c in range(n):
-        out.append(rope(window.k[c], c * Lc + np.arange(Lc), base), window.v[c])
-    q_rot = rope(q, (n - 1) * Lc + np.arange(Lc), base)
+        out.append(fin(rope(window.k[c], shift + c * Lc + np.arange(Lc), base)), window.v[c])
+    q_rot = fin(rope(q, shift + (n - 1) * Lc + np.arange(Lc), base))
     return q_rot, out

@@ -567,3 +567,30 @@ def test_window_rope_positions_follow_the_window():
     assert np.allclose(wr.k[1], rope(chunks[2], Lc + np.arange(Lc)))
     assert np.allclose(qr, rope(q, Lc + np.arange(Lc)))
     assert np.array_equal(wr.v[1], chunks[2])
+
+
+def test_round_bf16_matches_torch_on_float32_values():
+    # from float32 values, torch's bf16 conversion (nearest even) is a single
+    # rounding, so it must agree exactly with the direct fp64 -> bf16 rounding
+    import torch
+    from oracle import round_bf16
+    r = np.random.default_rng(8)
+    x = (r.standard_normal(20000) * np.exp2(r.integers(-20, 20, 20000))).astype(np.float32)
+    ties = np.array([1.00390625, 1.01171875, -3.0078125, 257.0, 259.0], dtype=np.float32)   # exact halfway cases
+    x = np.concatenate([x, ties])
+    want = torch.from_numpy(x).to(torch.bfloat16).to(torch.float64).numpy()
+    assert np.array_equal(round_bf16(x.astype(np.float64)), want)
+    assert round_bf16(np.array([1.00390625]))[0] == 1.0 and round_bf16(np.array([1.01171875]))[0] == 1.015625
+
+
+def test_window_rope_shift_and_rounding():
+    from oracle import round_bf16
+    r = np.random.default_rng(9)
+    Lc, D = 8, 16
+    w = RollingWindow(2)
+    for _ in range(2):
+        w.append(r.standard_normal((1, Lc, 1, D)), r.standard_normal((1, Lc, 1, D)))
+    q = r.standard_normal((1, Lc, 1, D))
+    qs, ws = window_rope(q, w, shift=5 * Lc, to_bf16=True)
+    assert np.array_equal(ws.k[1], round_bf16(rope(w.k[1], 6 * Lc + np.arange(Lc))))
+    assert np.array_equal(qs, round_bf16(rope(q, 6 * Lc + np.arange(Lc))))
