@@ -104,6 +104,11 @@ def append_bytes(cfg):
     return 2 * chunk + 2 * slot + cfg.B * cfg.G * cfg.nb * cfg.D * 4
 
 
+def rope_q_bytes(cfg):
+    # uf_rope of the chunk's queries: read and write Q once (timed with the append)
+    return 2 * cfg.B * cfg.Lc * cfg.H * cfg.D * 2
+
+
 def mask_call_name(args):
     return "uf_block_mask_local + " if (args.mask_local or args.mask_local_only) else "uf_block_mask + "
 
@@ -207,28 +212,38 @@ def run_ours(args, cfg, rank, world, device):
     idx = [torch.empty(cfg.B, cfg.H, cfg.nb, k, dtype=torch.int32, device=device) for _ in range(n_idx)]
     cnt = [torch.empty(cfg.B, cfg.H, cfg.nb, dtype=torch.int32, device=device) for _ in range(n_idx)]
 
+    q_rot = torch.empty_like(dev_chunks[0]["q"]) if args.rope else None
+
     def step(s, chunk, ev=None):
+        # RoPE variant: the chunk sits at stream position (W + s) * Lc
+        pos0 = (cfg.W + s) * cfg.Lc
         if ev is not None:
             ev[0].record(stream)
-        win.append(chunk["k"], chunk["v"], keep_chunks=cfg.W)
+        if args.rope:
+            win.append(chunk["k"], chunk["v"], keep_chunks=cfg.W, rope_pos0=pos0)
+            uf.uf_rope(chunk["q"], q_rot, cfg.B, cfg.Lc, cfg.H, pos0)
+            q = q_rot
+        else:
+            win.append(chunk["k"], chunk["v"], keep_chunks=cfg.W)
+            q = chunk["q"]
         if ev is not None:
             ev[1].record(stream)
         if cfg.dense:
             if ev is not None:
                 ev[2].record(stream)
-            uf.uf_block_sparse_attn(chunk["q"], cfg.H, win.desc, None, None, 0, scale, o, lse)
+            uf.uf_block_sparse_attn(q, cfg.H, win.desc, None, None, 0, scale, o, lse)
         else:
             if args.mask_local or args.mask_local_only:
-                uf.uf_block_mask_local(chunk["q"], cfg.H, win.desc, k, args.mask_local, local_flags, idx[s], cnt[s])
+                uf.uf_block_mask_local(q, cfg.H, win.desc, k, args.mask_local, local_flags, idx[s], cnt[s])
             else:
-                uf.uf_block_mask(chunk["q"], cfg.H, win.desc, k, idx[s], cnt[s])
+                uf.uf_block_mask(q, cfg.H, win.desc, k, idx[s], cnt[s])
             if ev is not None:
                 ev[2].record(stream)
-            uf.uf_block_sparse_attn(chunk["q"], cfg.H, win.desc, idx[s], cnt[s], k, scale, o, lse)
+            uf.uf_block_sparse_attn(q, cfg.H, win.desc, idx[s], cnt[s], k, scale, o, lse)
         if ev is not None:
             ev[3].record(stream)
 
-    launches_per_step = 2 if cfg.dense else 3
+    launches_per_step = (2 if cfg.dense else 3) + (1 if args.rope else 0)
     for s in range(args.warmup):
         step(s, dev_chunks[cfg.W + s % n_distinct])
     torch.cuda.synchronize()
@@ -306,7 +321,8 @@ def run_ours(args, cfg, rank, world, device):
     traffic = attn_traffic_per_launch(args.config)
     hbm = peaks["hbm_gbs"]
     kernels = {
-        "append": {"ms": per["append"], "GB/s": append_bytes(cfg) / (per["append"] * 1e-3) / 1e9},
+        "append": {"ms": per["append"],
+                   "GB/s": (append_bytes(cfg) + (rope_q_bytes(cfg) if args.rope else 0)) / (per["append"] * 1e-3) / 1e9},
         "attn": {"ms": per["attn"], "TFLOP/s": attn_tflops},
     }
     kernels["append"]["frac_of_measured_hbm"] = kernels["append"]["GB/s"] / hbm
@@ -330,8 +346,9 @@ def run_ours(args, cfg, rank, world, device):
             "workload": args.config, "description": cfg.description, "B": cfg.B, "H": cfg.H, "G": cfg.G,
             "D": cfg.D, "Lc": cfg.Lc, "W": cfg.W, "blk": cfg.blk, "k": k,
             "density": cfg.density, "kept_flops_per_step": flops_per_step,
-            "mask_local": args.mask_local, "mask_local_only": bool(args.mask_local_only),
-            "step": "uf_kv_append + " + ("" if cfg.dense else mask_call_name(args)) + "uf_block_sparse_attn",
+            "mask_local": args.mask_local, "mask_local_only": bool(args.mask_local_only), "rope": bool(args.rope),
+            "step": ("uf_kv_append_rope + uf_rope + " if args.rope else "uf_kv_append + ")
+                    + ("" if cfg.dense else mask_call_name(args)) + "uf_block_sparse_attn",
             "l2": "no flush: every step's working set (%.0f MB) exceeds the 126 MB L2" % (
                 (cfg.B * cfg.Lc * (cfg.H * 2 + cfg.G * 2) * cfg.D * 2
                  + 2 * cfg.B * cfg.G * cfg.nkv() * cfg.blk * cfg.D * 2) / 1e6),
@@ -465,6 +482,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing leg")
     ap.add_argument("--mask-local", type=int, default=0,
                     help="radius of the forced local band of blocks around the diagonal (uf_block_mask_local)")
+    ap.add_argument("--rope", action="store_true",
+                    help="rotary position embedding: K rotated in the append, Q by uf_rope, at stream positions")
     ap.add_argument("--mask-local-only", action="store_true",
                     help="keep the local band only (the fixed-local-window mask)")
     args = ap.parse_args()

@@ -54,6 +54,8 @@ def _load() -> ctypes.CDLL:
         "uf_kv_cache_init": ([pc, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32], i32),
         "uf_kv_reset": ([pc, vp], i32),
         "uf_kv_append": ([pc, vp, vp, i32, i32, vp], i32),
+        "uf_kv_append_rope": ([pc, vp, vp, i32, i32, ctypes.c_int64, ctypes.c_float, vp], i32),
+        "uf_rope": ([vp, vp, i32, i32, i32, ctypes.c_int64, ctypes.c_float, vp], i32),
         "uf_block_mask": ([vp, i32, pc, i32, vp, vp, vp, vp], i32),
         "uf_block_mask_local": ([vp, i32, pc, i32, i32, i32, vp, vp, vp, vp], i32),
         "uf_block_sparse_attn": ([vp, i32, pc, vp, vp, i32, ctypes.c_float, vp, vp, vp], i32),
@@ -114,6 +116,16 @@ def uf_kv_reset(cache: UfKvCache, stream=None) -> None:
 def uf_kv_append(cache: UfKvCache, k_new, v_new, keep_chunks: int, flags: int = 0, stream=None) -> None:
     _check(lib.uf_kv_append(ctypes.byref(cache), _ptr(k_new), _ptr(v_new), keep_chunks, flags, _stream(stream)),
            "uf_kv_append")
+
+
+def uf_kv_append_rope(cache: UfKvCache, k_new, v_new, keep_chunks: int, flags: int, pos0: int,
+                      base: float = 10000.0, stream=None) -> None:
+    _check(lib.uf_kv_append_rope(ctypes.byref(cache), _ptr(k_new), _ptr(v_new), keep_chunks, flags, pos0, base,
+                                 _stream(stream)), "uf_kv_append_rope")
+
+
+def uf_rope(x, y, B: int, L: int, heads: int, pos0: int, base: float = 10000.0, stream=None) -> None:
+    _check(lib.uf_rope(_ptr(x), _ptr(y), B, L, heads, pos0, base, _stream(stream)), "uf_rope")
 
 
 def uf_block_mask(q, H: int, cache: UfKvCache, k: int, idx, cnt, scores=None, stream=None) -> None:

@@ -19,6 +19,13 @@
 // thread block to finish commits the new window state to meta; every block
 // read the old state before counting in, so no block can observe a
 // half-updated window.
+//
+// With RoPE (uf_kv_append_rope) each K row is rotated at its stream position
+// before it is stored and pooled.  Rotary scores depend only on position
+// differences, so stream positions give the same scores as the positions
+// relative to the current window that the method assigns (FlashDecoder, long
+// video decoding), and a stored K never needs rotating again when the window
+// slides.
 #pragma once
 
 #include "uf_device.cuh"
@@ -33,6 +40,8 @@ struct AppendParams {
   float *kpool;                // [B, G, W*nb, D]
   int32_t *meta;               // {start, n_valid, counter, reserved}
   int32_t G, W, Lc, nb, lslot, keep, replace;
+  long long pos0;              // RoPE variant: stream position of the chunk's first token
+  double log2_base;
 };
 
 // New window state and the slot the chunk goes to (see uf_kv_append).
@@ -98,7 +107,7 @@ __device__ __forceinline__ void transpose8x8_b16(const uint4 (&in)[8], uint4 (&o
   for (int c = 0; c < 8; ++c) out[c] = make_uint4(w[c][0], w[c][1], w[c][2], w[c][3]);
 }
 
-template <int BLK>
+template <int BLK, bool ROPE>
 __global__ void __launch_bounds__(256) kv_append_kernel(const AppendParams p) {
   constexpr int D = 128;
   constexpr int PASSES = BLK / 16;
@@ -156,6 +165,21 @@ __global__ void __launch_bounds__(256) kv_append_kernel(const AppendParams p) {
                                        : make_uint4(0, 0, 0, 0);
     }
   }
+  if (ROPE) {
+    // channels 8 dc .. 8 dc + 7 of this thread are the pairs 4 dc .. 4 dc + 3
+    double theta[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) theta[e] = rope_theta(4 * dc + e, D, p.log2_base);
+#pragma unroll
+    for (int m = 0; m < PASSES; ++m) {
+      const int t = tl + 16 * m;
+      if (t < cnt) {
+        float sn[4], cs[4];
+        rope_sincos4(p.pos0 + t0 + t, theta, sn, cs);
+        kr[m] = rope_rotate8(kr[m], sn, cs);
+      }
+    }
+  }
   float acc[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) acc[e] = 0.f;
@@ -211,6 +235,35 @@ __global__ void __launch_bounds__(256) kv_append_kernel(const AppendParams p) {
       atomicExch(p.meta + 1, s_plan[2]);
       atomicExch(p.meta + 2, 0);
       __threadfence();
+    }
+  }
+}
+
+}  // namespace uf
+
+namespace uf {
+
+// RoPE of a [B, L, heads, D] bf16 tensor, token t at stream position
+// pos0 + t (y may alias x).  One thread per (batch, token, 16-byte run of four
+// pairs): the angles depend on the token and the pairs only, so they are
+// formed once and applied to the run of every head.
+__global__ void __launch_bounds__(256) rope_kernel(const __nv_bfloat16 *x, __nv_bfloat16 *y, long long units,
+                                                   int32_t L, int32_t heads, long long pos0, double log2_base) {
+  constexpr int D = 128;
+  for (long long u = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; u < units;
+       u += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const int run = static_cast<int>(u & 15);              // 16 runs of 8 channels per row
+    const long long bt = u >> 4;                           // batch * L + token
+    const long long tok = bt % L;
+    double theta[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) theta[e] = rope_theta(4 * run + e, D, log2_base);
+    float sn[4], cs[4];
+    rope_sincos4(pos0 + tok, theta, sn, cs);
+    const size_t base_run = static_cast<size_t>(bt) * heads * 16 + run;
+    for (int h = 0; h < heads; ++h) {
+      const uint4 v = __ldg(reinterpret_cast<const uint4 *>(x) + base_run + 16 * h);
+      reinterpret_cast<uint4 *>(y)[base_run + 16 * h] = rope_rotate8(v, sn, cs);
     }
   }
 }

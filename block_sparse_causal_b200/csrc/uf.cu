@@ -146,6 +146,79 @@ std::atomic<int> g_attn128_smem[kMaxDevices], g_attn64_smem[kMaxDevices], g_mask
 
 }  // namespace
 
+namespace {
+
+// RoPE arguments: base > 1 and finite; positions in [0, kMaxRopePos): the
+// fp64 product pos * theta of a position below 2^40 is within 1.2e-4 rad.
+constexpr long long kMaxRopePos = 1LL << 40;
+bool rope_args_ok(long long pos0, float base) {
+  return pos0 >= 0 && pos0 < kMaxRopePos && isfinite(base) && base > 1.0f;
+}
+
+// uf_kv_append and uf_kv_append_rope (rope = 1: K rotated at pos0 + token).
+int32_t append_impl(uf_kv_cache *c, const void *k_new, const void *v_new, int32_t keep_chunks, int32_t flags,
+                    int32_t rope, long long pos0, double log2_base, uf_stream_t s) {
+  if (!cache_ok(c)) return UF_EINVAL;
+  if (!k_new || !v_new || !aligned16(k_new) || !aligned16(v_new)) return UF_EINVAL;
+  if (keep_chunks < 1 || keep_chunks > c->W) return UF_EINVAL;
+  if (flags & ~UF_APPEND_REPLACE_NEWEST) return UF_EINVAL;
+  const int32_t replace = (flags & UF_APPEND_REPLACE_NEWEST) ? 1 : 0;
+  if (replace && c->host_n_valid == 0) return UF_EINVAL;
+
+  uf::AppendParams p;
+  p.k_new = static_cast<const __nv_bfloat16 *>(k_new);
+  p.v_new = static_cast<const __nv_bfloat16 *>(v_new);
+  p.k = static_cast<__nv_bfloat16 *>(c->k);
+  p.v = static_cast<__nv_bfloat16 *>(c->v);
+  p.kpool = c->kpool;
+  p.meta = c->meta;
+  p.G = c->G;
+  p.W = c->W;
+  p.Lc = c->Lc;
+  p.nb = ceil_div(c->Lc, c->blk);
+  p.lslot = p.nb * c->blk;
+  p.keep = keep_chunks;
+  p.replace = replace;
+  p.pos0 = pos0;
+  p.log2_base = log2_base;
+  const dim3 grid(p.nb, c->G, c->B);
+  cudaGetLastError();
+  const cudaStream_t st0 = reinterpret_cast<cudaStream_t>(s);
+  if (c->blk == 128) {
+    if (rope)
+      uf::kv_append_kernel<128, true><<<grid, 256, 0, st0>>>(p);
+    else
+      uf::kv_append_kernel<128, false><<<grid, 256, 0, st0>>>(p);
+  } else {
+    if (rope)
+      uf::kv_append_kernel<64, true><<<grid, 256, 0, st0>>>(p);
+    else
+      uf::kv_append_kernel<64, false><<<grid, 256, 0, st0>>>(p);
+  }
+  const int32_t st = launch_status();
+  if (st != UF_OK) return st;
+  // host mirror (same rule as the kernel)
+  int32_t start2, n2;
+  const int32_t start = c->host_start, n = c->host_n_valid, W = c->W, keep = keep_chunks;
+  if (replace && n > 0) {
+    start2 = start;
+    n2 = n;
+  } else {
+    const int32_t evict = n + 1 - keep > 0 ? n + 1 - keep : 0;
+    start2 = (start + evict) % W;
+    n2 = n - evict + 1;
+  }
+  if (n2 > keep) {
+    start2 = (start2 + (n2 - keep)) % W;
+    n2 = keep;
+  }
+  c->host_start = start2;
+  c->host_n_valid = n2;
+  return UF_OK;
+}
+
+}  // namespace
+
 extern "C" {
 
 int32_t uf_version(void) { return UF_VERSION; }
@@ -205,54 +278,35 @@ int32_t uf_kv_reset(uf_kv_cache *c, uf_stream_t s) {
 
 int32_t uf_kv_append(uf_kv_cache *c, const void *k_new, const void *v_new, int32_t keep_chunks, int32_t flags,
                      uf_stream_t s) {
-  if (!cache_ok(c)) return UF_EINVAL;
-  if (!k_new || !v_new || !aligned16(k_new) || !aligned16(v_new)) return UF_EINVAL;
-  if (keep_chunks < 1 || keep_chunks > c->W) return UF_EINVAL;
-  if (flags & ~UF_APPEND_REPLACE_NEWEST) return UF_EINVAL;
-  const int32_t replace = (flags & UF_APPEND_REPLACE_NEWEST) ? 1 : 0;
-  if (replace && c->host_n_valid == 0) return UF_EINVAL;
-
-  uf::AppendParams p;
-  p.k_new = static_cast<const __nv_bfloat16 *>(k_new);
-  p.v_new = static_cast<const __nv_bfloat16 *>(v_new);
-  p.k = static_cast<__nv_bfloat16 *>(c->k);
-  p.v = static_cast<__nv_bfloat16 *>(c->v);
-  p.kpool = c->kpool;
-  p.meta = c->meta;
-  p.G = c->G;
-  p.W = c->W;
-  p.Lc = c->Lc;
-  p.nb = ceil_div(c->Lc, c->blk);
-  p.lslot = p.nb * c->blk;
-  p.keep = keep_chunks;
-  p.replace = replace;
-  const dim3 grid(p.nb, c->G, c->B);
-  cudaGetLastError();
-  if (c->blk == 128)
-    uf::kv_append_kernel<128><<<grid, 256, 0, reinterpret_cast<cudaStream_t>(s)>>>(p);
-  else
-    uf::kv_append_kernel<64><<<grid, 256, 0, reinterpret_cast<cudaStream_t>(s)>>>(p);
-  const int32_t st = launch_status();
-  if (st != UF_OK) return st;
-  // host mirror (same rule as the kernel)
-  int32_t start2, n2;
-  const int32_t start = c->host_start, n = c->host_n_valid, W = c->W, keep = keep_chunks;
-  if (replace && n > 0) {
-    start2 = start;
-    n2 = n;
-  } else {
-    const int32_t evict = n + 1 - keep > 0 ? n + 1 - keep : 0;
-    start2 = (start + evict) % W;
-    n2 = n - evict + 1;
-  }
-  if (n2 > keep) {
-    start2 = (start2 + (n2 - keep)) % W;
-    n2 = keep;
-  }
-  c->host_start = start2;
-  c->host_n_valid = n2;
-  return UF_OK;
+  return append_impl(c, k_new, v_new, keep_chunks, flags, 0, 0, 0.0, s);
 }
+
+int32_t uf_kv_append_rope(uf_kv_cache *c, const void *k_new, const void *v_new, int32_t keep_chunks,
+                          int32_t flags, int64_t pos0, float base, uf_stream_t s) {
+  if (!rope_args_ok(pos0, base)) return UF_EINVAL;
+  if (c && pos0 > kMaxRopePos - c->Lc) return UF_EINVAL;
+  return append_impl(c, k_new, v_new, keep_chunks, flags, 1, pos0, log2(static_cast<double>(base)), s);
+}
+
+int32_t uf_rope(const void *x, void *y, int32_t B, int32_t L, int32_t heads, int64_t pos0, float base,
+                uf_stream_t s) {
+  if (!x || !y || !aligned16(x) || !aligned16(y)) return UF_EINVAL;
+  if (B < 1 || L < 1 || heads < 1) return UF_EINVAL;
+  if (!rope_args_ok(pos0, base) || pos0 > kMaxRopePos - L) return UF_EINVAL;
+  const long long units = static_cast<long long>(B) * L * 16;   // (batch, token, run); heads loop inside
+  if (static_cast<long long>(B) * L * heads > (1LL << 40)) return UF_EINVAL;
+  int sms = 0;
+  const int32_t se = sm_count(&sms);
+  if (se != UF_OK) return se;
+  const long long want = (units + 255) / 256;
+  const unsigned grid = static_cast<unsigned>(want < 8LL * sms ? want : 8LL * sms);
+  cudaGetLastError();
+  uf::rope_kernel<<<grid, 256, 0, reinterpret_cast<cudaStream_t>(s)>>>(
+      static_cast<const __nv_bfloat16 *>(x), static_cast<__nv_bfloat16 *>(y), units, L, heads, pos0,
+      log2(static_cast<double>(base)));
+  return launch_status();
+}
+
 
 int32_t uf_block_mask(const void *q, int32_t H, const uf_kv_cache *c, int32_t k, int32_t *idx, int32_t *cnt,
                       float *scores, uf_stream_t s) {

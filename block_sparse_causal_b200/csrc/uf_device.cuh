@@ -297,6 +297,46 @@ __device__ __forceinline__ void warpgroup_reg_raise() {
   asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
 }
 
+// ------------------------------------------------------------ RoPE ----------
+// Rotary position embedding (RoFormer, Su et al. 2021): channel pairs
+// (x_2i, x_2i+1) of a D-channel row rotate by pos * theta_i, with
+// theta_i = base^(-2i / D).  The angle is formed and reduced to [-pi, pi] in
+// fp64 (positions are integers that can grow with a stream), then its sine and
+// cosine come from the fast fp32 intrinsic (absolute error ~2^-21 on
+// [-pi, pi], far below a bf16 step).
+__device__ __forceinline__ double rope_theta(int pair, int D, double log2_base) {
+  return exp2(-2.0 * static_cast<double>(pair) / static_cast<double>(D) * log2_base);
+}
+
+__device__ __forceinline__ void rope_sincos(long long pos, double theta, float &sn, float &cs) {
+  const double two_pi_hi = 6.283185307179586;             // 2 pi rounded to double
+  const double two_pi_lo = 2.4492935982947064e-16;        // 2 pi - two_pi_hi
+  const double a = static_cast<double>(pos) * theta;
+  const double k = rint(a * (1.0 / 6.283185307179586));
+  const double r = fma(-k, two_pi_lo, fma(-k, two_pi_hi, a));
+  __sincosf(static_cast<float>(r), &sn, &cs);
+}
+
+// Sine and cosine of the four pairs of one 16-byte run at position pos.
+__device__ __forceinline__ void rope_sincos4(long long pos, const double (&theta)[4], float (&sn)[4],
+                                             float (&cs)[4]) {
+#pragma unroll
+  for (int e = 0; e < 4; ++e) rope_sincos(pos, theta[e], sn[e], cs[e]);
+}
+
+// Four consecutive pairs (eight bf16 channels, one 16-byte run) rotated by
+// their angles (sine / cosine given); the result rounded to bf16 (nearest even).
+__device__ __forceinline__ uint4 rope_rotate8(uint4 v, const float (&sn)[4], const float (&cs)[4]) {
+  uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w[e]));
+    const __nv_bfloat162 r = __floats2bfloat162_rn(f.x * cs[e] - f.y * sn[e], f.x * sn[e] + f.y * cs[e]);
+    w[e] = *reinterpret_cast<const uint32_t *>(&r);
+  }
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t *>(&v);

@@ -33,6 +33,13 @@ class KVWindow:
     def reset(self, stream=None) -> None:
         _uf.uf_kv_reset(self.desc, stream)
 
-    def append(self, k_new, v_new, keep_chunks: int | None = None, replace_newest: bool = False, stream=None):
-        _uf.uf_kv_append(self.desc, k_new, v_new, self.W if keep_chunks is None else keep_chunks,
-                         _uf.UF_APPEND_REPLACE_NEWEST if replace_newest else 0, stream)
+    def append(self, k_new, v_new, keep_chunks: int | None = None, replace_newest: bool = False, stream=None,
+               rope_pos0: int | None = None, rope_base: float = 10000.0):
+        """Append the chunk's K and V (uf_kv_append); with ``rope_pos0``, K is
+        rotated at stream positions rope_pos0 + token (uf_kv_append_rope)."""
+        keep = self.W if keep_chunks is None else keep_chunks
+        flags = _uf.UF_APPEND_REPLACE_NEWEST if replace_newest else 0
+        if rope_pos0 is None:
+            _uf.uf_kv_append(self.desc, k_new, v_new, keep, flags, stream)
+        else:
+            _uf.uf_kv_append_rope(self.desc, k_new, v_new, keep, flags, rope_pos0, rope_base, stream)

@@ -4,6 +4,8 @@
  * Three calls make up one attention layer of a streaming video DiT, per chunk:
  *
  *   uf_kv_append         rolling-window append / evict of the new chunk's K and V
+ *                        (uf_kv_append_rope / uf_rope: with rotary position
+ *                        embedding of K and of the queries)
  *   uf_block_mask        per-head block mean-pooling of Q and K, pooled block
  *                        scores, top-k block selection with the diagonal kept
  *                        (uf_block_mask_local: with a forced local band of
@@ -147,6 +149,38 @@ int32_t uf_kv_reset(uf_kv_cache *c, uf_stream_t s);
  */
 int32_t uf_kv_append(uf_kv_cache *c, const void *k_new, const void *v_new,
                      int32_t keep_chunks, int32_t flags, uf_stream_t s);
+
+/*
+ * Rotary position embedding with positions relative to the window
+ * (FlashDecoder, long video decoding: RoPE positions are assigned relative to
+ * the current window rather than the absolute frame index; Algorithm 1:
+ * "RoPE offset t * L_frm").  The pages do not give the rotation's form; it is
+ * RoFormer's (Su et al. 2021): channel pairs (x_2i, x_2i+1) rotate by
+ * pos * theta_i, theta_i = base^(-2i / D).
+ *
+ * Rotary scores q(m) . k(n) depend only on m - n, and so do the pooled block
+ * scores, so rotating every token at its position in the stream gives the
+ * scores of window-relative positions exactly (up to rounding), and a stored
+ * key never has to be rotated again when the window slides.  The caller gives
+ * each chunk's stream position pos0 (e.g. chunk number * Lc) to both calls:
+ *
+ *   uf_kv_append_rope  uf_kv_append whose K rows are rotated at pos0 + token
+ *                      (token = 0 .. Lc-1 within the chunk) before they are
+ *                      stored and pooled; V is stored as is.
+ *   uf_rope            x, y device bf16 [B, L, heads, D]: y = RoPE(x) with
+ *                      token t at pos0 + t (y may be x: in place); for the
+ *                      queries of the newest chunk, pos0 = that chunk's pos0.
+ *
+ * pos0 >= 0 and pos0 + Lc (resp. L) <= 2^40; base > 1 and finite (10000 is
+ * RoFormer's).  Angles are formed and reduced in fp64 (within 1.2e-4 rad below
+ * 2^40), sine / cosine in fp32, results rounded to bf16 (nearest even).  UF_EINVAL on bad arguments,
+ * otherwise as uf_kv_append.  One kernel launch each.
+ */
+int32_t uf_kv_append_rope(uf_kv_cache *c, const void *k_new, const void *v_new,
+                          int32_t keep_chunks, int32_t flags, int64_t pos0, float base,
+                          uf_stream_t s);
+int32_t uf_rope(const void *x, void *y, int32_t B, int32_t L, int32_t heads, int64_t pos0,
+                float base, uf_stream_t s);
 
 /*
  * Dynamic block mask of the newest chunk's queries (Ultra Flash notes, Method,

@@ -100,6 +100,18 @@ def test_calls_reject_bad_arguments_before_launch(uf):
         with pytest.raises(uf.UfError) as e:
             uf.uf_kv_append(c, k_new, vn, keep, flags, stream=0)
         assert e.value.status == uf.UF_EINVAL
+    # RoPE: negative or too large position, base <= 1 or not finite, misaligned or empty input
+    for pos0, base in [(-1, 10000.0), (1 << 40, 10000.0), (0, 1.0), (0, 0.5), (0, float("nan")), (0, float("inf"))]:
+        with pytest.raises(uf.UfError) as e:
+            uf.uf_kv_append_rope(c, kn, vn, 2, 0, pos0, base, stream=0)
+        assert e.value.status == uf.UF_EINVAL
+        with pytest.raises(uf.UfError) as e:
+            uf.uf_rope(q, q, 1, 4, 2, pos0, base, stream=0)
+        assert e.value.status == uf.UF_EINVAL
+    for args in [(FakeTensor(0x500008), q, 1, 4, 2), (q, q, 0, 4, 2), (q, q, 1, 0, 2), (q, q, 1, 4, 0)]:
+        with pytest.raises(uf.UfError) as e:
+            uf.uf_rope(*args, 0, 10000.0, stream=0)
+        assert e.value.status == uf.UF_EINVAL
     idx, cnt = FakeTensor(0x800000), FakeTensor(0x900000)
     # mask / attention on an empty window (host mirror) are rejected
     with pytest.raises(uf.UfError):
