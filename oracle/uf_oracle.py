@@ -80,6 +80,13 @@ class RollingWindow:
       computation of the same chunk (no eviction);
     * ``keep_chunks``: the window is cropped to at most ``keep_chunks`` chunks
       (oldest dropped first), ``1 <= keep_chunks <= W``.
+
+    HiStream (aipapers summary), innovation 2, anchor-guided sliding window:
+    one anchor key frame plus a small cache of neighbouring frames keeps the
+    attention context at a fixed size.  ``anchor=True`` on an empty window
+    pins the chunk as the window's first chunk: it is never evicted or
+    cropped, ``keep_chunks`` counts it (2..W afterwards), and eviction drops
+    the oldest of the other chunks.
     """
 
     def __init__(self, W: int):
@@ -88,12 +95,22 @@ class RollingWindow:
         self.W = W
         self.k: List[np.ndarray] = []
         self.v: List[np.ndarray] = []
+        self.anchored = False
 
     def append(self, k_new: np.ndarray, v_new: np.ndarray,
-               keep_chunks: Optional[int] = None, replace_newest: bool = False) -> None:
+               keep_chunks: Optional[int] = None, replace_newest: bool = False, anchor: bool = False) -> None:
         keep = self.W if keep_chunks is None else keep_chunks
         if not 1 <= keep <= self.W:
             raise ValueError("keep_chunks must be in [1, W]")
+        if anchor:
+            if self.k or replace_newest or self.W < 2:
+                raise ValueError("an anchor starts an empty window of W >= 2")
+            self.anchored = True
+            self.k.append(np.array(k_new, dtype=np.float64))
+            self.v.append(np.array(v_new, dtype=np.float64))
+            return
+        if self.anchored and keep < 2:
+            raise ValueError("keep_chunks counts the anchor and must leave room for one more chunk")
         if replace_newest:
             if not self.k:
                 raise ValueError("replace_newest on an empty window")
@@ -102,9 +119,10 @@ class RollingWindow:
         else:
             self.k.append(np.array(k_new, dtype=np.float64))
             self.v.append(np.array(v_new, dtype=np.float64))
+        first = 1 if self.anchored else 0          # the anchor is never dropped
         while len(self.k) > keep:
-            self.k.pop(0)
-            self.v.pop(0)
+            self.k.pop(first)
+            self.v.pop(first)
 
     @property
     def n_valid(self) -> int:

@@ -594,3 +594,69 @@ def test_window_rope_shift_and_rounding():
     qs, ws = window_rope(q, w, shift=5 * Lc, to_bf16=True)
     assert np.array_equal(ws.k[1], round_bf16(rope(w.k[1], 6 * Lc + np.arange(Lc))))
     assert np.array_equal(qs, round_bf16(rope(q, 6 * Lc + np.arange(Lc))))
+
+
+# ---------------------------------------------------------- anchor pins ------
+def _chunks(n, Lc=4, D=2):
+    return [np.full((1, Lc, 1, D), float(t)) for t in range(n)]
+
+
+def test_anchor_window_keeps_the_anchor_and_the_newest():
+    # HiStream's anchor-guided window: the anchor plus the W - 1 newest chunks
+    w = RollingWindow(3)
+    ch = _chunks(6)
+    w.append(ch[0], ch[0], anchor=True)
+    for t in range(1, 6):
+        w.append(ch[t], ch[t])
+    assert [c[0, 0, 0, 0] for c in w.k] == [0.0, 4.0, 5.0]
+    w.append(ch[1], ch[1], keep_chunks=2)                        # crop: the anchor stays
+    assert [c[0, 0, 0, 0] for c in w.k] == [0.0, 1.0]
+    w.append(ch[3], ch[3], keep_chunks=2, replace_newest=True)    # replace the newest, not the anchor
+    assert [c[0, 0, 0, 0] for c in w.k] == [0.0, 3.0]
+
+
+def test_anchor_alone_is_the_newest_chunk():
+    w = RollingWindow(2)
+    a, b = _chunks(2)
+    w.append(a, a, anchor=True)
+    w.append(b, b, replace_newest=True)                           # only the anchor: it is replaced
+    assert w.n_valid == 1 and w.k[0][0, 0, 0, 0] == 1.0 and w.anchored
+
+
+@pytest.mark.parametrize("bad", [dict(W=1), dict(nonempty=True), dict(replace=True)])
+def test_anchor_rejections(bad):
+    w = RollingWindow(bad.get("W", 3))
+    a = _chunks(1)[0]
+    if bad.get("nonempty"):
+        w.append(a, a)
+    with pytest.raises(ValueError):
+        w.append(a, a, anchor=True, replace_newest=bad.get("replace", False))
+
+
+def test_anchor_keep_must_leave_room():
+    w = RollingWindow(3)
+    a = _chunks(1)[0]
+    w.append(a, a, anchor=True)
+    with pytest.raises(ValueError):
+        w.append(a, a, keep_chunks=1)
+
+
+def test_dense_attention_over_anchored_window_is_plain_softmax():
+    # dense attention over the anchored window equals a softmax over the
+    # explicit concatenation anchor | recent chunks
+    r = np.random.default_rng(12)
+    Lc, blk, D = 12, 4, 8
+    w = RollingWindow(3)
+    ks = [r.standard_normal((1, Lc, 1, D)) for _ in range(5)]
+    vs = [r.standard_normal((1, Lc, 1, D)) for _ in range(5)]
+    w.append(ks[0], vs[0], anchor=True)
+    for t in range(1, 5):
+        w.append(ks[t], vs[t])
+    q = r.standard_normal((1, Lc, 1, D))
+    O, L = block_sparse_attention(q, w, blk)
+    K = np.concatenate([ks[0], ks[3], ks[4]], axis=1)[0, :, 0]
+    V = np.concatenate([vs[0], vs[3], vs[4]], axis=1)[0, :, 0]
+    s = q[0, :, 0] @ K.T / math.sqrt(D)
+    p = np.exp(s - s.max(axis=1, keepdims=True))
+    assert np.allclose(O[0, :, 0], (p @ V) / p.sum(axis=1, keepdims=True), atol=1e-12)
+    assert np.allclose(L[0, 0], np.log(np.exp(s).sum(axis=1)), atol=1e-12)
