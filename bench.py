@@ -204,8 +204,8 @@ def run_ours(args, cfg, rank, world, device):
     dev_chunks = [{n: x.to(device) for n, x in c.items()} for c in host_chunks]
     win = uf.KVWindow(cfg.B, cfg.G, cfg.W, cfg.Lc, cfg.blk, cfg.D, device=device)
     win.reset()
-    for t in range(cfg.W):                       # fill the window
-        win.append(dev_chunks[t]["k"], dev_chunks[t]["v"], keep_chunks=cfg.W)
+    for t in range(cfg.W):                       # fill the window (--anchor: the first chunk is pinned)
+        win.append(dev_chunks[t]["k"], dev_chunks[t]["v"], keep_chunks=cfg.W, anchor=bool(args.anchor and t == 0))
     o = torch.empty(cfg.B, cfg.Lc, cfg.H, cfg.D, dtype=torch.bfloat16, device=device)
     lse = torch.empty(cfg.B, cfg.H, cfg.Lc, dtype=torch.float32, device=device)
     n_idx = args.steps + args.warmup
@@ -347,6 +347,7 @@ def run_ours(args, cfg, rank, world, device):
             "D": cfg.D, "Lc": cfg.Lc, "W": cfg.W, "blk": cfg.blk, "k": k,
             "density": cfg.density, "kept_flops_per_step": flops_per_step,
             "mask_local": args.mask_local, "mask_local_only": bool(args.mask_local_only), "rope": bool(args.rope),
+            "anchor": bool(args.anchor),
             "step": ("uf_kv_append_rope + uf_rope + " if args.rope else "uf_kv_append + ")
                     + ("" if cfg.dense else mask_call_name(args)) + "uf_block_sparse_attn",
             "l2": "no flush: every step's working set (%.0f MB) exceeds the 126 MB L2" % (
@@ -380,7 +381,7 @@ class OracleSample:
     mask of one query head over the full window, then attention for up to
     ``n_items`` work items of that head.  Inputs are prepared once."""
 
-    def __init__(self, cfg, seed, local=0, local_only=False):
+    def __init__(self, cfg, seed, local=0, local_only=False, anchor=False):
         import oracle
         from workloads import to_f64
         self.oracle = oracle
@@ -388,8 +389,8 @@ class OracleSample:
         self.local, self.local_only = local, local_only
         chunks = [chunk_inputs(cfg, seed, t) for t in range(cfg.W)]
         self.win = oracle.RollingWindow(cfg.W)
-        for c in chunks:
-            self.win.append(to_f64(c["k"][:, :, 0:1]), to_f64(c["v"][:, :, 0:1]))
+        for t, c in enumerate(chunks):
+            self.win.append(to_f64(c["k"][:, :, 0:1]), to_f64(c["v"][:, :, 0:1]), anchor=anchor and t == 0)
         self.q = to_f64(chunks[-1]["q"][:, :, 0:1])
         self.k = cfg.k_for() if not cfg.dense else cfg.nkv()
         if not cfg.dense:
@@ -425,15 +426,15 @@ def blas_threads():
     return os.cpu_count()
 
 
-def cpu_baseline(cfg, seed, local=0, local_only=False):
-    flops, dt, desc = OracleSample(cfg, seed, local, local_only).run(n_items=10_000, budget_s=12.0)
+def cpu_baseline(cfg, seed, local=0, local_only=False, anchor=False):
+    flops, dt, desc = OracleSample(cfg, seed, local, local_only, anchor).run(n_items=10_000, budget_s=12.0)
     return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
             "sample": desc + f", {dt:.1f} s of fp64 numpy", "seconds": dt}
 
 
 def run_reference(args, cfg):
     # each step: the oracle on a bounded sample (one head's mask + 1 work item)
-    sample = OracleSample(cfg, args.seed, args.mask_local, args.mask_local_only)
+    sample = OracleSample(cfg, args.seed, args.mask_local, args.mask_local_only, args.anchor)
     for s in range(args.warmup):
         sample.run(n_items=1, budget_s=5.0, first_item=s)
     tot_f, tot_t = 0.0, 0.0
@@ -450,7 +451,8 @@ def run_reference(args, cfg):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": args.config, "description": cfg.description, "B": cfg.B, "H": cfg.H, "G": cfg.G,
                    "D": cfg.D, "Lc": cfg.Lc, "W": cfg.W, "blk": cfg.blk, "k": k, "density": cfg.density,
-                   "mask_local": args.mask_local, "mask_local_only": bool(args.mask_local_only)},
+                   "mask_local": args.mask_local, "mask_local_only": bool(args.mask_local_only),
+                   "anchor": bool(args.anchor)},
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
                          "sample": "per step: " + desc},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -482,6 +484,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing leg")
     ap.add_argument("--mask-local", type=int, default=0,
                     help="radius of the forced local band of blocks around the diagonal (uf_block_mask_local)")
+    ap.add_argument("--anchor", action="store_true",
+                    help="anchored window: the first chunk stays pinned, the others roll (W >= 2)")
     ap.add_argument("--rope", action="store_true",
                     help="rotary position embedding: K rotated in the append, Q by uf_rope, at stream positions")
     ap.add_argument("--mask-local-only", action="store_true",
@@ -510,7 +514,8 @@ def main():
         result = run_ours(args, cfg, rank, world, device)
         if rank == 0:
             if world == 1 and not args.no_cpu_baseline:
-                result["cpu_baseline"] = cpu_baseline(cfg, args.seed, args.mask_local, args.mask_local_only)
+                result["cpu_baseline"] = cpu_baseline(cfg, args.seed, args.mask_local, args.mask_local_only,
+                                                      args.anchor)
             else:
                 result["cpu_baseline"] = None
             print(json.dumps(result), flush=True)

@@ -4,7 +4,7 @@ The library is ``libuf.so`` (C ABI in include/uf.h); this package binds it
 with ctypes and adds a small owner of the window's device buffers.  Every step
 of the hot path runs in the CUDA kernels.
 """
-from ._uf import (UF_APPEND_REPLACE_NEWEST, UF_EBOUNDS, UF_ECUDA, UF_EINVAL, UF_ETIMEOUT, UF_EUNSUPPORTED,
+from ._uf import (UF_APPEND_ANCHOR, UF_APPEND_REPLACE_NEWEST, UF_EBOUNDS, UF_ECUDA, UF_EINVAL, UF_ETIMEOUT, UF_EUNSUPPORTED,
                   UF_MASK_LOCAL_ONLY, UF_OK, UfError, UfKvCache, strerror, uf_block_mask, uf_block_mask_local,
                   uf_block_sparse_attn, uf_debug_wait_timeout, uf_kv_append_rope, uf_rope,
                   uf_get_error, uf_kv_append, uf_kv_cache_bytes, uf_kv_cache_init, uf_kv_reset, uf_set_wait_limit,
@@ -12,7 +12,7 @@ from ._uf import (UF_APPEND_REPLACE_NEWEST, UF_EBOUNDS, UF_ECUDA, UF_EINVAL, UF_
 from .window import KVWindow
 
 __all__ = [
-    "UF_APPEND_REPLACE_NEWEST", "UF_EBOUNDS", "UF_ECUDA", "UF_EINVAL", "UF_ETIMEOUT", "UF_EUNSUPPORTED",
+    "UF_APPEND_ANCHOR", "UF_APPEND_REPLACE_NEWEST", "UF_EBOUNDS", "UF_ECUDA", "UF_EINVAL", "UF_ETIMEOUT", "UF_EUNSUPPORTED",
     "UF_MASK_LOCAL_ONLY", "UF_OK", "UfError", "UfKvCache", "strerror", "uf_block_mask", "uf_block_mask_local",
     "uf_block_sparse_attn", "uf_kv_append_rope", "uf_rope", "uf_debug_wait_timeout",
     "uf_get_error", "uf_kv_append", "uf_kv_cache_bytes", "uf_kv_cache_init", "uf_kv_reset", "uf_set_wait_limit",

@@ -14,6 +14,7 @@ _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libuf.so")
 
 UF_OK, UF_EINVAL, UF_ECUDA, UF_ETIMEOUT, UF_EBOUNDS, UF_EUNSUPPORTED = range(6)
 UF_APPEND_REPLACE_NEWEST = 1
+UF_APPEND_ANCHOR = 2
 UF_MASK_LOCAL_ONLY = 1
 
 
@@ -27,7 +28,7 @@ class UfKvCache(ctypes.Structure):
         ("meta", ctypes.c_void_p),
         ("B", ctypes.c_int32), ("G", ctypes.c_int32), ("D", ctypes.c_int32),
         ("W", ctypes.c_int32), ("Lc", ctypes.c_int32), ("blk", ctypes.c_int32),
-        ("host_start", ctypes.c_int32), ("host_n_valid", ctypes.c_int32),
+        ("host_start", ctypes.c_int32), ("host_n_valid", ctypes.c_int32), ("host_anchor", ctypes.c_int32),
     ]
 
 

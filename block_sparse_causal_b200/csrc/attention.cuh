@@ -101,18 +101,17 @@ struct AttnSmem {
 // Logical kv block j (0 <= j < n_valid * nb) of the window -> first row of its
 // tile in the cache and its number of true tokens.  Chunk c = j / nb comes
 // from a multiply-high by floor(2^32 / nb), which is at most one below the
-// quotient, and one correction step; the ring slot start + c (both below W)
-// wraps with one subtraction.  No divide instruction on the per-block path.
-__device__ __forceinline__ void kv_block_coords(int j, int start, int W, int nb, uint32_t nb_mul, int lslot,
-                                                int blk, int Lc, int &row, int &valid) {
+// quotient, and one correction step; the slot (window_slot) wraps with one
+// subtraction.  No divide instruction on the per-block path.
+__device__ __forceinline__ void kv_block_coords(int j, int start, int W, int anchor, int nb, uint32_t nb_mul,
+                                                int lslot, int blk, int Lc, int &row, int &valid) {
   int c = static_cast<int>(__umulhi(static_cast<uint32_t>(j), nb_mul));
   int r = j - c * nb;
   if (r >= nb) {
     ++c;
     r -= nb;
   }
-  int slot = start + c;
-  if (slot >= W) slot -= W;
+  const int slot = window_slot(c, start, W, anchor);
   row = slot * lslot + r * blk;
   valid = (r == nb - 1) ? (Lc - (nb - 1) * blk) : blk;
 }
@@ -179,8 +178,8 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // window state (written by the append call earlier on the stream)
-  const int start = __ldcg(p.meta + 0), n_valid = __ldcg(p.meta + 1);
-  const bool bad_meta = start < 0 || start >= p.W || n_valid < 1 || n_valid > p.W;
+  const int start = __ldcg(p.meta + 0), n_valid = __ldcg(p.meta + 1), anchor = __ldcg(p.meta + 3);
+  const bool bad_meta = !window_state_ok(start, n_valid, anchor, p.W);
   const int NKV = bad_meta ? 0 : n_valid * p.nb;
 
   if (threadIdx.x == 0) {
@@ -248,7 +247,7 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
             const int jb = attn_block(it, t, NKV, bad);
             if (bad) record_error(UF_EBOUNDS);
             int row, valid;
-            kv_block_coords(jb, start, p.W, p.nb, p.nb_mul, p.lslot, BLK, p.Lc, row, valid);
+            kv_block_coords(jb, start, p.W, anchor, p.nb, p.nb_mul, p.lslot, BLK, p.Lc, row, valid);
             uint64_t *full = &full_bars[stage];
             mbar_arrive_expect_tx(full, L::STAGE);
             uint8_t *dst = ring + stage * L::STAGE;
@@ -499,7 +498,7 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
         bool bad;
         const int jb = attn_block(cur, t, NKV, bad);
         int krow, valid;
-        kv_block_coords(jb, start, p.W, p.nb, p.nb_mul, p.lslot, BLK, p.Lc, krow, valid);
+        kv_block_coords(jb, start, p.W, anchor, p.nb, p.nb_mul, p.lslot, BLK, p.Lc, krow, valid);
         if (!(ok = wwait(&bar_s[x], (gb >> 1) & 1))) break;
         tc_fence_after();
         const bool full = valid == BLK;

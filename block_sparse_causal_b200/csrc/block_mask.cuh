@@ -75,7 +75,7 @@ __global__ void __launch_bounds__(256, 2) block_mask_kernel(const __grid_constan
   float *s_red = s_qpool + MASK_TQ * D;                 // [2][4][D]
   float *s_kt = s_red + 2 * 4 * D;                      // [KT][KSTRIDE]
   float *s_sc = s_kt + MASK_KT * MASK_KSTRIDE;          // [TQ][W*nb]
-  __shared__ int32_t s_meta[2];
+  __shared__ int32_t s_meta[3];
   __shared__ uint64_t bar_q[MASK_QBUF];
   __shared__ int32_t s_abort;
 
@@ -86,20 +86,22 @@ __global__ void __launch_bounds__(256, 2) block_mask_kernel(const __grid_constan
   const int nkv_max = p.W * p.nb;
 
   if (tid == 0) {
-    int32_t start = __ldcg(p.meta + 0), n = __ldcg(p.meta + 1);
-    if (start < 0 || start >= p.W || n < 1 || n > p.W) {
+    int32_t start = __ldcg(p.meta + 0), n = __ldcg(p.meta + 1), anc = __ldcg(p.meta + 3);
+    if (!window_state_ok(start, n, anc, p.W)) {
       record_error(UF_EBOUNDS);
       n = 0;
       start = 0;
+      anc = 0;
     }
     s_meta[0] = start;
     s_meta[1] = n;
+    s_meta[2] = anc;
     for (int q = 0; q < MASK_QBUF; ++q) mbar_init(&bar_q[q], 1);
     s_abort = 0;
     fence_mbar_init();
   }
   __syncthreads();
-  const int start = s_meta[0], n_valid = s_meta[1];
+  const int start = s_meta[0], n_valid = s_meta[1], anchor = s_meta[2];
   const int NKV = n_valid * p.nb;
   const int tq_count = min(MASK_TQ, p.nb - i0);
   if (n_valid == 0) {     // empty window: nothing to select
@@ -162,7 +164,7 @@ __global__ void __launch_bounds__(256, 2) block_mask_kernel(const __grid_constan
       v[it] = make_float4(0.f, 0.f, 0.f, 0.f);
       if (j < NKV) {
         const int c = j / p.nb, rr = j - c * p.nb;
-        const int slot = (start + c) % p.W;
+        const int slot = window_slot(c, start, p.W, anchor);
         v[it] = __ldg(reinterpret_cast<const float4 *>(kp_head + (static_cast<size_t>(slot) * p.nb + rr) * D) + (e & 31));
       }
     }

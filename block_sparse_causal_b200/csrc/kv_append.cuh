@@ -40,26 +40,42 @@ struct AppendParams {
   float *kpool;                // [B, G, W*nb, D]
   int32_t *meta;               // {start, n_valid, counter, reserved}
   int32_t G, W, Lc, nb, lslot, keep, replace;
+  int32_t make_anchor;         // pin this chunk as the window's anchor (window empty)
   long long pos0;              // RoPE variant: stream position of the chunk's first token
   double log2_base;
 };
 
-// New window state and the slot the chunk goes to (see uf_kv_append).
-__device__ __forceinline__ void append_plan(int32_t start, int32_t n, int32_t W, int32_t keep, int32_t replace,
-                                            int32_t &slot, int32_t &start2, int32_t &n2) {
+// New window state and the slot the chunk goes to (see uf_kv_append).  With
+// an anchor (window_slot), the rolling part is a ring of W - 1 slots holding
+// n - 1 chunks, keep counts the anchor, and the anchor itself is never
+// evicted or cropped.
+__host__ __device__ __forceinline__ void append_plan(int32_t start, int32_t n, int32_t W, int32_t keep,
+                                                     int32_t replace, int32_t anchor, int32_t make_anchor,
+                                                     int32_t &slot, int32_t &start2, int32_t &n2,
+                                                     int32_t &anchor2) {
+  if (make_anchor) {          // the first chunk of an anchored window
+    slot = W - 1;
+    start2 = 0;
+    n2 = 1;
+    anchor2 = 1;
+    return;
+  }
+  anchor2 = anchor;
+  const int32_t a = anchor ? 1 : 0;
+  const int32_t R = W - a, nr = n - a, keep_r = keep - a;   // ring size, ring chunks, ring keep
   if (replace && n > 0) {
-    slot = (start + n - 1) % W;
+    slot = nr > 0 ? (start + nr - 1) % R : W - 1;             // the newest chunk (the anchor when alone)
     start2 = start;
     n2 = n;
   } else {
-    slot = (start + n) % W;   // free: at most keep-1 <= W-1 chunks survive eviction
-    const int32_t evict = max(0, n + 1 - keep);
-    start2 = (start + evict) % W;
+    slot = (start + nr) % R;   // free: at most keep_r - 1 <= R - 1 ring chunks survive eviction
+    const int32_t evict = max(0, nr + 1 - keep_r);
+    start2 = (start + evict) % R;
     n2 = n - evict + 1;
   }
-  if (n2 > keep) {            // crop (replace with a smaller keep_chunks)
-    start2 = (start2 + (n2 - keep)) % W;
-    n2 = keep;
+  if (n2 - a > keep_r) {      // crop (replace with a smaller keep_chunks)
+    start2 = (start2 + (n2 - a - keep_r)) % R;
+    n2 = keep_r + a;
   }
 }
 
@@ -114,21 +130,24 @@ __global__ void __launch_bounds__(256) kv_append_kernel(const AppendParams p) {
   const int r = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, tl = tid >> 4, dc = tid & 15;
 
-  __shared__ int32_t s_plan[3];
+  __shared__ int32_t s_plan[4];
   __shared__ __align__(16) float s_red[16][D];
 
   if (tid == 0) {
-    int32_t start = __ldcg(p.meta + 0), n = __ldcg(p.meta + 1);
-    if (start < 0 || start >= p.W || n < 0 || n > p.W) {
+    int32_t start = __ldcg(p.meta + 0), n = __ldcg(p.meta + 1), anc = __ldcg(p.meta + 3);
+    const bool empty = n == 0 && anc == 0 && start >= 0 && start < p.W;
+    if (!empty && !window_state_ok(start, n, anc, p.W)) {
       record_error(UF_EBOUNDS);
       start = 0;
       n = 0;
+      anc = 0;
     }
-    int32_t slot, start2, n2;
-    append_plan(start, n, p.W, p.keep, p.replace, slot, start2, n2);
+    int32_t slot, start2, n2, anc2;
+    append_plan(start, n, p.W, p.keep, p.replace, anc, p.make_anchor, slot, start2, n2, anc2);
     s_plan[0] = slot;
     s_plan[1] = start2;
     s_plan[2] = n2;
+    s_plan[3] = anc2;
   }
   __syncthreads();
   const int slot = s_plan[0];
@@ -233,6 +252,7 @@ __global__ void __launch_bounds__(256) kv_append_kernel(const AppendParams p) {
     if (prev == total - 1) {
       atomicExch(p.meta + 0, s_plan[1]);
       atomicExch(p.meta + 1, s_plan[2]);
+      atomicExch(p.meta + 3, s_plan[3]);
       atomicExch(p.meta + 2, 0);
       __threadfence();
     }

@@ -161,9 +161,14 @@ int32_t append_impl(uf_kv_cache *c, const void *k_new, const void *v_new, int32_
   if (!cache_ok(c)) return UF_EINVAL;
   if (!k_new || !v_new || !aligned16(k_new) || !aligned16(v_new)) return UF_EINVAL;
   if (keep_chunks < 1 || keep_chunks > c->W) return UF_EINVAL;
-  if (flags & ~UF_APPEND_REPLACE_NEWEST) return UF_EINVAL;
+  if (flags & ~(UF_APPEND_REPLACE_NEWEST | UF_APPEND_ANCHOR)) return UF_EINVAL;
   const int32_t replace = (flags & UF_APPEND_REPLACE_NEWEST) ? 1 : 0;
+  const int32_t make_anchor = (flags & UF_APPEND_ANCHOR) ? 1 : 0;
   if (replace && c->host_n_valid == 0) return UF_EINVAL;
+  // an anchor starts an empty window of at least two slots; while one is
+  // pinned, keep_chunks counts it and must leave room for a recent chunk
+  if (make_anchor && (replace || c->host_n_valid != 0 || c->W < 2)) return UF_EINVAL;
+  if (!make_anchor && c->host_anchor && keep_chunks < 2) return UF_EINVAL;
 
   uf::AppendParams p;
   p.k_new = static_cast<const __nv_bfloat16 *>(k_new);
@@ -179,6 +184,7 @@ int32_t append_impl(uf_kv_cache *c, const void *k_new, const void *v_new, int32_
   p.lslot = p.nb * c->blk;
   p.keep = keep_chunks;
   p.replace = replace;
+  p.make_anchor = make_anchor;
   p.pos0 = pos0;
   p.log2_base = log2_base;
   const dim3 grid(p.nb, c->G, c->B);
@@ -197,21 +203,11 @@ int32_t append_impl(uf_kv_cache *c, const void *k_new, const void *v_new, int32_
   }
   const int32_t st = launch_status();
   if (st != UF_OK) return st;
-  // host mirror (same rule as the kernel)
-  int32_t start2, n2;
-  const int32_t start = c->host_start, n = c->host_n_valid, W = c->W, keep = keep_chunks;
-  if (replace && n > 0) {
-    start2 = start;
-    n2 = n;
-  } else {
-    const int32_t evict = n + 1 - keep > 0 ? n + 1 - keep : 0;
-    start2 = (start + evict) % W;
-    n2 = n - evict + 1;
-  }
-  if (n2 > keep) {
-    start2 = (start2 + (n2 - keep)) % W;
-    n2 = keep;
-  }
+  // host mirror (the kernel's rule)
+  int32_t slot2, start2, n2, anchor2;
+  uf::append_plan(c->host_start, c->host_n_valid, c->W, keep_chunks, replace, c->host_anchor, make_anchor, slot2,
+                  start2, n2, anchor2);
+  c->host_anchor = anchor2;
   c->host_start = start2;
   c->host_n_valid = n2;
   return UF_OK;
@@ -262,6 +258,7 @@ int32_t uf_kv_cache_init(uf_kv_cache *c, void *k, void *v, float *kpool, int32_t
   t.blk = blk;
   t.host_start = 0;
   t.host_n_valid = 0;
+  t.host_anchor = 0;
   if (!cache_ok(&t)) return UF_EINVAL;
   *c = t;
   return UF_OK;
@@ -273,6 +270,7 @@ int32_t uf_kv_reset(uf_kv_cache *c, uf_stream_t s) {
   if (st != UF_OK) return st;
   c->host_start = 0;
   c->host_n_valid = 0;
+  c->host_anchor = 0;
   return UF_OK;
 }
 

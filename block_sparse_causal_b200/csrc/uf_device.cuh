@@ -79,6 +79,29 @@ __device__ __forceinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, vol
   }
 }
 
+// ------------------------------------------------------------ window -------
+// Window state (meta): {start, n_valid, counter, anchor}.  Without an anchor
+// the W slots form one ring and logical chunk c (0 = oldest) lives in slot
+// (start + c) mod W.  With an anchor (HiStream, anchor-guided sliding window:
+// one pinned anchor frame plus a fixed number of recent frames), logical
+// chunk 0 is the anchor, pinned in slot W - 1, and chunks 1 .. n_valid - 1
+// form a ring over slots 0 .. W - 2: slot (start + c - 1) mod (W - 1).
+__device__ __forceinline__ int window_slot(int c, int start, int W, int anchor) {
+  if (anchor) {
+    if (c == 0) return W - 1;
+    const int s = start + c - 1;
+    return s >= W - 1 ? s - (W - 1) : s;
+  }
+  const int s = start + c;
+  return s >= W ? s - W : s;
+}
+
+// A window state the kernels accept.
+__device__ __forceinline__ bool window_state_ok(int start, int n_valid, int anchor, int W) {
+  if (anchor == 0) return start >= 0 && start < W && n_valid >= 1 && n_valid <= W;
+  return anchor == 1 && W >= 2 && start >= 0 && start < W - 1 && n_valid >= 1 && n_valid <= W;
+}
+
 // ------------------------------------------------------------ TMA -----------
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");

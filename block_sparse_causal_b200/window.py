@@ -34,11 +34,12 @@ class KVWindow:
         _uf.uf_kv_reset(self.desc, stream)
 
     def append(self, k_new, v_new, keep_chunks: int | None = None, replace_newest: bool = False, stream=None,
-               rope_pos0: int | None = None, rope_base: float = 10000.0):
+               rope_pos0: int | None = None, rope_base: float = 10000.0, anchor: bool = False):
         """Append the chunk's K and V (uf_kv_append); with ``rope_pos0``, K is
-        rotated at stream positions rope_pos0 + token (uf_kv_append_rope)."""
+        rotated at stream positions rope_pos0 + token (uf_kv_append_rope); with
+        ``anchor`` (empty window) the chunk becomes the pinned anchor."""
         keep = self.W if keep_chunks is None else keep_chunks
-        flags = _uf.UF_APPEND_REPLACE_NEWEST if replace_newest else 0
+        flags = (_uf.UF_APPEND_REPLACE_NEWEST if replace_newest else 0) | (_uf.UF_APPEND_ANCHOR if anchor else 0)
         if rope_pos0 is None:
             _uf.uf_kv_append(self.desc, k_new, v_new, keep, flags, stream)
         else:

@@ -58,6 +58,7 @@ typedef enum uf_status {
 
 /* Flags of uf_kv_append. */
 #define UF_APPEND_REPLACE_NEWEST 1
+#define UF_APPEND_ANCHOR 2
 
 /*
  * Rolling KV window ("cache") descriptor: plain data, caller-owned.
@@ -65,7 +66,12 @@ typedef enum uf_status {
  * Ring of W slots, each holding one chunk of Lslot tokens.  Logical chunk
  * c (0 = oldest of the window) lives in physical slot (start + c) % W; logical
  * kv block j of the window is block j % nb of logical chunk j / nb.  The
- * physical order is never visible through the API.
+ * physical order is never visible through the API.  Anchored window (HiStream,
+ * aipapers summary, innovation 2: one anchor key frame plus a small cache of
+ * neighbouring frames): after uf_kv_append(..., UF_APPEND_ANCHOR) on an empty
+ * window, logical chunk 0 is that anchor, pinned in slot W - 1 and never
+ * evicted or cropped, and chunks 1 .. n_valid - 1 are the most recent ones,
+ * on a ring over slots 0 .. W - 2 (slot (start + c - 1) % (W - 1)).
  *
  *   k      device bf16 [B, G, W * Lslot, D] (token rows).
  *   v      device bf16 [B, G, D, W * Lslot] (transposed: each channel holds
@@ -76,12 +82,12 @@ typedef enum uf_status {
  *   kpool  device fp32 [B, G, W * nb, D]: mean of K over the true tokens of
  *          each block of each slot, written by uf_kv_append, read by
  *          uf_block_mask (pooling K once per chunk instead of once per call).
- *   meta   device int32[4] = {start, n_valid, append_counter, reserved}.  The
+ *   meta   device int32[4] = {start, n_valid, append_counter, anchor}.  The
  *          window state lives on the device so that a captured sequence of
  *          calls stays correct when replayed.  Zeroed by uf_kv_reset.
- *   host_start, host_n_valid: host mirror of meta[0..1], updated by
- *          uf_kv_append / uf_kv_reset and used only for host-side argument
- *          checks.
+ *   host_start, host_n_valid, host_anchor: host mirror of meta[0], meta[1],
+ *          meta[3], updated by uf_kv_append / uf_kv_reset and used only for
+ *          host-side argument checks.
  *
  * Sources: FlashDecoder (xllm-io blog), Sec. 3, Eq. 4 (cache shape
  * B x G x (W_frm L_frm) x D_h under grouped-query attention) and Algorithm 1
@@ -95,7 +101,7 @@ typedef struct uf_kv_cache {
   float *kpool;
   int32_t *meta;
   int32_t B, G, D, W, Lc, blk;
-  int32_t host_start, host_n_valid;
+  int32_t host_start, host_n_valid, host_anchor;
 } uf_kv_cache;
 
 /* Library version: major * 10000 + minor * 100 + patch. */
@@ -140,6 +146,12 @@ int32_t uf_kv_reset(uf_kv_cache *c, uf_stream_t s);
  *                 (a recomputation of the same chunk) instead of appending.
  *                 Rejected (UF_EINVAL) when the host mirror says the window is
  *                 empty; on the device an empty window turns it into an append.
+ *                 Or UF_APPEND_ANCHOR: the chunk becomes the window's pinned
+ *                 anchor (the window must be empty and W >= 2; not combined
+ *                 with REPLACE_NEWEST).  While an anchor is pinned, keep_chunks
+ *                 counts it (2..W) and eviction / cropping remove the oldest
+ *                 of the other chunks; REPLACE_NEWEST on a window holding only
+ *                 the anchor overwrites the anchor.
  *
  * Writes the chunk into its ring slot of k (BLGD -> BGLD) and v (BLGD ->
  * BGDL),

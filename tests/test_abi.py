@@ -100,6 +100,19 @@ def test_calls_reject_bad_arguments_before_launch(uf):
         with pytest.raises(uf.UfError) as e:
             uf.uf_kv_append(c, k_new, vn, keep, flags, stream=0)
         assert e.value.status == uf.UF_EINVAL
+    # anchor: with replace, on a non-empty window, and keep_chunks 1 while an anchor is pinned
+    with pytest.raises(uf.UfError) as e:
+        uf.uf_kv_append(c, kn, vn, 2, uf.UF_APPEND_ANCHOR | uf.UF_APPEND_REPLACE_NEWEST, stream=0)
+    assert e.value.status == uf.UF_EINVAL
+    c.host_n_valid = 1
+    with pytest.raises(uf.UfError) as e:
+        uf.uf_kv_append(c, kn, vn, 2, uf.UF_APPEND_ANCHOR, stream=0)
+    assert e.value.status == uf.UF_EINVAL
+    c.host_anchor = 1
+    with pytest.raises(uf.UfError) as e:
+        uf.uf_kv_append(c, kn, vn, 1, 0, stream=0)
+    assert e.value.status == uf.UF_EINVAL
+    c.host_n_valid, c.host_anchor = 0, 0
     # RoPE: negative or too large position, base <= 1 or not finite, misaligned or empty input
     for pos0, base in [(-1, 10000.0), (1 << 40, 10000.0), (0, 1.0), (0, 0.5), (0, float("nan")), (0, float("inf"))]:
         with pytest.raises(uf.UfError) as e:

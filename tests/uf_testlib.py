@@ -37,10 +37,10 @@ class GpuStream:
         self.win.reset()
         self.device = device
 
-    def append(self, inp, keep=None, replace=False):
+    def append(self, inp, keep=None, replace=False, anchor=False):
         k = inp["k"].to(self.device)
         v = inp["v"].to(self.device)
-        self.win.append(k, v, keep_chunks=keep, replace_newest=replace)
+        self.win.append(k, v, keep_chunks=keep, replace_newest=replace, anchor=anchor)
 
     def mask(self, q_cpu, k: int, want_scores=True, local: int = 0, local_only: bool = False):
         cfg = self.cfg
@@ -76,10 +76,10 @@ class OracleStream:
         self.cfg = cfg
         self.windows = [oracle.RollingWindow(cfg.W) for _ in range(cfg.G)]
 
-    def append(self, inp, keep=None, replace=False):
+    def append(self, inp, keep=None, replace=False, anchor=False):
         for g, w in enumerate(self.windows):
             w.append(to_f64(inp["k"][:, :, g:g + 1]), to_f64(inp["v"][:, :, g:g + 1]),
-                     keep_chunks=keep, replace_newest=replace)
+                     keep_chunks=keep, replace_newest=replace, anchor=anchor)
 
     @property
     def n_valid(self):
