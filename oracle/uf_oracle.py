@@ -63,6 +63,9 @@ __all__ = [
     "rope",
     "window_rope",
     "round_bf16",
+    "tile_order",
+    "to_tile_order",
+    "from_tile_order",
 ]
 
 
@@ -374,3 +377,38 @@ def window_rope(q: np.ndarray, window: RollingWindow, base: float = 10000.0, shi
         out.append(fin(rope(window.k[c], shift + c * Lc + np.arange(Lc), base)), window.v[c])
     q_rot = fin(rope(q, shift + (n - 1) * Lc + np.arange(Lc), base))
     return q_rot, out
+
+
+# --------------------------------------------------------------------------
+# 3-D block token order
+# --------------------------------------------------------------------------
+def tile_order(T: int, Hg: int, Wg: int, tile: Tuple[int, int, int] = (2, 8, 8)) -> np.ndarray:
+    """Token order of a chunk cut into 3-D tiles (Ultra Flash notes, Method, key
+    design 3: the spatio-temporal token grid is divided into non-overlapping
+    (2, 8, 8) blocks).
+
+    The chunk's tokens are a (T, Hg, Wg) grid in row-major order (token
+    t * Hg * Wg + y * Wg + x).  Tiles of ``tile`` = (bt, by, bx) are taken in
+    row-major tile order, the tokens inside a tile in row-major order; tiles at
+    the grid's far edges are clipped.  Returns ``order`` with
+    order[p] = the row-major index of the token at position p of the tiled
+    order (a permutation of range(T * Hg * Wg)).
+    """
+    bt, by, bx = tile
+    t, y, x = np.meshgrid(np.arange(T), np.arange(Hg), np.arange(Wg), indexing="ij")
+    t, y, x = t.ravel(), y.ravel(), x.ravel()
+    # sort keys, most significant last for lexsort
+    keys = (x % bx, y % by, t % bt, x // bx, y // by, t // bt)
+    return np.lexsort(keys)
+
+
+def to_tile_order(x: np.ndarray, order: np.ndarray) -> np.ndarray:
+    """x [B, L, heads, D] in row-major token order -> tiled order."""
+    return x[:, order]
+
+
+def from_tile_order(x: np.ndarray, order: np.ndarray) -> np.ndarray:
+    """Inverse of to_tile_order."""
+    out = np.empty_like(x)
+    out[:, order] = x
+    return out

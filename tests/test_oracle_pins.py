@@ -11,7 +11,8 @@ import numpy as np
 import pytest
 
 from oracle import (RollingWindow, block_mask, block_ranges, block_scores, block_sparse_attention,
-                    pool_blocks, rope, select_blocks, window_blocks, window_rope)
+                    from_tile_order, pool_blocks, rope, select_blocks, tile_order, to_tile_order,
+                    window_blocks, window_rope)
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 rng = np.random.default_rng(1234)
@@ -660,3 +661,45 @@ def test_dense_attention_over_anchored_window_is_plain_softmax():
     p = np.exp(s - s.max(axis=1, keepdims=True))
     assert np.allclose(O[0, :, 0], (p @ V) / p.sum(axis=1, keepdims=True), atol=1e-12)
     assert np.allclose(L[0, 0], np.log(np.exp(s).sum(axis=1)), atol=1e-12)
+
+
+# ---------------------------------------------------------- tile order pins --
+
+def test_tile_order_worked_example():
+    # a 2 x 2 x 4 grid with (1, 2, 2) tiles, written out by hand:
+    # frame 0: rows [0 1 2 3], [4 5 6 7]; frame 1: rows [8 9 10 11], [12 13 14 15]
+    want = [0, 1, 4, 5, 2, 3, 6, 7, 8, 9, 12, 13, 10, 11, 14, 15]
+    assert tile_order(2, 2, 4, (1, 2, 2)).tolist() == want
+
+
+def test_tile_order_clipped_edges_worked_example():
+    # 1 x 3 x 3 grid, (1, 2, 2) tiles: tiles (0,0) {0,1,3,4}, (0,1) {2,5}, (1,0) {6,7}, (1,1) {8}
+    assert tile_order(1, 3, 3, (1, 2, 2)).tolist() == [0, 1, 3, 4, 2, 5, 6, 7, 8]
+
+
+@pytest.mark.parametrize("grid", [(3, 60, 104), (3, 30, 52), (1, 45, 80), (4, 16, 16), (3, 90, 156)])
+def test_tile_order_is_a_permutation_with_full_interior_tiles(grid):
+    T, Hg, Wg = grid
+    o = tile_order(T, Hg, Wg)
+    assert np.array_equal(np.sort(o), np.arange(T * Hg * Wg))
+    t, rem = np.divmod(o, Hg * Wg)
+    y, x = np.divmod(rem, Wg)
+    tile_id = (t // 2) * (-(-Hg // 8)) * (-(-Wg // 8)) + (y // 8) * (-(-Wg // 8)) + x // 8
+    assert np.all(np.diff(tile_id) >= 0)                   # tiles are contiguous runs, in tile order
+    # every full (2, 8, 8) tile is one run of 128 tokens spanning exactly 2 x 8 x 8
+    ids, starts, counts = np.unique(tile_id, return_index=True, return_counts=True)
+    full = counts == 128
+    for s0 in starts[full][:50]:
+        seg = slice(s0, s0 + 128)
+        assert np.ptp(t[seg]) == 1 and np.ptp(y[seg]) == 7 and np.ptp(x[seg]) == 7
+    if T % 2 == 0 and Hg % 8 == 0 and Wg % 8 == 0:
+        assert np.all(full)
+
+
+def test_tile_order_round_trip():
+    r = np.random.default_rng(13)
+    o = tile_order(3, 10, 12, (2, 4, 4))
+    x = r.standard_normal((2, 360, 3, 4))
+    y = to_tile_order(x, o)
+    assert np.array_equal(from_tile_order(y, o), x)
+    assert np.array_equal(y[:, 5], x[:, o[5]])
