@@ -204,15 +204,18 @@ def run_ours(args, cfg, rank, world, device):
     dev_chunks = [{n: x.to(device) for n, x in c.items()} for c in host_chunks]
     win = uf.KVWindow(cfg.B, cfg.G, cfg.W, cfg.Lc, cfg.blk, cfg.D, device=device)
     win.reset()
+    tile_grid = cfg.grid if args.tiled else None
     for t in range(cfg.W):                       # fill the window (--anchor: the first chunk is pinned)
-        win.append(dev_chunks[t]["k"], dev_chunks[t]["v"], keep_chunks=cfg.W, anchor=bool(args.anchor and t == 0))
+        win.append(dev_chunks[t]["k"], dev_chunks[t]["v"], keep_chunks=cfg.W, anchor=bool(args.anchor and t == 0),
+                   tile_grid=tile_grid)
     o = torch.empty(cfg.B, cfg.Lc, cfg.H, cfg.D, dtype=torch.bfloat16, device=device)
     lse = torch.empty(cfg.B, cfg.H, cfg.Lc, dtype=torch.float32, device=device)
     n_idx = args.steps + args.warmup
     idx = [torch.empty(cfg.B, cfg.H, cfg.nb, k, dtype=torch.int32, device=device) for _ in range(n_idx)]
     cnt = [torch.empty(cfg.B, cfg.H, cfg.nb, dtype=torch.int32, device=device) for _ in range(n_idx)]
 
-    q_rot = torch.empty_like(dev_chunks[0]["q"]) if args.rope else None
+    q_rot = torch.empty_like(dev_chunks[0]["q"]) if (args.rope or args.tiled) else None
+    o_tiled = torch.empty_like(o) if args.tiled else None
 
     def step(s, chunk, ev=None):
         # RoPE variant: the chunk sits at stream position (W + s) * Lc
@@ -223,6 +226,11 @@ def run_ours(args, cfg, rank, world, device):
             win.append(chunk["k"], chunk["v"], keep_chunks=cfg.W, rope_pos0=pos0)
             uf.uf_rope(chunk["q"], q_rot, cfg.B, cfg.Lc, cfg.H, pos0)
             q = q_rot
+        elif args.tiled:
+            # tiled token order: K and V gathered by the append, the queries permuted
+            win.append(chunk["k"], chunk["v"], keep_chunks=cfg.W, tile_grid=cfg.grid)
+            uf.uf_tile_tokens(chunk["q"], q_rot, cfg.B, cfg.grid, cfg.H)
+            q = q_rot
         else:
             win.append(chunk["k"], chunk["v"], keep_chunks=cfg.W)
             q = chunk["q"]
@@ -231,7 +239,7 @@ def run_ours(args, cfg, rank, world, device):
         if cfg.dense:
             if ev is not None:
                 ev[2].record(stream)
-            uf.uf_block_sparse_attn(q, cfg.H, win.desc, None, None, 0, scale, o, lse)
+            uf.uf_block_sparse_attn(q, cfg.H, win.desc, None, None, 0, scale, o_tiled if args.tiled else o, lse)
         else:
             if args.mask_local or args.mask_local_only:
                 uf.uf_block_mask_local(q, cfg.H, win.desc, k, args.mask_local, local_flags, idx[s], cnt[s])
@@ -239,11 +247,13 @@ def run_ours(args, cfg, rank, world, device):
                 uf.uf_block_mask(q, cfg.H, win.desc, k, idx[s], cnt[s])
             if ev is not None:
                 ev[2].record(stream)
-            uf.uf_block_sparse_attn(q, cfg.H, win.desc, idx[s], cnt[s], k, scale, o, lse)
+            uf.uf_block_sparse_attn(q, cfg.H, win.desc, idx[s], cnt[s], k, scale, o_tiled if args.tiled else o, lse)
         if ev is not None:
             ev[3].record(stream)
+        if args.tiled:                             # O back to row-major order (in the step, not in "attn")
+            uf.uf_tile_tokens(o_tiled, o, cfg.B, cfg.grid, cfg.H, inverse=True)
 
-    launches_per_step = (2 if cfg.dense else 3) + (1 if args.rope else 0)
+    launches_per_step = (2 if cfg.dense else 3) + (1 if args.rope else 0) + (2 if args.tiled else 0)
     for s in range(args.warmup):
         step(s, dev_chunks[cfg.W + s % n_distinct])
     torch.cuda.synchronize()
@@ -322,7 +332,8 @@ def run_ours(args, cfg, rank, world, device):
     hbm = peaks["hbm_gbs"]
     kernels = {
         "append": {"ms": per["append"],
-                   "GB/s": (append_bytes(cfg) + (rope_q_bytes(cfg) if args.rope else 0)) / (per["append"] * 1e-3) / 1e9},
+                   "GB/s": (append_bytes(cfg) + (rope_q_bytes(cfg) if (args.rope or args.tiled) else 0))
+                   / (per["append"] * 1e-3) / 1e9},
         "attn": {"ms": per["attn"], "TFLOP/s": attn_tflops},
     }
     kernels["append"]["frac_of_measured_hbm"] = kernels["append"]["GB/s"] / hbm
@@ -347,9 +358,11 @@ def run_ours(args, cfg, rank, world, device):
             "D": cfg.D, "Lc": cfg.Lc, "W": cfg.W, "blk": cfg.blk, "k": k,
             "density": cfg.density, "kept_flops_per_step": flops_per_step,
             "mask_local": args.mask_local, "mask_local_only": bool(args.mask_local_only), "rope": bool(args.rope),
-            "anchor": bool(args.anchor),
-            "step": ("uf_kv_append_rope + uf_rope + " if args.rope else "uf_kv_append + ")
-                    + ("" if cfg.dense else mask_call_name(args)) + "uf_block_sparse_attn",
+            "anchor": bool(args.anchor), "tiled": list(cfg.grid) if args.tiled else None,
+            "step": ("uf_kv_append_rope + uf_rope + " if args.rope else
+                     "uf_kv_append_tiled + uf_tile_tokens + " if args.tiled else "uf_kv_append + ")
+                    + ("" if cfg.dense else mask_call_name(args)) + "uf_block_sparse_attn"
+                    + (" + uf_tile_tokens (O)" if args.tiled else ""),
             "l2": "no flush: every step's working set (%.0f MB) exceeds the 126 MB L2" % (
                 (cfg.B * cfg.Lc * (cfg.H * 2 + cfg.G * 2) * cfg.D * 2
                  + 2 * cfg.B * cfg.G * cfg.nkv() * cfg.blk * cfg.D * 2) / 1e6),
@@ -486,6 +499,8 @@ def main():
                     help="radius of the forced local band of blocks around the diagonal (uf_block_mask_local)")
     ap.add_argument("--anchor", action="store_true",
                     help="anchored window: the first chunk stays pinned, the others roll (W >= 2)")
+    ap.add_argument("--tiled", action="store_true",
+                    help="(2,8,8) tile token order: K/V gathered by the append, Q and O permuted")
     ap.add_argument("--rope", action="store_true",
                     help="rotary position embedding: K rotated in the append, Q by uf_rope, at stream positions")
     ap.add_argument("--mask-local-only", action="store_true",
@@ -493,6 +508,8 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.rope and args.tiled:
+        ap.error("--rope and --tiled are separate variants")
     cfg = CONFIGS[args.config]
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

@@ -57,6 +57,8 @@ def _load() -> ctypes.CDLL:
         "uf_kv_append": ([pc, vp, vp, i32, i32, vp], i32),
         "uf_kv_append_rope": ([pc, vp, vp, i32, i32, ctypes.c_int64, ctypes.c_float, vp], i32),
         "uf_rope": ([vp, vp, i32, i32, i32, ctypes.c_int64, ctypes.c_float, vp], i32),
+        "uf_tile_tokens": ([vp, vp, i32, i32, i32, i32, i32, i32, i32, i32, i32, vp], i32),
+        "uf_kv_append_tiled": ([pc, vp, vp, i32, i32, i32, i32, i32, i32, i32, i32, vp], i32),
         "uf_block_mask": ([vp, i32, pc, i32, vp, vp, vp, vp], i32),
         "uf_block_mask_local": ([vp, i32, pc, i32, i32, i32, vp, vp, vp, vp], i32),
         "uf_block_sparse_attn": ([vp, i32, pc, vp, vp, i32, ctypes.c_float, vp, vp, vp], i32),
@@ -127,6 +129,18 @@ def uf_kv_append_rope(cache: UfKvCache, k_new, v_new, keep_chunks: int, flags: i
 
 def uf_rope(x, y, B: int, L: int, heads: int, pos0: int, base: float = 10000.0, stream=None) -> None:
     _check(lib.uf_rope(_ptr(x), _ptr(y), B, L, heads, pos0, base, _stream(stream)), "uf_rope")
+
+
+def uf_tile_tokens(x, y, B: int, grid, heads: int, tile=(2, 8, 8), inverse: bool = False, stream=None) -> None:
+    T, Hg, Wg = grid
+    _check(lib.uf_tile_tokens(_ptr(x), _ptr(y), B, T, Hg, Wg, heads, *tile, 1 if inverse else 0, _stream(stream)),
+           "uf_tile_tokens")
+
+
+def uf_kv_append_tiled(cache: UfKvCache, k_new, v_new, keep_chunks: int, flags: int, grid, tile=(2, 8, 8),
+                       stream=None) -> None:
+    _check(lib.uf_kv_append_tiled(ctypes.byref(cache), _ptr(k_new), _ptr(v_new), keep_chunks, flags, *grid, *tile,
+                                  _stream(stream)), "uf_kv_append_tiled")
 
 
 def uf_block_mask(q, H: int, cache: UfKvCache, k: int, idx, cnt, scores=None, stream=None) -> None:

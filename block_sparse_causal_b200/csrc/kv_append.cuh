@@ -32,6 +32,48 @@
 
 namespace uf {
 
+// ------------------------------------------------------------ tile order ----
+// Ultra Flash (papernotes notes), Method, key design 3: the spatio-temporal
+// token grid is cut into non-overlapping (2, 8, 8) blocks.  A chunk's tokens
+// form a (T, Hg, Wg) grid in row-major order; the tiled order takes tiles of
+// (bt, by, bx) in row-major tile order and the tokens inside each tile in
+// row-major order, with the tiles at the grid's far edges clipped.
+struct TileGrid {
+  int32_t T, Hg, Wg, bt, by, bx;
+};
+
+// Row-major token index -> position in the tiled order.
+__host__ __device__ __forceinline__ int32_t tile_pos(const TileGrid &g, int32_t token) {
+  const int32_t HW = g.Hg * g.Wg;
+  const int32_t t = token / HW, rem = token - t * HW;
+  const int32_t y = rem / g.Wg, x = rem - y * g.Wg;
+  const int32_t ti = t / g.bt, yi = y / g.by, xi = x / g.bx;
+  const int32_t st = min(g.bt, g.T - ti * g.bt), sy = min(g.by, g.Hg - yi * g.by), sx = min(g.bx, g.Wg - xi * g.bx);
+  // tokens before the tile: earlier slabs, earlier bands of this slab, earlier tiles of this band
+  const int32_t before = ti * g.bt * HW + st * yi * g.by * g.Wg + st * sy * xi * g.bx;
+  return before + ((t - ti * g.bt) * sy + (y - yi * g.by)) * sx + (x - xi * g.bx);
+}
+
+// Position in the tiled order -> row-major token index (inverse of tile_pos):
+// every slab but the last holds bt * Hg * Wg tokens, every band of a slab but
+// the last st * by * Wg, every tile of a band but the last st * sy * bx.
+__host__ __device__ __forceinline__ int32_t tile_token(const TileGrid &g, int32_t p) {
+  const int32_t HW = g.Hg * g.Wg;
+  const int32_t ti = p / (g.bt * HW);
+  int32_t r = p - ti * g.bt * HW;
+  const int32_t st = min(g.bt, g.T - ti * g.bt);
+  const int32_t yi = r / (st * g.by * g.Wg);
+  r -= yi * st * g.by * g.Wg;
+  const int32_t sy = min(g.by, g.Hg - yi * g.by);
+  const int32_t xi = r / (st * sy * g.bx);
+  r -= xi * st * sy * g.bx;
+  const int32_t sx = min(g.bx, g.Wg - xi * g.bx);
+  const int32_t dt = r / (sy * sx);
+  r -= dt * sy * sx;
+  const int32_t dy = r / sx, dx = r - dy * sx;
+  return (ti * g.bt + dt) * HW + (yi * g.by + dy) * g.Wg + xi * g.bx + dx;
+}
+
 struct AppendParams {
   const __nv_bfloat16 *k_new;  // [B, Lc, G, D]
   const __nv_bfloat16 *v_new;
@@ -42,6 +84,7 @@ struct AppendParams {
   int32_t G, W, Lc, nb, lslot, keep, replace;
   int32_t make_anchor;         // pin this chunk as the window's anchor (window empty)
   long long pos0;              // RoPE variant: stream position of the chunk's first token
+  TileGrid grid;               // tiled variant: the chunk's grid and tile
   double log2_base;
 };
 
@@ -123,7 +166,7 @@ __device__ __forceinline__ void transpose8x8_b16(const uint4 (&in)[8], uint4 (&o
   for (int c = 0; c < 8; ++c) out[c] = make_uint4(w[c][0], w[c][1], w[c][2], w[c][3]);
 }
 
-template <int BLK, bool ROPE>
+template <int BLK, bool ROPE, bool TILED>
 __global__ void __launch_bounds__(256) kv_append_kernel(const AppendParams p) {
   constexpr int D = 128;
   constexpr int PASSES = BLK / 16;
@@ -131,6 +174,7 @@ __global__ void __launch_bounds__(256) kv_append_kernel(const AppendParams p) {
   const int tid = threadIdx.x, tl = tid >> 4, dc = tid & 15;
 
   __shared__ int32_t s_plan[4];
+  __shared__ int32_t s_src[TILED ? BLK : 1];   // tiled variant: source token of each position of the block
   __shared__ __align__(16) float s_red[16][D];
 
   if (tid == 0) {
@@ -149,13 +193,18 @@ __global__ void __launch_bounds__(256) kv_append_kernel(const AppendParams p) {
     s_plan[2] = n2;
     s_plan[3] = anc2;
   }
+  if (TILED && tid < BLK && r * BLK + tid < p.Lc) s_src[tid] = tile_token(p.grid, r * BLK + tid);
   __syncthreads();
   const int slot = s_plan[0];
 
   const int t0 = r * BLK;
   const int cnt = min(BLK, p.Lc - t0);
   const size_t src_stride = static_cast<size_t>(p.G) * D;                       // elements per token
-  const __nv_bfloat16 *ksrc = p.k_new + (static_cast<size_t>(b) * p.Lc + t0) * src_stride + g * D + dc * 8;
+  // source token of position t0 + t of the chunk (tiled variant: gathered in tile order)
+  auto src_row = [&](int t) -> size_t {
+    const int tok = TILED ? s_src[t] : t0 + t;
+    return (static_cast<size_t>(b) * p.Lc + tok) * src_stride + g * D;
+  };
   const size_t dst_row0 = (static_cast<size_t>(b) * p.G + g) * p.W * p.lslot + static_cast<size_t>(slot) * p.lslot + t0;
   __nv_bfloat16 *kdst = p.k + dst_row0 * D + dc * 8;
 
@@ -163,7 +212,7 @@ __global__ void __launch_bounds__(256) kv_append_kernel(const AppendParams p) {
 #pragma unroll
   for (int m = 0; m < PASSES; ++m) {
     const int t = tl + 16 * m;
-    kr[m] = (t < cnt) ? __ldg(reinterpret_cast<const uint4 *>(ksrc + t * src_stride))
+    kr[m] = (t < cnt) ? __ldg(reinterpret_cast<const uint4 *>(p.k_new + src_row(t) + dc * 8))
                       : make_uint4(0, 0, 0, 0);   // padding rows of the chunk's last block
   }
   // V tile of this thread: tokens 8*tg .. 8*tg+7, channels 8*cg .. 8*cg+7
@@ -176,12 +225,11 @@ __global__ void __launch_bounds__(256) kv_append_kernel(const AppendParams p) {
     const int tile = tid + 256 * q;
     const int tg = tile % TG, cg = tile / TG;
     if (tile < vtiles) {
-      const __nv_bfloat16 *src =
-          p.v_new + (static_cast<size_t>(b) * p.Lc + t0 + 8 * tg) * src_stride + g * D + 8 * cg;
 #pragma unroll
       for (int e = 0; e < 8; ++e)
-        vr[q][e] = (8 * tg + e < cnt) ? __ldg(reinterpret_cast<const uint4 *>(src + e * src_stride))
-                                       : make_uint4(0, 0, 0, 0);
+        vr[q][e] = (8 * tg + e < cnt)
+                       ? __ldg(reinterpret_cast<const uint4 *>(p.v_new + src_row(8 * tg + e) + 8 * cg))
+                       : make_uint4(0, 0, 0, 0);
     }
   }
   if (ROPE) {
@@ -285,6 +333,32 @@ __global__ void __launch_bounds__(256) rope_kernel(const __nv_bfloat16 *x, __nv_
       const uint4 v = __ldg(reinterpret_cast<const uint4 *>(x) + base_run + 16 * h);
       reinterpret_cast<uint4 *>(y)[base_run + 16 * h] = rope_rotate8(v, sn, cs);
     }
+  }
+}
+
+}  // namespace uf
+
+namespace uf {
+
+// x, y [B, L = T * Hg * Wg, heads, D] bf16 (y must not alias x): y in tiled
+// order from row-major x (inverse = 0), or row-major y from tiled x
+// (inverse = 1).  One warp per token row (heads * D * 2 bytes, contiguous on
+// both sides): the position is mapped once, the lanes copy the row's 16-byte
+// pieces.
+__global__ void __launch_bounds__(256) tile_tokens_kernel(const uint4 *__restrict__ x, uint4 *__restrict__ y,
+                                                          long long rows, int32_t L, int32_t row_pieces,
+                                                          TileGrid g, int32_t inverse) {
+  const int lane = threadIdx.x & 31;
+  const long long warps = static_cast<long long>(gridDim.x) * (blockDim.x >> 5);
+  for (long long row = static_cast<long long>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); row < rows;
+       row += warps) {
+    const long long b = row / L;
+    const int32_t tok = static_cast<int32_t>(row - b * L);
+    const int32_t p = tile_pos(g, tok);
+    const long long src_row = inverse ? b * L + p : row;
+    const long long dst_row = inverse ? row : b * L + p;
+    for (int piece = lane; piece < row_pieces; piece += 32)
+      y[dst_row * row_pieces + piece] = __ldg(x + src_row * row_pieces + piece);
   }
 }
 

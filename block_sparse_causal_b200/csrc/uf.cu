@@ -157,7 +157,8 @@ bool rope_args_ok(long long pos0, float base) {
 
 // uf_kv_append and uf_kv_append_rope (rope = 1: K rotated at pos0 + token).
 int32_t append_impl(uf_kv_cache *c, const void *k_new, const void *v_new, int32_t keep_chunks, int32_t flags,
-                    int32_t rope, long long pos0, double log2_base, uf_stream_t s) {
+                    int32_t rope, long long pos0, double log2_base, uf_stream_t s,
+                    const uf::TileGrid *tile_grid = nullptr) {
   if (!cache_ok(c)) return UF_EINVAL;
   if (!k_new || !v_new || !aligned16(k_new) || !aligned16(v_new)) return UF_EINVAL;
   if (keep_chunks < 1 || keep_chunks > c->W) return UF_EINVAL;
@@ -187,19 +188,25 @@ int32_t append_impl(uf_kv_cache *c, const void *k_new, const void *v_new, int32_
   p.make_anchor = make_anchor;
   p.pos0 = pos0;
   p.log2_base = log2_base;
+  const bool tiled = tile_grid != nullptr;
+  if (tiled) p.grid = *tile_grid;
   const dim3 grid(p.nb, c->G, c->B);
   cudaGetLastError();
   const cudaStream_t st0 = reinterpret_cast<cudaStream_t>(s);
   if (c->blk == 128) {
     if (rope)
-      uf::kv_append_kernel<128, true><<<grid, 256, 0, st0>>>(p);
+      uf::kv_append_kernel<128, true, false><<<grid, 256, 0, st0>>>(p);
+    else if (tiled)
+      uf::kv_append_kernel<128, false, true><<<grid, 256, 0, st0>>>(p);
     else
-      uf::kv_append_kernel<128, false><<<grid, 256, 0, st0>>>(p);
+      uf::kv_append_kernel<128, false, false><<<grid, 256, 0, st0>>>(p);
   } else {
     if (rope)
-      uf::kv_append_kernel<64, true><<<grid, 256, 0, st0>>>(p);
+      uf::kv_append_kernel<64, true, false><<<grid, 256, 0, st0>>>(p);
+    else if (tiled)
+      uf::kv_append_kernel<64, false, true><<<grid, 256, 0, st0>>>(p);
     else
-      uf::kv_append_kernel<64, false><<<grid, 256, 0, st0>>>(p);
+      uf::kv_append_kernel<64, false, false><<<grid, 256, 0, st0>>>(p);
   }
   const int32_t st = launch_status();
   if (st != UF_OK) return st;
@@ -496,6 +503,47 @@ int32_t uf_debug_wait_timeout(int64_t cycles, uf_stream_t s) {
   cudaGetLastError();
   uf::wait_timeout_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(s)>>>(cycles);
   return launch_status();
+}
+
+// Tile-grid arguments: positive, L = T * Hg * Wg within int32, tile sides >= 1.
+static bool tile_grid_ok(int32_t T, int32_t Hg, int32_t Wg, int32_t bt, int32_t by, int32_t bx) {
+  if (T < 1 || Hg < 1 || Wg < 1 || bt < 1 || by < 1 || bx < 1) return false;
+  return static_cast<long long>(T) * Hg * Wg < (1LL << 30);
+}
+
+int32_t uf_tile_tokens(const void *x, void *y, int32_t B, int32_t T, int32_t Hg, int32_t Wg, int32_t heads,
+                       int32_t bt, int32_t by, int32_t bx, int32_t inverse, uf_stream_t s) {
+  if (!x || !y || x == y || !aligned16(x) || !aligned16(y)) return UF_EINVAL;
+  if (B < 1 || heads < 1 || (inverse != 0 && inverse != 1) || !tile_grid_ok(T, Hg, Wg, bt, by, bx))
+    return UF_EINVAL;
+  const int32_t L = T * Hg * Wg;
+  const long long row_bytes = static_cast<long long>(heads) * 128 * 2;
+  const long long pieces = static_cast<long long>(B) * L * (row_bytes / 16);
+  if (pieces / (row_bytes / 16) / L != B || row_bytes / 16 > (1LL << 30)) return UF_EINVAL;
+  const char *xe = static_cast<const char *>(x), *ye = static_cast<const char *>(y);
+  const long long bytes = pieces * 16;
+  if (xe < ye + bytes && ye < xe + bytes) return UF_EINVAL;      // overlapping buffers
+  int sms = 0;
+  const int32_t se = sm_count(&sms);
+  if (se != UF_OK) return se;
+  const long long rows = static_cast<long long>(B) * L;
+  const long long want = (rows + 7) / 8;                     // 8 warps (rows in flight) per block
+  const unsigned grid = static_cast<unsigned>(want < 16LL * sms ? want : 16LL * sms);
+  const uf::TileGrid g{T, Hg, Wg, bt, by, bx};
+  cudaGetLastError();
+  uf::tile_tokens_kernel<<<grid, 256, 0, reinterpret_cast<cudaStream_t>(s)>>>(
+      static_cast<const uint4 *>(x), static_cast<uint4 *>(y), rows, L, static_cast<int32_t>(row_bytes / 16), g,
+      inverse);
+  return launch_status();
+}
+
+int32_t uf_kv_append_tiled(uf_kv_cache *c, const void *k_new, const void *v_new, int32_t keep_chunks,
+                           int32_t flags, int32_t T, int32_t Hg, int32_t Wg, int32_t bt, int32_t by, int32_t bx,
+                           uf_stream_t s) {
+  if (!cache_ok(c) || !tile_grid_ok(T, Hg, Wg, bt, by, bx)) return UF_EINVAL;
+  if (static_cast<long long>(T) * Hg * Wg != c->Lc) return UF_EINVAL;
+  const uf::TileGrid g{T, Hg, Wg, bt, by, bx};
+  return append_impl(c, k_new, v_new, keep_chunks, flags, 0, 0, 0.0, s, &g);
 }
 
 }  // extern "C"

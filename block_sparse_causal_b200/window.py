@@ -34,13 +34,20 @@ class KVWindow:
         _uf.uf_kv_reset(self.desc, stream)
 
     def append(self, k_new, v_new, keep_chunks: int | None = None, replace_newest: bool = False, stream=None,
-               rope_pos0: int | None = None, rope_base: float = 10000.0, anchor: bool = False):
+               rope_pos0: int | None = None, rope_base: float = 10000.0, anchor: bool = False,
+               tile_grid=None, tile=(2, 8, 8)):
         """Append the chunk's K and V (uf_kv_append); with ``rope_pos0``, K is
         rotated at stream positions rope_pos0 + token (uf_kv_append_rope); with
-        ``anchor`` (empty window) the chunk becomes the pinned anchor."""
+        ``tile_grid`` = (T, Hg, Wg), K and V are stored in tiled token order
+        (uf_kv_append_tiled); with ``anchor`` (empty window) the chunk becomes
+        the pinned anchor."""
         keep = self.W if keep_chunks is None else keep_chunks
         flags = (_uf.UF_APPEND_REPLACE_NEWEST if replace_newest else 0) | (_uf.UF_APPEND_ANCHOR if anchor else 0)
-        if rope_pos0 is None:
+        if tile_grid is not None:
+            if rope_pos0 is not None:
+                raise ValueError("the tiled append does not rotate")
+            _uf.uf_kv_append_tiled(self.desc, k_new, v_new, keep, flags, tile_grid, tile, stream)
+        elif rope_pos0 is None:
             _uf.uf_kv_append(self.desc, k_new, v_new, keep, flags, stream)
         else:
             _uf.uf_kv_append_rope(self.desc, k_new, v_new, keep, flags, rope_pos0, rope_base, stream)

@@ -195,6 +195,35 @@ int32_t uf_rope(const void *x, void *y, int32_t B, int32_t L, int32_t heads, int
                 float base, uf_stream_t s);
 
 /*
+ * 3-D block token order (Ultra Flash notes, Method, key design 3: the
+ * spatio-temporal token grid is cut into non-overlapping (2, 8, 8) blocks).
+ * A chunk's Lc = T * Hg * Wg tokens form a (T, Hg, Wg) grid in row-major
+ * order; the tiled order takes tiles of (bt, by, bx) -- (2, 8, 8) on the
+ * pages -- in row-major tile order and the tokens inside each tile in
+ * row-major order, with the tiles at the grid's far edges clipped.  In the
+ * tiled order every full tile is one run of bt * by * bx tokens, so with
+ * blk = bt * by * bx the library's blocks are the pages' 3-D blocks wherever
+ * the grid allows.
+ *
+ *   uf_tile_tokens      x, y device bf16 [B, T * Hg * Wg, heads, D], not
+ *                       overlapping: inverse = 0 writes x in tiled order,
+ *                       inverse = 1 writes tiled x back in row-major order
+ *                       (for the queries before the mask and attention, and
+ *                       for O after).
+ *   uf_kv_append_tiled  uf_kv_append whose K and V rows are gathered in tiled
+ *                       order (T * Hg * Wg must equal Lc): the window holds
+ *                       the chunk in tiled order without a separate pass.
+ *
+ * UF_EINVAL on bad arguments.  One kernel launch each.
+ */
+int32_t uf_tile_tokens(const void *x, void *y, int32_t B, int32_t T, int32_t Hg, int32_t Wg,
+                       int32_t heads, int32_t bt, int32_t by, int32_t bx, int32_t inverse,
+                       uf_stream_t s);
+int32_t uf_kv_append_tiled(uf_kv_cache *c, const void *k_new, const void *v_new,
+                           int32_t keep_chunks, int32_t flags, int32_t T, int32_t Hg, int32_t Wg,
+                           int32_t bt, int32_t by, int32_t bx, uf_stream_t s);
+
+/*
  * Dynamic block mask of the newest chunk's queries (Ultra Flash notes, Method,
  * key design 3: tokens are cut into non-overlapping blocks; queries and keys
  * are mean-pooled per block; blocks are scored by the dot product of the

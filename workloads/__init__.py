@@ -24,7 +24,7 @@ from __future__ import annotations
 
 import dataclasses
 import math
-from typing import Dict, Optional
+from typing import Dict, Optional, Tuple
 
 import torch
 
@@ -47,6 +47,7 @@ class Config:
     offset_std: float = 0.5
     stream_len: int = 0        # frames in a rolling stream (GQA decoder config)
     description: str = ""
+    grid: Optional[Tuple[int, int, int]] = None   # the chunk's (frames, rows, cols) token grid, Lc = product
 
     @property
     def nb(self) -> int:
@@ -82,15 +83,18 @@ class Config:
 CONFIGS: Dict[str, Config] = {
     c.name: c
     for c in [
-        Config("tiny", B=1, H=2, G=2, D=128, Lc=256, W=2, blk=64, density=None, k_fixed=4,
+        Config("tiny", B=1, H=2, G=2, D=128, Lc=256, W=2, blk=64, density=None, k_fixed=4, grid=(1, 16, 16),
                description="1 latent frame of 16x16 tokens, window of 2 frames, block 64, top-4 of 8"),
-        Config("480p_dense", B=1, H=12, G=12, D=128, Lc=4680, W=3, blk=128, density=1.0,
+        Config("480p_dense", B=1, H=12, G=12, D=128, Lc=4680, W=3, blk=128, density=1.0, grid=(3, 30, 52),
                description="3 frames x 30x52 tokens, window of 3 chunks, dense"),
         Config("1k_sr", B=1, H=12, G=12, D=128, Lc=18720, W=2, blk=128, density=0.25, offsets=True,
+               grid=(3, 60, 104),
                description="3 frames x 60x104 tokens, window of 2 chunks, top-k density 25%"),
         Config("2k_sr", B=1, H=12, G=12, D=128, Lc=42120, W=2, blk=128, density=0.15, offsets=True,
+               grid=(3, 90, 156),
                description="3 frames x 90x156 tokens, window of 2 chunks, top-k density 15%"),
         Config("gqa_decoder", B=1, H=12, G=3, D=128, Lc=3600, W=2, blk=128, density=1.0, stream_len=16,
+               grid=(1, 45, 80),
                description="1 frame of 45x80 tokens, 12 q heads / 3 KV groups, rolling window of 2 frames"),
     ]
 }
