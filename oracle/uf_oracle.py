@@ -66,6 +66,9 @@ __all__ = [
     "tile_order",
     "to_tile_order",
     "from_tile_order",
+    "E4M3_MAX",
+    "quantize_e4m3",
+    "fp8_scores_attention",
 ]
 
 
@@ -412,3 +415,40 @@ def from_tile_order(x: np.ndarray, order: np.ndarray) -> np.ndarray:
     out = np.empty_like(x)
     out[:, order] = x
     return out
+
+
+# --------------------------------------------------------------------------
+# FP8 (e4m3) scores
+# --------------------------------------------------------------------------
+E4M3_MAX = 448.0
+
+
+def quantize_e4m3(x: np.ndarray, scale: float) -> np.ndarray:
+    """Static-scale FP8 quantisation (FlashDecoder, inference optimisations:
+    statically calibrated FP8): the e4m3 value nearest to x / scale (ties to
+    even; e4m3 keeps 4 significant bits, exponent bias 7, subnormal spacing
+    2^-9, saturating at +-448), returned in e4m3 units as float64."""
+    v = np.asarray(x, dtype=np.float64) / scale
+    a = np.abs(v)
+    e = np.floor(np.log2(np.where(a > 0, a, 1.0)))
+    ulp = np.exp2(np.maximum(e, -6.0) - 3.0)             # normal spacing 2^(e-3); below 2^-6 the subnormal 2^-9
+    q = np.round(v / ulp) * ulp
+    return np.clip(q, -E4M3_MAX, E4M3_MAX)
+
+
+def fp8_scores_attention(q: np.ndarray, window: RollingWindow, blk: int, q_scale: float, k_scale: float,
+                         idx: Optional[np.ndarray] = None, cnt: Optional[np.ndarray] = None,
+                         scale: Optional[float] = None,
+                         items: Optional[Sequence[Tuple[int, int, int]]] = None):
+    """block_sparse_attention with the scores taken from FP8 queries and keys:
+    q8 = quantize_e4m3(q, q_scale), k8 = quantize_e4m3(k, k_scale), and
+    s = scale * q_scale * k_scale * (q8 . k8); V and the softmax are as in
+    block_sparse_attention."""
+    w8 = RollingWindow(window.W)
+    w8.anchored = window.anchored
+    for kc, vc in zip(window.k, window.v):
+        w8.k.append(quantize_e4m3(kc, k_scale))
+        w8.v.append(vc)
+    D = q.shape[-1]
+    s0 = 1.0 / math.sqrt(D) if scale is None else scale
+    return block_sparse_attention(quantize_e4m3(q, q_scale), w8, blk, idx, cnt, s0 * q_scale * k_scale, items)

@@ -703,3 +703,38 @@ def test_tile_order_round_trip():
     y = to_tile_order(x, o)
     assert np.array_equal(from_tile_order(y, o), x)
     assert np.array_equal(y[:, 5], x[:, o[5]])
+
+
+# ------------------------------------------------------------- FP8 pins ------
+def test_quantize_e4m3_matches_torch_float8():
+    import torch
+    from oracle import quantize_e4m3
+    r = np.random.default_rng(14)
+    x = (r.standard_normal(50000) * np.exp2(r.integers(-12, 8, 50000))).astype(np.float32)
+    x = x[np.abs(x) <= 448]
+    halfway = np.array([1.0625, 1.1875, -3.125, 2.0 ** -9 * 1.5, 2.0 ** -9 * 0.5, 240.0, 416.0], dtype=np.float32)
+    x = np.concatenate([x, halfway])
+    want = torch.from_numpy(x).to(torch.float8_e4m3fn).to(torch.float64).numpy()
+    assert np.array_equal(quantize_e4m3(x.astype(np.float64), 1.0), want)
+    assert quantize_e4m3(np.array([1.0625, 1.1875]), 1.0).tolist() == [1.0, 1.25]    # ties to even
+
+
+def test_quantize_e4m3_saturates_and_scales():
+    from oracle import quantize_e4m3
+    assert quantize_e4m3(np.array([1000.0, -1e9, 449.0]), 1.0).tolist() == [448.0, -448.0, 448.0]
+    assert quantize_e4m3(np.array([3.0]), 0.5)[0] == 6.0                              # in units of the scale
+
+
+def test_fp8_scores_attention_is_exact_on_the_e4m3_grid():
+    # queries and keys already on the scaled e4m3 grid: nothing to round, so the
+    # FP8-score attention is the plain one
+    from oracle import fp8_scores_attention, quantize_e4m3
+    r = np.random.default_rng(15)
+    Lc, blk, D, qs, ks = 16, 8, 16, 0.01, 0.02
+    w = RollingWindow(2)
+    for _ in range(2):
+        w.append(quantize_e4m3(r.standard_normal((1, Lc, 1, D)), ks) * ks, r.standard_normal((1, Lc, 1, D)))
+    q = quantize_e4m3(r.standard_normal((1, Lc, 2, D)), qs) * qs
+    O1, L1 = block_sparse_attention(q, w, blk)
+    O2, L2 = fp8_scores_attention(q, w, blk, qs, ks)
+    assert np.allclose(O1, O2, atol=1e-12) and np.allclose(L1, L2, atol=1e-12)
