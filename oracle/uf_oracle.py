@@ -427,8 +427,13 @@ def quantize_e4m3(x: np.ndarray, scale: float) -> np.ndarray:
     """Static-scale FP8 quantisation (FlashDecoder, inference optimisations:
     statically calibrated FP8): the e4m3 value nearest to x / scale (ties to
     even; e4m3 keeps 4 significant bits, exponent bias 7, subnormal spacing
-    2^-9, saturating at +-448), returned in e4m3 units as float64."""
-    v = np.asarray(x, dtype=np.float64) / scale
+    2^-9, saturating at +-448), returned in e4m3 units as float64.
+
+    The pages fix no precision for x / scale.  Because the quotient decides an
+    integer code, it is taken here as the kernels take it: in IEEE binary32,
+    x rounded to fp32 times the fp32 reciprocal of the fp32 scale."""
+    inv = np.float32(1.0) / np.float32(scale)
+    v = (np.asarray(x, dtype=np.float64).astype(np.float32) * inv).astype(np.float64)
     a = np.abs(v)
     e = np.floor(np.log2(np.where(a > 0, a, 1.0)))
     ulp = np.exp2(np.maximum(e, -6.0) - 3.0)             # normal spacing 2^(e-3); below 2^-6 the subnormal 2^-9

@@ -719,6 +719,19 @@ def test_quantize_e4m3_matches_torch_float8():
     assert quantize_e4m3(np.array([1.0625, 1.1875]), 1.0).tolist() == [1.0, 1.25]    # ties to even
 
 
+def test_quantize_e4m3_scaled_decision_in_fp32():
+    # x / scale is taken as fp32(x) * fp32(1 / fp32(scale)) before the e4m3
+    # rounding; torch's own fp32 product and float8 cast give the same codes
+    import torch
+    from oracle import quantize_e4m3
+    r = np.random.default_rng(16)
+    x = (r.standard_normal(50000) * 3.0).astype(np.float32)
+    for scale in (0.01, 0.0123, 1.0 / 7.0, 3.3):
+        inv = torch.tensor(1.0, dtype=torch.float32) / torch.tensor(scale, dtype=torch.float32)
+        want = (torch.from_numpy(x) * inv).clamp(-448, 448).to(torch.float8_e4m3fn).to(torch.float64).numpy()
+        assert np.array_equal(quantize_e4m3(x, scale), want)
+
+
 def test_quantize_e4m3_saturates_and_scales():
     from oracle import quantize_e4m3
     assert quantize_e4m3(np.array([1000.0, -1e9, 449.0]), 1.0).tolist() == [448.0, -448.0, 448.0]
