@@ -97,11 +97,17 @@ def kept_flops(cfg, idx, cnt, device):
     return 4.0 * cfg.D * float(per_item.sum())
 
 
-def append_bytes(cfg):
-    # read K,V of the chunk; write them into the slot (incl. padding rows); write pooled K
+def append_bytes(cfg, fp8=False):
+    # read K,V of the chunk; write them into the slot (incl. padding rows); write pooled K;
+    # FP8 variant: also the e4m3 copy of K's slot rows
     chunk = cfg.B * cfg.Lc * cfg.G * cfg.D * 2
     slot = cfg.B * cfg.lslot * cfg.G * cfg.D * 2
-    return 2 * chunk + 2 * slot + cfg.B * cfg.G * cfg.nb * cfg.D * 4
+    return 2 * chunk + 2 * slot + cfg.B * cfg.G * cfg.nb * cfg.D * 4 + (slot // 2 if fp8 else 0)
+
+
+def fp8_scales(chunk):
+    """Static per-tensor scales calibrated once on one chunk: amax / 448 (e4m3)."""
+    return (float(chunk["q"].float().abs().max()) / 448.0, float(chunk["k"].float().abs().max()) / 448.0)
 
 
 def rope_q_bytes(cfg):
@@ -202,7 +208,8 @@ def run_ours(args, cfg, rank, world, device):
     n_distinct = 3
     host_chunks = [chunk_inputs(cfg, args.seed + 1000 * rank, t) for t in range(cfg.W + n_distinct)]
     dev_chunks = [{n: x.to(device) for n, x in c.items()} for c in host_chunks]
-    win = uf.KVWindow(cfg.B, cfg.G, cfg.W, cfg.Lc, cfg.blk, cfg.D, device=device)
+    q_scale, k_scale = fp8_scales(host_chunks[0]) if args.fp8 else (None, None)
+    win = uf.KVWindow(cfg.B, cfg.G, cfg.W, cfg.Lc, cfg.blk, cfg.D, device=device, k_scale=k_scale)
     win.reset()
     tile_grid = cfg.grid if args.tiled else None
     for t in range(cfg.W):                       # fill the window (--anchor: the first chunk is pinned)
@@ -216,6 +223,13 @@ def run_ours(args, cfg, rank, world, device):
 
     q_rot = torch.empty_like(dev_chunks[0]["q"]) if (args.rope or args.tiled) else None
     o_tiled = torch.empty_like(o) if args.tiled else None
+
+    def attention(q, idx_s, cnt_s, k_s, out):
+        if args.fp8:
+            uf.uf_block_sparse_attn_fp8k(q, cfg.H, win.desc, win.k8, q_scale, k_scale, idx_s, cnt_s, k_s, scale,
+                                         out, lse)
+        else:
+            uf.uf_block_sparse_attn(q, cfg.H, win.desc, idx_s, cnt_s, k_s, scale, out, lse)
 
     def step(s, chunk, ev=None):
         # RoPE variant: the chunk sits at stream position (W + s) * Lc
@@ -239,7 +253,7 @@ def run_ours(args, cfg, rank, world, device):
         if cfg.dense:
             if ev is not None:
                 ev[2].record(stream)
-            uf.uf_block_sparse_attn(q, cfg.H, win.desc, None, None, 0, scale, o_tiled if args.tiled else o, lse)
+            attention(q, None, None, 0, o_tiled if args.tiled else o)
         else:
             if args.mask_local or args.mask_local_only:
                 uf.uf_block_mask_local(q, cfg.H, win.desc, k, args.mask_local, local_flags, idx[s], cnt[s])
@@ -247,7 +261,7 @@ def run_ours(args, cfg, rank, world, device):
                 uf.uf_block_mask(q, cfg.H, win.desc, k, idx[s], cnt[s])
             if ev is not None:
                 ev[2].record(stream)
-            uf.uf_block_sparse_attn(q, cfg.H, win.desc, idx[s], cnt[s], k, scale, o_tiled if args.tiled else o, lse)
+            attention(q, idx[s], cnt[s], k, o_tiled if args.tiled else o)
         if ev is not None:
             ev[3].record(stream)
         if args.tiled:                             # O back to row-major order (in the step, not in "attn")
@@ -328,11 +342,14 @@ def run_ours(args, cfg, rank, world, device):
     value = world * flops_per_step / (ms_per_step * 1e-3) / 1e12
     peaks, peaks_src = load_peaks()
     attn_tflops = flops_per_step / (per["attn"] * 1e-3) / 1e12
-    traffic = attn_traffic_per_launch(args.config)
+    traffic = None if args.fp8 else attn_traffic_per_launch(args.config)
+    # FP8 variant: half the FLOPs (QK) at the e4m3 rate, twice bf16's (nominal
+    # ratio applied to the measured bf16 peak), half (PV) at the bf16 rate
+    peak = peaks["bf16_tflops"] * (4.0 / 3.0 if args.fp8 else 1.0)
     hbm = peaks["hbm_gbs"]
     kernels = {
         "append": {"ms": per["append"],
-                   "GB/s": (append_bytes(cfg) + (rope_q_bytes(cfg) if (args.rope or args.tiled) else 0))
+                   "GB/s": (append_bytes(cfg, args.fp8) + (rope_q_bytes(cfg) if (args.rope or args.tiled) else 0))
                    / (per["append"] * 1e-3) / 1e9},
         "attn": {"ms": per["attn"], "TFLOP/s": attn_tflops},
     }
@@ -351,7 +368,7 @@ def run_ours(args, cfg, rank, world, device):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "bf16",
+        "dtype": "e4m3 QK, bf16 PV" if args.fp8 else "bf16",
         "data": "synthetic",
         "config": {
             "workload": args.config, "description": cfg.description, "B": cfg.B, "H": cfg.H, "G": cfg.G,
@@ -359,9 +376,13 @@ def run_ours(args, cfg, rank, world, device):
             "density": cfg.density, "kept_flops_per_step": flops_per_step,
             "mask_local": args.mask_local, "mask_local_only": bool(args.mask_local_only), "rope": bool(args.rope),
             "anchor": bool(args.anchor), "tiled": list(cfg.grid) if args.tiled else None,
+            "fp8": {"q_scale": q_scale, "k_scale": k_scale, "calibration": "amax / 448 of the first chunk"}
+            if args.fp8 else None,
             "step": ("uf_kv_append_rope + uf_rope + " if args.rope else
-                     "uf_kv_append_tiled + uf_tile_tokens + " if args.tiled else "uf_kv_append + ")
-                    + ("" if cfg.dense else mask_call_name(args)) + "uf_block_sparse_attn"
+                     "uf_kv_append_tiled + uf_tile_tokens + " if args.tiled else
+                     "uf_kv_append_fp8k + " if args.fp8 else "uf_kv_append + ")
+                    + ("" if cfg.dense else mask_call_name(args))
+                    + ("uf_block_sparse_attn_fp8k" if args.fp8 else "uf_block_sparse_attn")
                     + (" + uf_tile_tokens (O)" if args.tiled else ""),
             "l2": "no flush: every step's working set (%.0f MB) exceeds the 126 MB L2" % (
                 (cfg.B * cfg.Lc * (cfg.H * 2 + cfg.G * 2) * cfg.D * 2
@@ -373,12 +394,13 @@ def run_ours(args, cfg, rank, world, device):
         "roofline": {
             "bound": "tensor",
             "achieved": attn_tflops,
-            "peak": peaks["bf16_tflops"],
+            "peak": peak,
             "unit": "TFLOP/s",
-            "frac": attn_tflops / peaks["bf16_tflops"],
+            "frac": attn_tflops / peak,
             "traffic": traffic,
-            "kernel": "uf::attn_kernel<128>" if cfg.blk == 128 else "uf::attn_kernel<64>",
-            "peak_source": f"{peaks_src} bf16 dense burst (cuBLAS 8192^3)",
+            "kernel": "uf::attn_kernel<%d, %s>" % (cfg.blk, "true" if args.fp8 else "false"),
+            "peak_source": f"{peaks_src} bf16 dense burst (cuBLAS 8192^3)"
+                           + (" x 4/3: QK at the nominal e4m3/bf16 ratio of 2" if args.fp8 else ""),
         },
         "e2e": {"value": world * flops_per_step / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
@@ -394,13 +416,14 @@ class OracleSample:
     mask of one query head over the full window, then attention for up to
     ``n_items`` work items of that head.  Inputs are prepared once."""
 
-    def __init__(self, cfg, seed, local=0, local_only=False, anchor=False):
+    def __init__(self, cfg, seed, local=0, local_only=False, anchor=False, fp8=False):
         import oracle
         from workloads import to_f64
         self.oracle = oracle
         self.cfg = cfg
         self.local, self.local_only = local, local_only
         chunks = [chunk_inputs(cfg, seed, t) for t in range(cfg.W)]
+        self.scales = fp8_scales(chunks[0]) if fp8 else None
         self.win = oracle.RollingWindow(cfg.W)
         for t, c in enumerate(chunks):
             self.win.append(to_f64(c["k"][:, :, 0:1]), to_f64(c["v"][:, :, 0:1]), anchor=anchor and t == 0)
@@ -420,7 +443,12 @@ class OracleSample:
         done = 0
         while done < n_items and time.perf_counter() - t0 < budget_s:
             i = (first_item + done) % cfg.nb
-            self.oracle.block_sparse_attention(self.q, self.win, cfg.blk, m["idx"], m["cnt"], items=[(0, 0, i)])
+            if self.scales:
+                self.oracle.fp8_scores_attention(self.q, self.win, cfg.blk, *self.scales, m["idx"], m["cnt"],
+                                                 items=[(0, 0, i)])
+            else:
+                self.oracle.block_sparse_attention(self.q, self.win, cfg.blk, m["idx"], m["cnt"],
+                                                   items=[(0, 0, i)])
             flops += 4.0 * cfg.D * self.vq[i] * sum(self.vkv[j] for j in m["idx"][0, 0, i, :m["cnt"][0, 0, i]])
             done += 1
         dt = time.perf_counter() - t0
@@ -439,15 +467,15 @@ def blas_threads():
     return os.cpu_count()
 
 
-def cpu_baseline(cfg, seed, local=0, local_only=False, anchor=False):
-    flops, dt, desc = OracleSample(cfg, seed, local, local_only, anchor).run(n_items=10_000, budget_s=12.0)
+def cpu_baseline(cfg, seed, local=0, local_only=False, anchor=False, fp8=False):
+    flops, dt, desc = OracleSample(cfg, seed, local, local_only, anchor, fp8).run(n_items=10_000, budget_s=12.0)
     return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
             "sample": desc + f", {dt:.1f} s of fp64 numpy", "seconds": dt}
 
 
 def run_reference(args, cfg):
     # each step: the oracle on a bounded sample (one head's mask + 1 work item)
-    sample = OracleSample(cfg, args.seed, args.mask_local, args.mask_local_only, args.anchor)
+    sample = OracleSample(cfg, args.seed, args.mask_local, args.mask_local_only, args.anchor, args.fp8)
     for s in range(args.warmup):
         sample.run(n_items=1, budget_s=5.0, first_item=s)
     tot_f, tot_t = 0.0, 0.0
@@ -465,7 +493,7 @@ def run_reference(args, cfg):
         "config": {"workload": args.config, "description": cfg.description, "B": cfg.B, "H": cfg.H, "G": cfg.G,
                    "D": cfg.D, "Lc": cfg.Lc, "W": cfg.W, "blk": cfg.blk, "k": k, "density": cfg.density,
                    "mask_local": args.mask_local, "mask_local_only": bool(args.mask_local_only),
-                   "anchor": bool(args.anchor)},
+                   "anchor": bool(args.anchor), "fp8": bool(args.fp8)},
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
                          "sample": "per step: " + desc},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -503,13 +531,15 @@ def main():
                     help="(2,8,8) tile token order: K/V gathered by the append, Q and O permuted")
     ap.add_argument("--rope", action="store_true",
                     help="rotary position embedding: K rotated in the append, Q by uf_rope, at stream positions")
+    ap.add_argument("--fp8", action="store_true",
+                    help="FP8 scores: e4m3 K written by the append, e4m3 q . k on the tensor cores (static scales)")
     ap.add_argument("--mask-local-only", action="store_true",
                     help="keep the local band only (the fixed-local-window mask)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
-    if args.rope and args.tiled:
-        ap.error("--rope and --tiled are separate variants")
+    if sum(map(bool, (args.rope, args.tiled, args.fp8))) > 1:
+        ap.error("--rope, --tiled and --fp8 are separate variants")
     cfg = CONFIGS[args.config]
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -532,7 +562,7 @@ def main():
         if rank == 0:
             if world == 1 and not args.no_cpu_baseline:
                 result["cpu_baseline"] = cpu_baseline(cfg, args.seed, args.mask_local, args.mask_local_only,
-                                                      args.anchor)
+                                                      args.anchor, args.fp8)
             else:
                 result["cpu_baseline"] = None
             print(json.dumps(result), flush=True)

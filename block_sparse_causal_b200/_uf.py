@@ -62,6 +62,9 @@ def _load() -> ctypes.CDLL:
         "uf_block_mask": ([vp, i32, pc, i32, vp, vp, vp, vp], i32),
         "uf_block_mask_local": ([vp, i32, pc, i32, i32, i32, vp, vp, vp, vp], i32),
         "uf_block_sparse_attn": ([vp, i32, pc, vp, vp, i32, ctypes.c_float, vp, vp, vp], i32),
+        "uf_kv_append_fp8k": ([pc, vp, ctypes.c_float, vp, vp, i32, i32, vp], i32),
+        "uf_block_sparse_attn_fp8k": ([vp, i32, pc, vp, ctypes.c_float, ctypes.c_float, vp, vp, i32, ctypes.c_float,
+                                       vp, vp, vp], i32),
         "uf_get_error": ([ctypes.POINTER(i32), i32], i32),
         "uf_last_cuda_error": ([], ctypes.c_char_p),
         "uf_set_wait_limit": ([ctypes.c_int64], i32),
@@ -158,6 +161,19 @@ def uf_block_sparse_attn(q, H: int, cache: UfKvCache, idx, cnt, k: int, scale: f
                          stream=None) -> None:
     _check(lib.uf_block_sparse_attn(_ptr(q), H, ctypes.byref(cache), _ptr(idx), _ptr(cnt), k, scale, _ptr(o),
                                     _ptr(lse), _stream(stream)), "uf_block_sparse_attn")
+
+
+def uf_kv_append_fp8k(cache: UfKvCache, k8, k_scale: float, k_new, v_new, keep_chunks: int, flags: int = 0,
+                      stream=None) -> None:
+    _check(lib.uf_kv_append_fp8k(ctypes.byref(cache), _ptr(k8), k_scale, _ptr(k_new), _ptr(v_new), keep_chunks,
+                                 flags, _stream(stream)), "uf_kv_append_fp8k")
+
+
+def uf_block_sparse_attn_fp8k(q, H: int, cache: UfKvCache, k8, q_scale: float, k_scale: float, idx, cnt, k: int,
+                              scale: float, o, lse=None, stream=None) -> None:
+    _check(lib.uf_block_sparse_attn_fp8k(_ptr(q), H, ctypes.byref(cache), _ptr(k8), q_scale, k_scale, _ptr(idx),
+                                         _ptr(cnt), k, scale, _ptr(o), _ptr(lse), _stream(stream)),
+           "uf_block_sparse_attn_fp8k")
 
 
 def uf_get_error(clear: bool = True) -> int:

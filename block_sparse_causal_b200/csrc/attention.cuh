@@ -85,7 +85,8 @@ struct AttnParams {
   int32_t items;             // B * H * nb
   int32_t H, G, W, Lc, nb, lslot, k;
   uint32_t nb_mul;           // floor(2^32 / nb) (2^32 - 1 for nb = 1): j / nb without a divide
-  float scale_log2;          // softmax scale * log2(e)
+  float scale_log2;          // softmax scale * log2(e) (FP8 variant: times q_scale * k_scale)
+  float q_inv_scale;         // FP8 variant: 1 / q_scale
   long long wait_limit;
 };
 
@@ -151,7 +152,10 @@ __device__ __forceinline__ int attn_block(const AttnItem &it, int t, int NKV, bo
   return bad ? it.diag : jb;
 }
 
-template <int BLK>
+// FP8: the QK product from e4m3 queries and keys (kind::f8f6f4, K = 32 per
+// instruction): tmK then maps the window's e4m3 copy of K (one 128-byte panel
+// per tile row), and the queries go into tensor memory as e4m3 of q / q_scale.
+template <int BLK, bool FP8>
 __global__ void __launch_bounds__(ATTN_THREADS, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
@@ -249,9 +253,12 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
             int row, valid;
             kv_block_coords(jb, start, p.W, anchor, p.nb, p.nb_mul, p.lslot, BLK, p.Lc, row, valid);
             uint64_t *full = &full_bars[stage];
-            mbar_arrive_expect_tx(full, L::STAGE);
+            mbar_arrive_expect_tx(full, (FP8 && !is_v) ? L::STAGE / 2 : L::STAGE);
             uint8_t *dst = ring + stage * L::STAGE;
-            if (is_v) {
+            if (FP8 && !is_v) {
+              // e4m3 K tile: BLK token rows x 128 channels of one byte, one panel
+              tma_load_3d(dst, &tmK, full, 0, row, zc);
+            } else if (is_v) {
               // V^T tile: 128 channel rows x BLK tokens, in 64-token panels
 #pragma unroll
               for (int pnl = 0; pnl < BLK / 64; ++pnl)
@@ -322,10 +329,19 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
             if (!(ok = wait_bounded(&bar_kfull[stage], phase, abort_flag, p.wait_limit))) break;
             tc_fence_after();
             const uint32_t k_addr = k_base + stage * L::STAGE;
+            if (FP8) {
+              // four K = 32 steps over the 128-byte rows of the e4m3 tile
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-              const uint64_t bd = sdesc_sw128(k_addr + (kk >> 2) * L::PANEL + (kk & 3) * 32, 16, 1024);
-              mma_ts(tb + tm_s(buf), tb + TM_Q + kk * 8, bd, idesc_qk, kk > 0);
+              for (int kk = 0; kk < 4; ++kk) {
+                const uint64_t bd = sdesc_sw128(k_addr + kk * 32, 16, 1024);
+                mma_ts_f8(tb + tm_s(buf), tb + TM_Q + kk * 8, bd, idesc_e4m3_f32(128, BLK), kk > 0);
+              }
+            } else {
+#pragma unroll
+              for (int kk = 0; kk < 8; ++kk) {
+                const uint64_t bd = sdesc_sw128(k_addr + (kk >> 2) * L::PANEL + (kk & 3) * 32, 16, 1024);
+                mma_ts(tb + tm_s(buf), tb + TM_Q + kk * 8, bd, idesc_qk, kk > 0);
+              }
             }
             mma_commit(&bar_kempty[stage]);
             mma_commit(&bar_s[buf]);
@@ -476,7 +492,20 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
         qw[4 * c + 2] = v.z;
         qw[4 * c + 3] = v.w;
       }
-      tmem_st32(lane_base + TM_Q + 32 * x, qw);
+      if (FP8) {
+        // channels [64x, 64x + 64) as e4m3 of q / q_scale: 16 columns of four
+        uint32_t q8[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&qw[2 * e]));
+          const float2 c = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&qw[2 * e + 1]));
+          const float sc = p.q_inv_scale;
+          q8[e] = pack_e4m3x4(a.x * sc, a.y * sc, c.x * sc, c.y * sc);
+        }
+        tmem_st16(lane_base + TM_Q + 16 * x, q8);
+      } else {
+        tmem_st32(lane_base + TM_Q + 32 * x, qw);
+      }
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&bar_q);

@@ -85,6 +85,8 @@ struct AppendParams {
   int32_t make_anchor;         // pin this chunk as the window's anchor (window empty)
   long long pos0;              // RoPE variant: stream position of the chunk's first token
   TileGrid grid;               // tiled variant: the chunk's grid and tile
+  uint8_t *k8;                 // FP8 variant: [B, G, W*Lslot, D] e4m3 copy of K (same slots)
+  float k8_inv_scale;          // FP8 variant: 1 / k_scale
   double log2_base;
 };
 
@@ -166,8 +168,13 @@ __device__ __forceinline__ void transpose8x8_b16(const uint4 (&in)[8], uint4 (&o
   for (int c = 0; c < 8; ++c) out[c] = make_uint4(w[c][0], w[c][1], w[c][2], w[c][3]);
 }
 
-template <int BLK, bool ROPE, bool TILED>
+// MODE: APPEND_PLAIN, APPEND_ROPE (K rotated), APPEND_TILED (K / V gathered in
+// tile order), APPEND_FP8K (also an e4m3 copy of K).
+enum { APPEND_PLAIN = 0, APPEND_ROPE = 1, APPEND_TILED = 2, APPEND_FP8K = 3 };
+
+template <int BLK, int MODE>
 __global__ void __launch_bounds__(256) kv_append_kernel(const AppendParams p) {
+  constexpr bool ROPE = MODE == APPEND_ROPE, TILED = MODE == APPEND_TILED, FP8K = MODE == APPEND_FP8K;
   constexpr int D = 128;
   constexpr int PASSES = BLK / 16;
   const int r = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
@@ -254,6 +261,19 @@ __global__ void __launch_bounds__(256) kv_append_kernel(const AppendParams p) {
   for (int m = 0; m < PASSES; ++m) {
     const int t = tl + 16 * m;
     *reinterpret_cast<uint4 *>(kdst + static_cast<size_t>(t) * D) = kr[m];
+    if (FP8K) {
+      // the same eight channels as e4m3 of K / k_scale (padding rows: zeros)
+      const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&kr[m]);
+      float f[8];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 v = __bfloat1622float2(h[e]);
+        f[2 * e] = v.x * p.k8_inv_scale;
+        f[2 * e + 1] = v.y * p.k8_inv_scale;
+      }
+      *reinterpret_cast<uint2 *>(p.k8 + (dst_row0 + t) * D + dc * 8) =
+          make_uint2(pack_e4m3x4(f[0], f[1], f[2], f[3]), pack_e4m3x4(f[4], f[5], f[6], f[7]));
+    }
     const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&kr[m]);
 #pragma unroll
     for (int e = 0; e < 4; ++e) {

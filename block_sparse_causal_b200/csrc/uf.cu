@@ -68,11 +68,12 @@ EncodeTiledFn encode_fn() {
 
 // bf16 tensor map, 128-byte swizzle, box {64, box[1..]} (64 bf16 = 128 bytes inner).
 bool make_map(CUtensorMap *m, const void *base, int rank, const cuuint64_t *dims, const cuuint64_t *strides,
-              const cuuint32_t *box, CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
+              const cuuint32_t *box, CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B,
+              CUtensorMapDataType type = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint32_t es[5] = {1, 1, 1, 1, 1};
-  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void *>(base), dims, strides, box, es,
+  const CUresult r = fn(m, type, rank, const_cast<void *>(base), dims, strides, box, es,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
@@ -120,7 +121,8 @@ int32_t check_launch_regs(K kernel, std::atomic<int> (&done)[kMaxDevices]) {
   done[dev].store(1);
   return UF_OK;
 }
-std::atomic<int> g_attn128_regs[kMaxDevices], g_attn64_regs[kMaxDevices];
+std::atomic<int> g_attn128_regs[kMaxDevices], g_attn64_regs[kMaxDevices], g_attn128f8_regs[kMaxDevices],
+    g_attn64f8_regs[kMaxDevices];
 
 // Streaming multiprocessors of the current device (cached per device): the
 // persistent attention grid has one thread block per SM.
@@ -141,6 +143,7 @@ int32_t sm_count(int *out) {
   return UF_OK;
 }
 
+std::atomic<int> g_attn128f8_smem[kMaxDevices], g_attn64f8_smem[kMaxDevices];
 std::atomic<int> g_attn128_smem[kMaxDevices], g_attn64_smem[kMaxDevices], g_mask128_smem[kMaxDevices],
     g_mask64_smem[kMaxDevices], g_mask128b_smem[kMaxDevices], g_mask64b_smem[kMaxDevices];
 
@@ -158,7 +161,7 @@ bool rope_args_ok(long long pos0, float base) {
 // uf_kv_append and uf_kv_append_rope (rope = 1: K rotated at pos0 + token).
 int32_t append_impl(uf_kv_cache *c, const void *k_new, const void *v_new, int32_t keep_chunks, int32_t flags,
                     int32_t rope, long long pos0, double log2_base, uf_stream_t s,
-                    const uf::TileGrid *tile_grid = nullptr) {
+                    const uf::TileGrid *tile_grid = nullptr, void *k8 = nullptr, float k_scale = 1.0f) {
   if (!cache_ok(c)) return UF_EINVAL;
   if (!k_new || !v_new || !aligned16(k_new) || !aligned16(v_new)) return UF_EINVAL;
   if (keep_chunks < 1 || keep_chunks > c->W) return UF_EINVAL;
@@ -190,23 +193,26 @@ int32_t append_impl(uf_kv_cache *c, const void *k_new, const void *v_new, int32_
   p.log2_base = log2_base;
   const bool tiled = tile_grid != nullptr;
   if (tiled) p.grid = *tile_grid;
+  p.k8 = static_cast<uint8_t *>(k8);
+  p.k8_inv_scale = 1.0f / k_scale;
   const dim3 grid(p.nb, c->G, c->B);
   cudaGetLastError();
   const cudaStream_t st0 = reinterpret_cast<cudaStream_t>(s);
+  const int mode = rope ? uf::APPEND_ROPE : tiled ? uf::APPEND_TILED : k8 ? uf::APPEND_FP8K : uf::APPEND_PLAIN;
   if (c->blk == 128) {
-    if (rope)
-      uf::kv_append_kernel<128, true, false><<<grid, 256, 0, st0>>>(p);
-    else if (tiled)
-      uf::kv_append_kernel<128, false, true><<<grid, 256, 0, st0>>>(p);
-    else
-      uf::kv_append_kernel<128, false, false><<<grid, 256, 0, st0>>>(p);
+    switch (mode) {
+      case uf::APPEND_ROPE: uf::kv_append_kernel<128, uf::APPEND_ROPE><<<grid, 256, 0, st0>>>(p); break;
+      case uf::APPEND_TILED: uf::kv_append_kernel<128, uf::APPEND_TILED><<<grid, 256, 0, st0>>>(p); break;
+      case uf::APPEND_FP8K: uf::kv_append_kernel<128, uf::APPEND_FP8K><<<grid, 256, 0, st0>>>(p); break;
+      default: uf::kv_append_kernel<128, uf::APPEND_PLAIN><<<grid, 256, 0, st0>>>(p); break;
+    }
   } else {
-    if (rope)
-      uf::kv_append_kernel<64, true, false><<<grid, 256, 0, st0>>>(p);
-    else if (tiled)
-      uf::kv_append_kernel<64, false, true><<<grid, 256, 0, st0>>>(p);
-    else
-      uf::kv_append_kernel<64, false, false><<<grid, 256, 0, st0>>>(p);
+    switch (mode) {
+      case uf::APPEND_ROPE: uf::kv_append_kernel<64, uf::APPEND_ROPE><<<grid, 256, 0, st0>>>(p); break;
+      case uf::APPEND_TILED: uf::kv_append_kernel<64, uf::APPEND_TILED><<<grid, 256, 0, st0>>>(p); break;
+      case uf::APPEND_FP8K: uf::kv_append_kernel<64, uf::APPEND_FP8K><<<grid, 256, 0, st0>>>(p); break;
+      default: uf::kv_append_kernel<64, uf::APPEND_PLAIN><<<grid, 256, 0, st0>>>(p); break;
+    }
   }
   const int32_t st = launch_status();
   if (st != UF_OK) return st;
@@ -220,6 +226,109 @@ int32_t append_impl(uf_kv_cache *c, const void *k_new, const void *v_new, int32_
   return UF_OK;
 }
 
+}  // namespace
+
+namespace {
+// uf_block_sparse_attn and its FP8-score variant (k8 != NULL).
+int32_t attn_impl(const void *q, int32_t H, const uf_kv_cache *c, const int32_t *idx, const int32_t *cnt, int32_t k,
+                  float scale, void *o, float *lse, uf_stream_t s, const void *k8, float q_scale, float k_scale) {
+  if (!cache_ok(c)) return UF_EINVAL;
+  if (!q || !o || !aligned16(q) || !aligned16(o)) return UF_EINVAL;
+  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return UF_EINVAL;
+  if (H < 1 || H % c->G != 0) return UF_EINVAL;
+  if (!(scale > 0.f) || !isfinite(scale)) return UF_EINVAL;
+  const int32_t nb = ceil_div(c->Lc, c->blk);
+  if (idx) {
+    if (k < 1 || k > c->W * nb) return UF_EINVAL;
+    if (reinterpret_cast<uintptr_t>(idx) & 3u) return UF_EINVAL;
+    if (cnt && (reinterpret_cast<uintptr_t>(cnt) & 3u)) return UF_EINVAL;
+  } else {
+    k = 0;
+    cnt = nullptr;
+  }
+  if (c->host_n_valid < 1) return UF_EINVAL;
+  const long long items = static_cast<long long>(c->B) * H * nb;
+  if (items >= (1LL << 31)) return UF_EINVAL;
+
+  const int32_t lslot = nb * c->blk;
+  CUtensorMap tq, tk, tv, to;
+  {
+    // Q and O: [B, Lc, H, D] as {channels, heads, tokens, batch}.  Q: a
+    // 128-row tile of one head per 64-channel load (rows past Lc read as
+    // zero); O: one q-block (blk rows) of one head per 64-channel store
+    const cuuint64_t dims[4] = {128, static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(c->Lc),
+                                static_cast<cuuint64_t>(c->B)};
+    // byte strides of dims 1..3 (head, token, batch)
+    const cuuint64_t strides[3] = {256, static_cast<cuuint64_t>(H) * 256, static_cast<cuuint64_t>(c->Lc) * H * 256};
+    const cuuint32_t box[4] = {64, 1, 128, 1};
+    if (!make_map(&tq, q, 4, dims, strides, box)) return UF_ECUDA;
+    const cuuint32_t obox[4] = {64, 1, static_cast<cuuint32_t>(c->blk), 1};
+    if (!make_map(&to, o, 4, dims, strides, obox)) return UF_ECUDA;
+  }
+  if (!k8) {
+    // K: [B*G][W*Lslot][128] -> box {64 channels, blk tokens}
+    const cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(c->W) * lslot, static_cast<cuuint64_t>(c->B) * c->G};
+    const cuuint64_t strides[2] = {256, static_cast<cuuint64_t>(c->W) * lslot * 256};
+    const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(c->blk), 1};
+    if (!make_map(&tk, c->k, 3, dims, strides, box)) return UF_ECUDA;
+  } else {
+    // e4m3 K: [B*G][W*Lslot][128 bytes] -> box {128 channels, blk tokens}
+    const cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(c->W) * lslot, static_cast<cuuint64_t>(c->B) * c->G};
+    const cuuint64_t strides[2] = {128, static_cast<cuuint64_t>(c->W) * lslot * 128};
+    const cuuint32_t box[3] = {128, static_cast<cuuint32_t>(c->blk), 1};
+    if (!make_map(&tk, k8, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_DATA_TYPE_UINT8))
+      return UF_ECUDA;
+  }
+  {
+    // V^T: [B*G][128][W*Lslot] -> box {64 tokens, 128 channels}
+    const cuuint64_t row = static_cast<cuuint64_t>(c->W) * lslot;
+    const cuuint64_t dims[3] = {row, 128, static_cast<cuuint64_t>(c->B) * c->G};
+    const cuuint64_t strides[2] = {row * 2, row * 2 * 128};
+    const cuuint32_t box[3] = {64, 128, 1};
+    if (!make_map(&tv, c->v, 3, dims, strides, box)) return UF_ECUDA;
+  }
+  uf::AttnParams p;
+  p.meta = c->meta;
+  p.idx = idx;
+  p.cnt = cnt;
+  p.o = static_cast<__nv_bfloat16 *>(o);
+  p.items = static_cast<int32_t>(items);
+  p.lse = lse;
+  p.H = H;
+  p.G = c->G;
+  p.W = c->W;
+  p.Lc = c->Lc;
+  p.nb = nb;
+  p.lslot = lslot;
+  p.k = k;
+  p.nb_mul = nb == 1 ? 0xFFFFFFFFu : static_cast<uint32_t>((1ULL << 32) / static_cast<uint64_t>(nb));
+  p.scale_log2 = scale * q_scale * k_scale * 1.4426950408889634f;
+  p.q_inv_scale = 1.0f / q_scale;
+  p.wait_limit = g_wait_limit.load();
+  int sms = 0;
+  const int32_t se = sm_count(&sms);
+  if (se != UF_OK) return se;
+  const unsigned grid = static_cast<unsigned>(items < sms ? items : sms);
+  cudaGetLastError();
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(s);
+  const bool fp8 = k8 != nullptr;
+  if (c->blk == 128) {
+    constexpr int smem = uf::AttnSmem<128>::DYN;
+    auto kern = fp8 ? uf::attn_kernel<128, true> : uf::attn_kernel<128, false>;
+    int32_t e = check_launch_regs(kern, fp8 ? g_attn128f8_regs : g_attn128_regs);
+    if (e == UF_OK) e = ensure_smem(kern, smem, fp8 ? g_attn128f8_smem : g_attn128_smem);
+    if (e != UF_OK) return e;
+    kern<<<grid, uf::ATTN_THREADS, smem, st>>>(tq, tk, tv, to, p);
+  } else {
+    constexpr int smem = uf::AttnSmem<64>::DYN;
+    auto kern = fp8 ? uf::attn_kernel<64, true> : uf::attn_kernel<64, false>;
+    int32_t e = check_launch_regs(kern, fp8 ? g_attn64f8_regs : g_attn64_regs);
+    if (e == UF_OK) e = ensure_smem(kern, smem, fp8 ? g_attn64f8_smem : g_attn64_smem);
+    if (e != UF_OK) return e;
+    kern<<<grid, uf::ATTN_THREADS, smem, st>>>(tq, tk, tv, to, p);
+  }
+  return launch_status();
+}
 }  // namespace
 
 extern "C" {
@@ -387,92 +496,23 @@ int32_t uf_block_mask_local(const void *q, int32_t H, const uf_kv_cache *c, int3
 
 int32_t uf_block_sparse_attn(const void *q, int32_t H, const uf_kv_cache *c, const int32_t *idx, const int32_t *cnt,
                              int32_t k, float scale, void *o, float *lse, uf_stream_t s) {
-  if (!cache_ok(c)) return UF_EINVAL;
-  if (!q || !o || !aligned16(q) || !aligned16(o)) return UF_EINVAL;
-  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return UF_EINVAL;
-  if (H < 1 || H % c->G != 0) return UF_EINVAL;
-  if (!(scale > 0.f) || !isfinite(scale)) return UF_EINVAL;
-  const int32_t nb = ceil_div(c->Lc, c->blk);
-  if (idx) {
-    if (k < 1 || k > c->W * nb) return UF_EINVAL;
-    if (reinterpret_cast<uintptr_t>(idx) & 3u) return UF_EINVAL;
-    if (cnt && (reinterpret_cast<uintptr_t>(cnt) & 3u)) return UF_EINVAL;
-  } else {
-    k = 0;
-    cnt = nullptr;
-  }
-  if (c->host_n_valid < 1) return UF_EINVAL;
-  const long long items = static_cast<long long>(c->B) * H * nb;
-  if (items >= (1LL << 31)) return UF_EINVAL;
-
-  const int32_t lslot = nb * c->blk;
-  CUtensorMap tq, tk, tv, to;
-  {
-    // Q and O: [B, Lc, H, D] as {channels, heads, tokens, batch}.  Q: a
-    // 128-row tile of one head per 64-channel load (rows past Lc read as
-    // zero); O: one q-block (blk rows) of one head per 64-channel store
-    const cuuint64_t dims[4] = {128, static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(c->Lc),
-                                static_cast<cuuint64_t>(c->B)};
-    // byte strides of dims 1..3 (head, token, batch)
-    const cuuint64_t strides[3] = {256, static_cast<cuuint64_t>(H) * 256, static_cast<cuuint64_t>(c->Lc) * H * 256};
-    const cuuint32_t box[4] = {64, 1, 128, 1};
-    if (!make_map(&tq, q, 4, dims, strides, box)) return UF_ECUDA;
-    const cuuint32_t obox[4] = {64, 1, static_cast<cuuint32_t>(c->blk), 1};
-    if (!make_map(&to, o, 4, dims, strides, obox)) return UF_ECUDA;
-  }
-  {
-    // K: [B*G][W*Lslot][128] -> box {64 channels, blk tokens}
-    const cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(c->W) * lslot, static_cast<cuuint64_t>(c->B) * c->G};
-    const cuuint64_t strides[2] = {256, static_cast<cuuint64_t>(c->W) * lslot * 256};
-    const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(c->blk), 1};
-    if (!make_map(&tk, c->k, 3, dims, strides, box)) return UF_ECUDA;
-  }
-  {
-    // V^T: [B*G][128][W*Lslot] -> box {64 tokens, 128 channels}
-    const cuuint64_t row = static_cast<cuuint64_t>(c->W) * lslot;
-    const cuuint64_t dims[3] = {row, 128, static_cast<cuuint64_t>(c->B) * c->G};
-    const cuuint64_t strides[2] = {row * 2, row * 2 * 128};
-    const cuuint32_t box[3] = {64, 128, 1};
-    if (!make_map(&tv, c->v, 3, dims, strides, box)) return UF_ECUDA;
-  }
-  uf::AttnParams p;
-  p.meta = c->meta;
-  p.idx = idx;
-  p.cnt = cnt;
-  p.o = static_cast<__nv_bfloat16 *>(o);
-  p.items = static_cast<int32_t>(items);
-  p.lse = lse;
-  p.H = H;
-  p.G = c->G;
-  p.W = c->W;
-  p.Lc = c->Lc;
-  p.nb = nb;
-  p.lslot = lslot;
-  p.k = k;
-  p.nb_mul = nb == 1 ? 0xFFFFFFFFu : static_cast<uint32_t>((1ULL << 32) / static_cast<uint64_t>(nb));
-  p.scale_log2 = scale * 1.4426950408889634f;
-  p.wait_limit = g_wait_limit.load();
-  int sms = 0;
-  const int32_t se = sm_count(&sms);
-  if (se != UF_OK) return se;
-  const unsigned grid = static_cast<unsigned>(items < sms ? items : sms);
-  cudaGetLastError();
-  const cudaStream_t st = reinterpret_cast<cudaStream_t>(s);
-  if (c->blk == 128) {
-    constexpr int smem = uf::AttnSmem<128>::DYN;
-    int32_t e = check_launch_regs(uf::attn_kernel<128>, g_attn128_regs);
-    if (e == UF_OK) e = ensure_smem(uf::attn_kernel<128>, smem, g_attn128_smem);
-    if (e != UF_OK) return e;
-    uf::attn_kernel<128><<<grid, uf::ATTN_THREADS, smem, st>>>(tq, tk, tv, to, p);
-  } else {
-    constexpr int smem = uf::AttnSmem<64>::DYN;
-    int32_t e = check_launch_regs(uf::attn_kernel<64>, g_attn64_regs);
-    if (e == UF_OK) e = ensure_smem(uf::attn_kernel<64>, smem, g_attn64_smem);
-    if (e != UF_OK) return e;
-    uf::attn_kernel<64><<<grid, uf::ATTN_THREADS, smem, st>>>(tq, tk, tv, to, p);
-  }
-  return launch_status();
+  return attn_impl(q, H, c, idx, cnt, k, scale, o, lse, s, nullptr, 1.0f, 1.0f);
 }
+
+int32_t uf_block_sparse_attn_fp8k(const void *q, int32_t H, const uf_kv_cache *c, const void *k8, float q_scale,
+                                  float k_scale, const int32_t *idx, const int32_t *cnt, int32_t k, float scale,
+                                  void *o, float *lse, uf_stream_t s) {
+  if (!k8 || !aligned16(k8)) return UF_EINVAL;
+  if (!(q_scale > 0.f) || !isfinite(q_scale) || !(k_scale > 0.f) || !isfinite(k_scale)) return UF_EINVAL;
+  return attn_impl(q, H, c, idx, cnt, k, scale, o, lse, s, k8, q_scale, k_scale);
+}
+
+int32_t uf_kv_append_fp8k(uf_kv_cache *c, void *k8, float k_scale, const void *k_new, const void *v_new,
+                          int32_t keep_chunks, int32_t flags, uf_stream_t s) {
+  if (!k8 || !aligned16(k8) || !(k_scale > 0.f) || !isfinite(k_scale)) return UF_EINVAL;
+  return append_impl(c, k_new, v_new, keep_chunks, flags, 0, 0, 0.0, s, nullptr, k8, k_scale);
+}
+
 
 int32_t uf_get_error(int32_t *status, int32_t clear) {
   if (!status) return UF_EINVAL;

@@ -11,9 +11,11 @@ from . import _uf
 class KVWindow:
     """Allocates k, v, kpool and meta for a window of W chunks on ``device``
     (sizes from ``uf_kv_cache_bytes``) and holds the ``uf_kv_cache``
-    descriptor that the library calls take."""
+    descriptor that the library calls take.  With ``k_scale`` it also owns the
+    e4m3 copy of K (``k8``) that the FP8-score calls read and write."""
 
-    def __init__(self, B: int, G: int, W: int, Lc: int, blk: int = 128, D: int = 128, device="cuda"):
+    def __init__(self, B: int, G: int, W: int, Lc: int, blk: int = 128, D: int = 128, device="cuda",
+                 k_scale: float | None = None):
         kv_bytes, kpool_bytes, meta_bytes = _uf.uf_kv_cache_bytes(B, G, D, W, Lc, blk)
         self.B, self.G, self.D, self.W, self.Lc, self.blk = B, G, D, W, Lc, blk
         self.nb = math.ceil(Lc / blk)
@@ -24,6 +26,8 @@ class KVWindow:
         self.kpool = torch.zeros(kpool_bytes // 4, dtype=torch.float32, device=device).view(B, G, W * self.nb, D)
         self.meta = torch.zeros(meta_bytes // 4, dtype=torch.int32, device=device)
         self.desc = _uf.uf_kv_cache_init(self.k, self.v, self.kpool, self.meta, B, G, D, W, Lc, blk)
+        self.k_scale = k_scale
+        self.k8 = None if k_scale is None else torch.zeros(B, G, W * self.lslot, D, dtype=torch.uint8, device=device)
 
     @property
     def n_valid(self) -> int:
@@ -40,10 +44,15 @@ class KVWindow:
         rotated at stream positions rope_pos0 + token (uf_kv_append_rope); with
         ``tile_grid`` = (T, Hg, Wg), K and V are stored in tiled token order
         (uf_kv_append_tiled); with ``anchor`` (empty window) the chunk becomes
-        the pinned anchor."""
+        the pinned anchor.  A window made with ``k_scale`` also writes the e4m3
+        copy of K (uf_kv_append_fp8k)."""
         keep = self.W if keep_chunks is None else keep_chunks
         flags = (_uf.UF_APPEND_REPLACE_NEWEST if replace_newest else 0) | (_uf.UF_APPEND_ANCHOR if anchor else 0)
-        if tile_grid is not None:
+        if self.k8 is not None:
+            if rope_pos0 is not None or tile_grid is not None:
+                raise ValueError("the FP8 append neither rotates nor tiles")
+            _uf.uf_kv_append_fp8k(self.desc, self.k8, self.k_scale, k_new, v_new, keep, flags, stream)
+        elif tile_grid is not None:
             if rope_pos0 is not None:
                 raise ValueError("the tiled append does not rotate")
             _uf.uf_kv_append_tiled(self.desc, k_new, v_new, keep, flags, tile_grid, tile, stream)

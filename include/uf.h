@@ -305,6 +305,47 @@ int32_t uf_block_sparse_attn(const void *q, int32_t H, const uf_kv_cache *c,
                              void *o, float *lse, uf_stream_t s);
 
 /*
+ * FP8-score variant, append side (FlashDecoder, inference optimisations:
+ * statically calibrated FP8).  uf_kv_append(c, k_new, v_new, keep_chunks,
+ * flags, s) that also writes an e4m3 copy of each appended K row:
+ *
+ *   k8       device uint8 [B, G, W * Lslot, D], caller-owned, same slots and
+ *            token rows as c->k: k8 = e4m3(K / k_scale), rounded to nearest
+ *            (ties to even) from the fp32 product K * (1 / k_scale) and
+ *            saturated at +-448; padding rows get 0.  Must be 16-byte aligned.
+ *   k_scale  static per-tensor K scale, finite and > 0 (for instance
+ *            amax(K) / 448 of a calibration chunk).
+ *
+ * Use the same k8 buffer and k_scale for every append of a window; chunks
+ * appended without it have no e4m3 copy.  No RoPE or tile-order form.
+ * Errors as uf_kv_append, plus UF_EINVAL for a NULL or unaligned k8 or a bad
+ * k_scale.
+ */
+int32_t uf_kv_append_fp8k(uf_kv_cache *c, void *k8, float k_scale, const void *k_new,
+                          const void *v_new, int32_t keep_chunks, int32_t flags, uf_stream_t s);
+
+/*
+ * FP8-score variant, attention side: uf_block_sparse_attn with the scores
+ * q . k taken on the tensor cores in e4m3 x e4m3 with fp32 accumulation:
+ *
+ *   s = scale * q_scale * k_scale * (e4m3(q / q_scale) . k8)
+ *
+ * where e4m3(q / q_scale) rounds the fp32 product q * (1 / q_scale) to
+ * nearest (ties to even, saturated at +-448) and k8 is the buffer written by
+ * uf_kv_append_fp8k with k_scale.  The softmax (fp32), the probabilities
+ * (bf16) and the PV product (bf16 V) are those of uf_block_sparse_attn.
+ *
+ *   k8       device uint8 [B, G, W * Lslot, D] as above, 16-byte aligned.
+ *   q_scale  static per-tensor query scale, finite and > 0.
+ *   k_scale  the scale the window's k8 rows were written with.
+ *   other arguments, outputs and errors as uf_block_sparse_attn.
+ */
+int32_t uf_block_sparse_attn_fp8k(const void *q, int32_t H, const uf_kv_cache *c, const void *k8,
+                                  float q_scale, float k_scale, const int32_t *idx,
+                                  const int32_t *cnt, int32_t k, float scale, void *o, float *lse,
+                                  uf_stream_t s);
+
+/*
  * Read the device-side error word of the current device (the first error a
  * kernel recorded since the last clear) into *status; clear it if `clear` is
  * non-zero.  Synchronises the device (this is the one call that does).

@@ -113,6 +113,13 @@ def test_calls_reject_bad_arguments_before_launch(uf):
         uf.uf_kv_append(c, kn, vn, 1, 0, stream=0)
     assert e.value.status == uf.UF_EINVAL
     c.host_n_valid, c.host_anchor = 0, 0
+    # FP8 append: NULL or misaligned e4m3 buffer, scale not finite and positive
+    for k8, ks in [(None, 1.0), (FakeTensor(0xB00008), 1.0), (FakeTensor(0xB00000), 0.0),
+                   (FakeTensor(0xB00000), -2.0), (FakeTensor(0xB00000), float("nan")),
+                   (FakeTensor(0xB00000), float("inf"))]:
+        with pytest.raises(uf.UfError) as e:
+            uf.uf_kv_append_fp8k(c, k8, ks, kn, vn, 2, 0, stream=0)
+        assert e.value.status == uf.UF_EINVAL
     # RoPE: negative or too large position, base <= 1 or not finite, misaligned or empty input
     for pos0, base in [(-1, 10000.0), (1 << 40, 10000.0), (0, 1.0), (0, 0.5), (0, float("nan")), (0, float("inf"))]:
         with pytest.raises(uf.UfError) as e:
@@ -144,6 +151,14 @@ def test_calls_reject_bad_arguments_before_launch(uf):
     for scale in (0.0, -1.0, float("inf"), float("nan")):
         with pytest.raises(uf.UfError) as e:
             uf.uf_block_sparse_attn(q, 2, c, None, None, 0, scale, FakeTensor(0xA00000), None, stream=0)
+        assert e.value.status == uf.UF_EINVAL
+    # FP8 scores: NULL or misaligned e4m3 K, either scale not finite and positive
+    for k8, qs, ks in [(None, 1.0, 1.0), (FakeTensor(0xB00004), 1.0, 1.0), (FakeTensor(0xB00000), 0.0, 1.0),
+                       (FakeTensor(0xB00000), 1.0, -1.0), (FakeTensor(0xB00000), float("nan"), 1.0),
+                       (FakeTensor(0xB00000), 1.0, float("inf"))]:
+        with pytest.raises(uf.UfError) as e:
+            uf.uf_block_sparse_attn_fp8k(q, 2, c, k8, qs, ks, None, None, 0, 0.088, FakeTensor(0xA00000), None,
+                                         stream=0)
         assert e.value.status == uf.UF_EINVAL
     with pytest.raises(uf.UfError):
         uf.uf_block_sparse_attn(q, 2, c, idx, cnt, 9, 0.088, FakeTensor(0xA00000), None, stream=0)

@@ -1,0 +1,161 @@
+"""GPU parity of the FP8-score variant (FlashDecoder, inference optimisations:
+statically calibrated FP8): the e4m3 copy of K that the append writes, bit
+for bit, and the attention whose scores are e4m3 q . e4m3 k on the tensor
+cores, against the fp64 oracle's fp8_scores_attention on the same codes.
+
+The oracle quantises with the kernels' fp32 quotient, so both sides hold the
+same e4m3 codes; what remains between them is the fp32 accumulation of exact
+e4m3 products and the bf16 probabilities, as in the bf16 path, so the
+acceptance tolerances are the bf16 path's."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from uf_testlib import (GpuStream, OracleStream, assert_attention_ok, oracle_idx_array, sample_items)
+from workloads import CONFIGS, chunk_inputs, scaled
+
+pytestmark = [pytest.mark.gpu,
+              pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")]
+
+CASES = {
+    # 64-token blocks, top-4 of 8, ragged last block (300 = 4 * 64 + 44)
+    "blk64": scaled(CONFIGS["tiny"], H=2, G=1, Lc=300, k_fixed=3),
+    # grouped-query heads (4 per KV head), window of 3, dense
+    "gqa_w3": scaled(CONFIGS["gqa_decoder"], B=2, H=8, G=2, Lc=700, W=3),
+    # block-offset inputs, window of 3, top-k density 25%
+    "sr_w3": scaled(CONFIGS["1k_sr"], H=4, G=4, Lc=1000, W=3),
+}
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib(built_lib):
+    uf = built_lib
+    uf.uf_get_error(clear=True)
+    yield uf
+    assert uf.uf_get_error(clear=True) == 0, "a kernel recorded a device-side error"
+
+
+def static_scales(cfg, seed):
+    """Per-tensor scales calibrated once on chunk 0 of the stream: amax / 448."""
+    inp = chunk_inputs(cfg, seed, 0)
+    qs = float(inp["q"].float().abs().max()) / oracle.E4M3_MAX
+    ks = float(inp["k"].float().abs().max()) / oracle.E4M3_MAX
+    return qs, ks
+
+
+def _stream(cfg, n, seed, anchor=False):
+    qs, ks = static_scales(cfg, seed)
+    gpu, orc = GpuStream(cfg, k_scale=ks), OracleStream(cfg)
+    last = None
+    for t in range(n):
+        last = chunk_inputs(cfg, seed, t)
+        gpu.append(last, anchor=anchor and t == 0)
+        orc.append(last, anchor=anchor and t == 0)
+    torch.cuda.synchronize()
+    return gpu, orc, last, qs, ks
+
+
+def _slot(win, c):
+    start, anchor = int(win.meta[0].item()), int(win.meta[3].item())
+    if anchor:
+        return win.W - 1 if c == 0 else (start + c - 1) % (win.W - 1)
+    return (start + c) % win.W
+
+
+@pytest.mark.parametrize("name,anchor", [("blk64", False), ("gqa_w3", False), ("sr_w3", True)])
+def test_fp8_k_codes_bit_exact(name, anchor):
+    cfg = CASES[name]
+    gpu, orc, _, _, ks = _stream(cfg, cfg.W + 2, seed=21, anchor=anchor)
+    k8 = gpu.win.k8.view(torch.float8_e4m3fn).to(torch.float64).cpu().numpy()
+    raw = gpu.win.k8.cpu().numpy()
+    for g in range(cfg.G):
+        w = orc.windows[g]
+        for c in range(orc.n_valid):
+            slot = _slot(gpu.win, c)
+            r0 = slot * gpu.win.lslot
+            want = oracle.quantize_e4m3(w.k[c][:, :, 0, :], ks)
+            assert np.array_equal(k8[:, g, r0:r0 + cfg.Lc], want), (g, c)
+            assert not raw[:, g, r0 + cfg.Lc:r0 + gpu.win.lslot].any(), "padding rows must be zero"
+
+
+@pytest.mark.parametrize("name", ["blk64", "gqa_w3", "sr_w3"])
+def test_fp8_attention_parity(name):
+    cfg = CASES[name]
+    gpu, orc, last, qs, ks = _stream(cfg, cfg.W + 1, seed=22)
+    items = [(b, h, i) for b in range(cfg.B) for h in range(cfg.H) for i in range(cfg.nb)]
+    if cfg.dense:
+        o, lse = gpu.attention_fp8(last["q"], qs)
+        torch.cuda.synchronize()
+        assert_attention_ok(cfg, o, lse, orc.attention_fp8(last["q"], items, qs, ks), name)
+        return
+    k = cfg.k_for()
+    oidx, ocnt = oracle_idx_array(cfg, orc.mask(last["q"], k))
+    o, lse = gpu.attention_fp8(last["q"], qs, torch.from_numpy(oidx).cuda(), torch.from_numpy(ocnt).cuda(),
+                               oidx.shape[-1])
+    torch.cuda.synchronize()
+    assert_attention_ok(cfg, o, lse, orc.attention_fp8(last["q"], items, qs, ks, oidx, ocnt), name)
+
+
+def test_fp8_anchored_window_and_saturation():
+    # anchored window; the scales are calibrated on a quarter of chunk 0's
+    # amax, so the largest q and k saturate at +-448 on both sides
+    cfg = CASES["sr_w3"]
+    qs, ks = static_scales(cfg, 23)
+    qs, ks = qs / 4, ks / 4
+    gpu, orc = GpuStream(cfg, k_scale=ks), OracleStream(cfg)
+    last = None
+    for t in range(cfg.W + 2):
+        last = chunk_inputs(cfg, 23, t)
+        gpu.append(last, anchor=t == 0)
+        orc.append(last, anchor=t == 0)
+    k8 = gpu.win.k8.view(torch.float8_e4m3fn).to(torch.float64).cpu().numpy()
+    assert (np.abs(k8) == oracle.E4M3_MAX).any()
+    o, lse = gpu.attention_fp8(last["q"], qs)
+    items = [(b, h, i) for b in range(cfg.B) for h in range(cfg.H) for i in range(cfg.nb)]
+    torch.cuda.synchronize()
+    assert_attention_ok(cfg, o, lse, orc.attention_fp8(last["q"], items, qs, ks), "anchored saturated")
+
+
+def test_fp8_is_close_to_bf16_scores():
+    # the two variants differ only by the e4m3 rounding of q and k (scales
+    # calibrated on every chunk here, so nothing saturates).  With
+    # |dq| <= 2^-4 (|q| + 2^-6 q_scale) and the same for k, each score moves by
+    # at most D = (2^-3 + 2^-8) scale max_j sum_i (|q_i| + 2^-6 q_scale)(|k_ji| + 2^-6 k_scale),
+    # so |LSE8 - LSE16| <= D and each probability by a factor within e^(+-2D)
+    cfg = CASES["gqa_w3"]
+    chunks = [chunk_inputs(cfg, 24, t) for t in range(cfg.W)]
+    qs = float(chunks[-1]["q"].float().abs().max()) / oracle.E4M3_MAX
+    ks = max(float(c["k"].float().abs().max()) for c in chunks) / oracle.E4M3_MAX
+    gpu = GpuStream(cfg, k_scale=ks)
+    for c in chunks:
+        gpu.append(c)
+    q = chunks[-1]["q"]
+    o8, l8 = gpu.attention_fp8(q, qs)
+    o16, l16 = gpu.attention(q)
+    torch.cuda.synchronize()
+    scale = cfg.D ** -0.5
+    delta = 0.0
+    for b in range(cfg.B):
+        for h in range(cfg.H):
+            g = h // (cfg.H // cfg.G)
+            a = q[b, :, h, :].double().abs() + qs / 64
+            kk = torch.cat([c["k"][b, :, g, :] for c in chunks]).double().abs() + ks / 64
+            delta = max(delta, (2.0 ** -3 + 2.0 ** -8) * scale * float((a @ kk.t()).max()))
+    assert float((l8 - l16).abs().max()) <= delta
+    vmax = max(float(c["v"].float().abs().max()) for c in chunks)
+    # both outputs also carry bf16 probabilities (2^-9 relative each) and bf16 O
+    bound = (np.expm1(2 * delta) + 2.0 ** -7) * vmax
+    assert float((o8.float() - o16.float()).abs().max()) <= bound
+
+
+def test_fp8_full_size_1k():
+    cfg = CONFIGS["1k_sr"]
+    gpu, orc, last, qs, ks = _stream(cfg, cfg.W + 1, seed=0)
+    k = cfg.k_for()
+    oidx, ocnt = oracle_idx_array(cfg, orc.mask(last["q"], k))
+    o, lse = gpu.attention_fp8(last["q"], qs, torch.from_numpy(oidx).cuda(), torch.from_numpy(ocnt).cuda(),
+                               oidx.shape[-1])
+    items = sample_items(cfg, 12, seed=5)
+    torch.cuda.synchronize()
+    assert_attention_ok(cfg, o, lse, orc.attention_fp8(last["q"], items, qs, ks, oidx, ocnt), "1k fp8")

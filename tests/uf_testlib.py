@@ -29,11 +29,11 @@ NEAR_TIE_REL = 1e-4
 class GpuStream:
     """Rolling window on the GPU fed chunk by chunk through the C ABI."""
 
-    def __init__(self, cfg: Config, device="cuda"):
+    def __init__(self, cfg: Config, device="cuda", k_scale: Optional[float] = None):
         import block_sparse_causal_b200 as uf
         self.uf = uf
         self.cfg = cfg
-        self.win = uf.KVWindow(cfg.B, cfg.G, cfg.W, cfg.Lc, cfg.blk, cfg.D, device=device)
+        self.win = uf.KVWindow(cfg.B, cfg.G, cfg.W, cfg.Lc, cfg.blk, cfg.D, device=device, k_scale=k_scale)
         self.win.reset()
         self.device = device
 
@@ -64,6 +64,17 @@ class GpuStream:
         lse = torch.full((cfg.B, cfg.H, cfg.Lc), float("nan"), dtype=torch.float32, device=self.device)
         scale = 1.0 / math.sqrt(cfg.D) if scale is None else scale
         self.uf.uf_block_sparse_attn(q, cfg.H, self.win.desc, idx, cnt, k, scale, o, lse)
+        return o, lse
+
+    def attention_fp8(self, q_cpu, q_scale: float, idx=None, cnt=None, k=0, scale=None):
+        """FP8-score attention over the window's e4m3 K (window made with k_scale)."""
+        cfg = self.cfg
+        q = q_cpu.to(self.device)
+        o = torch.full((cfg.B, cfg.Lc, cfg.H, cfg.D), float("nan"), dtype=torch.bfloat16, device=self.device)
+        lse = torch.full((cfg.B, cfg.H, cfg.Lc), float("nan"), dtype=torch.float32, device=self.device)
+        scale = 1.0 / math.sqrt(cfg.D) if scale is None else scale
+        self.uf.uf_block_sparse_attn_fp8k(q, cfg.H, self.win.desc, self.win.k8, q_scale, self.win.k_scale, idx,
+                                          cnt, k, scale, o, lse)
         return o, lse
 
 
@@ -111,6 +122,25 @@ class OracleStream:
             sub_cnt = None if cnt is None else cnt[:, h:h + 1]
             O, L = oracle.block_sparse_attention(qh, self.head_window(h), cfg.blk, sub_idx, sub_cnt, scale,
                                                  items=[(b, 0, i) for (b, _, i) in its])
+            for (b, _, i) in its:
+                s0, e0 = i * cfg.blk, min(cfg.Lc, (i + 1) * cfg.blk)
+                res[(b, h, i)] = (O[b, s0:e0, 0, :], L[b, 0, s0:e0])
+        return res
+
+    def attention_fp8(self, q_cpu, items: Sequence[Tuple[int, int, int]], q_scale: float, k_scale: float,
+                      idx=None, cnt=None, scale=None):
+        """oracle.fp8_scores_attention per head, as ``attention``."""
+        cfg = self.cfg
+        res = {}
+        by_head: Dict[int, List[Tuple[int, int, int]]] = {}
+        for it in items:
+            by_head.setdefault(it[1], []).append(it)
+        for h, its in by_head.items():
+            qh = to_f64(q_cpu[:, :, h:h + 1])
+            sub_idx = None if idx is None else idx[:, h:h + 1]
+            sub_cnt = None if cnt is None else cnt[:, h:h + 1]
+            O, L = oracle.fp8_scores_attention(qh, self.head_window(h), cfg.blk, q_scale, k_scale, sub_idx,
+                                               sub_cnt, scale, items=[(b, 0, i) for (b, _, i) in its])
             for (b, _, i) in its:
                 s0, e0 = i * cfg.blk, min(cfg.Lc, (i + 1) * cfg.blk)
                 res[(b, h, i)] = (O[b, s0:e0, 0, :], L[b, 0, s0:e0])
