@@ -6,15 +6,18 @@
 // keeps its top-k highest-scoring blocks.
 //
 // One thread block per (TQ = 8 consecutive q-blocks, query head h, batch b),
-// 256 threads, two thread blocks per SM:
-//   1. pool: TMA copies each q-block's slice of Q (BLK tokens x 128 channels,
-//      two 64-channel panels) into a double-buffered shared-memory ring, so a
-//      whole slice is in flight while the previous one is reduced; each
-//      thread sums a channel pair over a quarter of the tokens in fp32;
-//   2. score: pooled K (written by the append call, one fp32 row per window
-//      block) is staged 32 rows at a time in shared memory; each warp takes 4
-//      kv rows, each lane an eighth of the head dim for all 8 q-blocks, and
-//      three xor-shuffles finish the dot products;
+// 256 threads (one warp per q-block), two thread blocks per SM:
+//   0. warp 0 starts bulk copies of the pooled K (written by the append call,
+//      one fp32 row per window block, 512 bytes; a window chunk's rows are
+//      contiguous, so one copy per run of a chunk's rows) into a ring of 3
+//      tiles of 32 rows, so the first tiles arrive while Q is pooled;
+//   1. pool: warp w sums q-block i0 + w over its tokens in fp32, each lane 8
+//      channels of every other token with 16-byte loads, 16 in flight;
+//   2. score: each lane keeps 4 channels of the 8 pooled queries in
+//      registers (as fp32 pairs for the packed f32x2 FMA); each warp takes 4
+//      kv rows of a tile, one 16-byte read per row and lane, and a 5-step
+//      reduce-scatter of the 8 partial dot products; the consumed tile's slot
+//      is refilled;
 //   3. select: one warp per q-block row finds the (k-1)-th largest
 //      non-diagonal score by a 32-step bitwise search over order-preserving
 //      integer keys, takes every key above it plus the lowest-index keys equal
@@ -26,13 +29,15 @@
 namespace uf {
 
 constexpr int MASK_TQ = 8;        // q-blocks per thread block (= warps)
-constexpr int MASK_KT = 32;       // pooled-K rows per shared-memory tile
-constexpr int MASK_KSTRIDE = 144; // padded row stride (floats): conflict-free float4 reads
-constexpr int MASK_QBUF = 2;      // q-block slices in flight per thread block
+constexpr int MASK_LOG_TQ = 3;
+constexpr int MASK_THREADS = 32 * MASK_TQ;
+constexpr int MASK_KT = 32;       // pooled-K rows per tile
+constexpr int MASK_KSTAGE = 3;    // pooled-K tiles in flight
+constexpr int MASK_QLOADS = 16;   // 16-byte Q loads in flight per lane
 
 // Dynamic shared memory of the mask kernel for a window of nkv_max blocks.
-__host__ __device__ constexpr int mask_smem_bytes(int blk, int nkv_max) {
-  return 1024 + MASK_QBUF * blk * 256 + (MASK_TQ * 128 + 2 * 4 * 128 + MASK_KT * MASK_KSTRIDE + MASK_TQ * nkv_max) * 4;
+__host__ __device__ constexpr int mask_smem_bytes(int nkv_max) {
+  return (MASK_KSTAGE * MASK_KT * 128 + MASK_TQ * 128 + MASK_TQ * nkv_max) * 4;
 }
 
 struct MaskParams {
@@ -65,18 +70,15 @@ __device__ __forceinline__ int warp_excl_scan(int v, int lane) {
 }
 
 template <int BLK, int MAXPER>
-__global__ void __launch_bounds__(256, 2) block_mask_kernel(const __grid_constant__ CUtensorMap tmQ, const MaskParams p) {
+__global__ void __launch_bounds__(MASK_THREADS, 2) block_mask_kernel(const MaskParams p) {
   constexpr int D = 128;
-  constexpr int QSLICE = BLK * 256;                     // bytes of one q-block slice (two panels)
-  extern __shared__ uint8_t mraw[];
-  uint8_t *mbase = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(mraw) + 1023) & ~uintptr_t(1023));
-  uint8_t *s_qbuf = mbase;                              // [QBUF][2 panels][BLK][128 B]
-  float *s_qpool = reinterpret_cast<float *>(mbase + MASK_QBUF * QSLICE);   // [TQ][D]
-  float *s_red = s_qpool + MASK_TQ * D;                 // [2][4][D]
-  float *s_kt = s_red + 2 * 4 * D;                      // [KT][KSTRIDE]
-  float *s_sc = s_kt + MASK_KT * MASK_KSTRIDE;          // [TQ][W*nb]
+  constexpr long long kWait = 1LL << 31;
+  extern __shared__ __align__(128) float mraw[];
+  float *s_kt = mraw;                                   // [KSTAGE][KT][D]
+  float *s_qpool = s_kt + MASK_KSTAGE * MASK_KT * D;    // [TQ][D]
+  float *s_sc = s_qpool + MASK_TQ * D;                  // [TQ][W*nb]
   __shared__ int32_t s_meta[3];
-  __shared__ uint64_t bar_q[MASK_QBUF];
+  __shared__ uint64_t bar_k[MASK_KSTAGE];
   __shared__ int32_t s_abort;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -96,7 +98,7 @@ __global__ void __launch_bounds__(256, 2) block_mask_kernel(const __grid_constan
     s_meta[0] = start;
     s_meta[1] = n;
     s_meta[2] = anc;
-    for (int q = 0; q < MASK_QBUF; ++q) mbar_init(&bar_q[q], 1);
+    for (int q = 0; q < MASK_KSTAGE; ++q) mbar_init(&bar_k[q], 1);
     s_abort = 0;
     fence_mbar_init();
   }
@@ -113,104 +115,133 @@ __global__ void __launch_bounds__(256, 2) block_mask_kernel(const __grid_constan
     return;
   }
 
-  // ---- 1. pool the query blocks -------------------------------------------
-  auto load_slice = [&](int tq) {
-    uint64_t *bar = &bar_q[tq % MASK_QBUF];
-    uint8_t *dst = s_qbuf + (tq % MASK_QBUF) * QSLICE;
-    mbar_arrive_expect_tx(bar, QSLICE);
-    tma_load_4d(dst, &tmQ, bar, 0, h, (i0 + tq) * BLK, b);
-    tma_load_4d(dst + QSLICE / 2, &tmQ, bar, 64, h, (i0 + tq) * BLK, b);
-  };
-  if (tid == 0)
-    for (int tq = 0; tq < min(MASK_QBUF, tq_count); ++tq) load_slice(tq);
-  const int cp = tid & 63, rg = tid >> 6;                // channel pair, quarter of the tokens
-  const int pnl = cp >> 5, cpo = (cp & 31) * 4;          // panel and byte offset of the pair in a row
-  for (int tq = 0; tq < tq_count; ++tq) {
-    const int t0 = (i0 + tq) * BLK;
-    const int ntok = min(BLK, p.Lc - t0);                // tokens past Lc were zero-filled by TMA
-    if (!wait_bounded(&bar_q[tq % MASK_QBUF], (tq / MASK_QBUF) & 1, &s_abort, 1LL << 31)) break;
-    const uint8_t *slice = s_qbuf + (tq % MASK_QBUF) * QSLICE + pnl * (QSLICE / 2) + cpo;
-    float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
-#pragma unroll 8
-    for (int r = rg * (BLK / 4); r < (rg + 1) * (BLK / 4); r += 2) {
-      const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(slice + r * 128));
-      const float2 g2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(slice + (r + 1) * 128));
-      a0 += f.x;
-      a1 += f.y;
-      b0 += g2.x;
-      b1 += g2.y;
+  // ---- 0. pooled-K tiles: one 512-byte bulk copy per window block ----------
+  const float *kp_head = p.kpool + (static_cast<size_t>(b) * p.G + g) * nkv_max * D;
+  const int ntiles = (NKV + MASK_KT - 1) / MASK_KT;
+  auto issue_tile = [&](int t) {          // all lanes of warp 0
+    const int st = t % MASK_KSTAGE, j0 = t * MASK_KT;
+    const int rows = min(MASK_KT, NKV - j0);
+    if (lane == 0) mbar_arrive_expect_tx(&bar_k[st], static_cast<uint32_t>(rows) * D * 4);
+    __syncwarp();
+    if (lane < rows) {
+      const int j = j0 + lane;
+      const int c = j / p.nb, rr = j - c * p.nb;
+      if (lane == 0 || rr == 0) {         // first row of a run of one chunk's rows
+        const int len = min(rows - lane, p.nb - rr);
+        const int slot = window_slot(c, start, p.W, anchor);
+        bulk_load(s_kt + (st * MASK_KT + lane) * D, kp_head + (static_cast<size_t>(slot) * p.nb + rr) * D,
+                  static_cast<uint32_t>(len) * D * 4, &bar_k[st]);
+      }
     }
-    float *red = s_red + (tq & 1) * 4 * D + rg * D;
-    red[2 * cp] = a0 + b0;
-    red[2 * cp + 1] = a1 + b1;
-    __syncthreads();                                     // slice consumed, partial sums visible
-    if (tid == 0 && tq + MASK_QBUF < tq_count) load_slice(tq + MASK_QBUF);
-    if (tid < D) {
-      const float *rr = s_red + (tq & 1) * 4 * D;
-      s_qpool[tq * D + tid] = ((rr[tid] + rr[D + tid]) + (rr[2 * D + tid] + rr[3 * D + tid])) / static_cast<float>(ntok);
+  };
+  int issued = 0;                         // tiles issued (warp 0's count)
+  if (warp == 0)
+    for (; issued < min(MASK_KSTAGE, ntiles); ++issued) issue_tile(issued);
+
+  // ---- 1. pool the query blocks: warp w takes q-block i0 + w ----------------
+  {
+    const int cg = lane & 15, rpar = lane >> 4;         // channels 8 cg .. 8 cg + 7, token parity
+    float acc[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+    const int t0 = (i0 + warp) * BLK;
+    const int ntok = warp < tq_count ? min(BLK, p.Lc - t0) : 0;
+    const size_t tok_stride = static_cast<size_t>(p.H) * D;
+    const __nv_bfloat16 *qb = p.q + ((static_cast<size_t>(b) * p.Lc + t0) * p.H + h) * D + cg * 8;
+#pragma unroll 1
+    for (int r0 = 0; r0 < ntok; r0 += 2 * MASK_QLOADS) {
+      uint4 v[MASK_QLOADS];
+#pragma unroll
+      for (int m = 0; m < MASK_QLOADS; ++m) {
+        const int r = r0 + 2 * m + rpar;
+        v[m] = r < ntok ? __ldg(reinterpret_cast<const uint4 *>(qb + r * tok_stride)) : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int m = 0; m < MASK_QLOADS; ++m) {
+        const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&v[m]);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = __bfloat1622float2(h2[e]);
+          acc[2 * e] += f.x;
+          acc[2 * e + 1] += f.y;
+        }
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], 16);
+    if (lane < 16) {
+      const float inv = ntok > 0 ? 1.0f / static_cast<float>(ntok) : 0.f;
+      float4 *dst = reinterpret_cast<float4 *>(s_qpool + warp * D + cg * 8);
+      dst[0] = make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
+      dst[1] = make_float4(acc[4] * inv, acc[5] * inv, acc[6] * inv, acc[7] * inv);
     }
   }
-  for (int e = tid; e < (MASK_TQ - tq_count) * D; e += blockDim.x) s_qpool[tq_count * D + e] = 0.f;
+  __syncthreads();                                      // s_qpool complete
 
   // ---- 2. pooled scores against every block of the window -----------------
-  const float *kp_head = p.kpool + (static_cast<size_t>(b) * p.G + g) * nkv_max * D;
-  const int jr = lane >> 3, dq = lane & 7;
-  // this thread's share of a pooled-K tile: 4 float4 of rows (e >> 5), e = it*256 + tid
-  auto fetch = [&](int j0, float4 (&v)[4]) {
+  // lane l keeps channels 4l .. 4l + 3 of the 8 pooled queries in registers,
+  // query (i ^ s) in slot i with s = lane >> 2, as fp32 pairs (slots 2i, 2i+1).
+  // Per kv row: one 16-byte read, 16 packed FMAs, then a reduce-scatter over
+  // the 32 lanes: at the steps xor 16, 8, 4 every lane keeps the lower half
+  // of its slots and sends the upper half (its partner's slot order is the
+  // same set of queries, so no selects), then xor 2 and 1 sum; each lane ends
+  // with the full dot product of query s.
+  static_assert(MASK_TQ == 8, "slot order below assumes 8 queries");
+  const int s_ord = lane >> 2;
+  uint64_t q2[MASK_TQ / 2][4];
 #pragma unroll
-    for (int it = 0; it < 4; ++it) {
-      const int e = it * 256 + tid;
-      const int j = j0 + (e >> 5);
-      v[it] = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (j < NKV) {
-        const int c = j / p.nb, rr = j - c * p.nb;
-        const int slot = window_slot(c, start, p.W, anchor);
-        v[it] = __ldg(reinterpret_cast<const float4 *>(kp_head + (static_cast<size_t>(slot) * p.nb + rr) * D) + (e & 31));
-      }
-    }
-  };
-  float4 nxt[4];
-  fetch(0, nxt);
-  for (int j0 = 0; j0 < NKV; j0 += MASK_KT) {
-    __syncthreads();   // previous tile fully consumed (and qpool complete on the first pass)
-#pragma unroll
-    for (int it = 0; it < 4; ++it) {
-      const int e = it * 256 + tid;
-      *reinterpret_cast<float4 *>(&s_kt[(e >> 5) * MASK_KSTRIDE + (e & 31) * 4]) = nxt[it];
-    }
-    __syncthreads();
-    if (j0 + MASK_KT < NKV) fetch(j0 + MASK_KT, nxt);   // in flight while this tile is scored
-    const int jl = warp * 4 + jr;
-    float acc[MASK_TQ];
-#pragma unroll
-    for (int t = 0; t < MASK_TQ; ++t) acc[t] = 0.f;
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      const int d = c * 32 + dq * 4;
-      const float4 kv = *reinterpret_cast<const float4 *>(&s_kt[jl * MASK_KSTRIDE + d]);
-#pragma unroll
-      for (int t = 0; t < MASK_TQ; ++t) {
-        const float4 qv = *reinterpret_cast<const float4 *>(&s_qpool[t * D + d]);
-        acc[t] = fmaf(qv.x, kv.x, acc[t]);
-        acc[t] = fmaf(qv.y, kv.y, acc[t]);
-        acc[t] = fmaf(qv.z, kv.z, acc[t]);
-        acc[t] = fmaf(qv.w, kv.w, acc[t]);
-      }
-    }
-#pragma unroll
-    for (int t = 0; t < MASK_TQ; ++t) {
-      acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], 1);
-      acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], 2);
-      acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], 4);
-    }
-    float mine = acc[0];
-#pragma unroll
-    for (int t = 1; t < MASK_TQ; ++t)
-      if (dq == t) mine = acc[t];
-    const int j = j0 + jl;
-    if (j < NKV) s_sc[dq * nkv_max + j] = mine * p.scale;
+  for (int i = 0; i < MASK_TQ / 2; ++i) {
+    const float4 lo = *reinterpret_cast<const float4 *>(&s_qpool[((2 * i) ^ s_ord) * D + 4 * lane]);
+    const float4 hi = *reinterpret_cast<const float4 *>(&s_qpool[((2 * i + 1) ^ s_ord) * D + 4 * lane]);
+    q2[i][0] = f2_pack(lo.x, hi.x);
+    q2[i][1] = f2_pack(lo.y, hi.y);
+    q2[i][2] = f2_pack(lo.z, hi.z);
+    q2[i][3] = f2_pack(lo.w, hi.w);
   }
-  __syncthreads();
+  const int q_own = s_ord;
+  for (int t = 0; t < ntiles; ++t) {
+    const int st = t % MASK_KSTAGE;
+    if (wait_bounded(&bar_k[st], (t / MASK_KSTAGE) & 1, &s_abort, kWait)) {
+      const float *kt = s_kt + st * MASK_KT * D;
+#pragma unroll
+      for (int r = 0; r < MASK_KT / MASK_TQ; ++r) {
+        const int jl = r * MASK_TQ + warp;
+        const float4 kv = *reinterpret_cast<const float4 *>(&kt[jl * D + 4 * lane]);
+        const uint64_t k0 = f2_pack(kv.x, kv.x), k1 = f2_pack(kv.y, kv.y), k2 = f2_pack(kv.z, kv.z),
+                       k3 = f2_pack(kv.w, kv.w);
+        float a[MASK_TQ];
+#pragma unroll
+        for (int i = 0; i < MASK_TQ / 2; ++i) {
+          const uint64_t acc = f2_fma(q2[i][3], k3, f2_fma(q2[i][2], k2, f2_fma(q2[i][1], k1, f2_mul(q2[i][0], k0))));
+          f2_unpack(acc, a[2 * i], a[2 * i + 1]);
+        }
+#pragma unroll
+        for (int step = 0; step < MASK_LOG_TQ; ++step) {
+          const int m = 16 >> step, half = MASK_TQ >> (step + 1);
+#pragma unroll
+          for (int i = 0; i < half; ++i) a[i] += __shfl_xor_sync(0xffffffffu, a[i + half], m);
+        }
+        float sum = a[0];
+#pragma unroll
+        for (int m = 16 >> MASK_LOG_TQ; m >= 1; m >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, m);
+        const int j = t * MASK_KT + jl;
+        if ((lane & ((32 >> MASK_LOG_TQ) - 1)) == 0 && j < NKV) s_sc[q_own * nkv_max + j] = sum * p.scale;
+      }
+    }
+    __syncthreads();                                    // tile consumed; every wait of this tile is over
+    if (*reinterpret_cast<volatile int32_t *>(&s_abort)) break;
+    if (warp == 0 && issued < ntiles) issue_tile(issued++);
+  }
+  if (*reinterpret_cast<volatile int32_t *>(&s_abort)) {
+    // a wait gave up: let the copies still in flight land (bounded) before exiting
+    if (tid == 0)
+      for (int t = max(0, issued - MASK_KSTAGE); t < issued; ++t) {
+        const long long t0 = clock64();
+        while (!mbar_try_wait(&bar_k[t % MASK_KSTAGE], (t / MASK_KSTAGE) & 1) && clock64() - t0 < kWait) {
+        }
+      }
+    return;
+  }
 
   // ---- 3. per-row selection (one warp per q-block) --------------------------
   if (warp < tq_count) {

@@ -144,8 +144,28 @@ int32_t sm_count(int *out) {
 }
 
 std::atomic<int> g_attn128f8_smem[kMaxDevices], g_attn64f8_smem[kMaxDevices];
-std::atomic<int> g_attn128_smem[kMaxDevices], g_attn64_smem[kMaxDevices], g_mask128_smem[kMaxDevices],
-    g_mask64_smem[kMaxDevices], g_mask128b_smem[kMaxDevices], g_mask64b_smem[kMaxDevices];
+std::atomic<int> g_attn128_smem[kMaxDevices], g_attn64_smem[kMaxDevices];
+
+// One mask kernel instance per (block size, selection keys per lane).
+template <int BLK, int MAXPER>
+int32_t launch_mask(const uf::MaskParams &p, dim3 grid, int smem, cudaStream_t st) {
+  static std::atomic<int> smem_set[kMaxDevices];
+  const int32_t e = ensure_smem(uf::block_mask_kernel<BLK, MAXPER>, smem, smem_set);
+  if (e != UF_OK) return e;
+  uf::block_mask_kernel<BLK, MAXPER><<<grid, uf::MASK_THREADS, smem, st>>>(p);
+  return UF_OK;
+}
+
+// keys per lane of the selection: the smallest of 8, 12, 16, 24, 32 >= ceil(W * nb / 32)
+template <int BLK>
+int32_t launch_mask_per(const uf::MaskParams &p, int nkv_max, dim3 grid, int smem, cudaStream_t st) {
+  const int per = (nkv_max + 31) / 32;
+  if (per <= 8) return launch_mask<BLK, 8>(p, grid, smem, st);
+  if (per <= 12) return launch_mask<BLK, 12>(p, grid, smem, st);
+  if (per <= 16) return launch_mask<BLK, 16>(p, grid, smem, st);
+  if (per <= 24) return launch_mask<BLK, 24>(p, grid, smem, st);
+  return launch_mask<BLK, 32>(p, grid, smem, st);
+}
 
 }  // namespace
 
@@ -458,38 +478,12 @@ int32_t uf_block_mask_local(const void *q, int32_t H, const uf_kv_cache *c, int3
   p.local = local;
   p.local_only = (flags & UF_MASK_LOCAL_ONLY) ? 1 : 0;
   p.scale = 1.0f / sqrtf(static_cast<float>(c->D));
-  const int smem = uf::mask_smem_bytes(c->blk, nkv_max);
-  // Q slices for the pooling: {channels, heads, tokens, batch}, box {64, 1, blk, 1}, no swizzle
-  CUtensorMap tq;
-  {
-    const cuuint64_t dims[4] = {128, static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(c->Lc),
-                                static_cast<cuuint64_t>(c->B)};
-    const cuuint64_t strides[3] = {256, static_cast<cuuint64_t>(H) * 256, static_cast<cuuint64_t>(c->Lc) * H * 256};
-    const cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(c->blk), 1};
-    if (!make_map(&tq, q, 4, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE)) return UF_ECUDA;
-  }
+  const int smem = uf::mask_smem_bytes(nkv_max);
   const dim3 grid(ceil_div(nb, uf::MASK_TQ), H, c->B);
   const cudaStream_t st = reinterpret_cast<cudaStream_t>(s);
   cudaGetLastError();
-  // keys per lane of the selection: ceil(W*nb / 32) <= MAXPER
-  int32_t e = UF_OK;
-  if (c->blk == 128) {
-    if (nkv_max <= 512) {
-      e = ensure_smem(uf::block_mask_kernel<128, 16>, smem, g_mask128_smem);
-      if (e == UF_OK) uf::block_mask_kernel<128, 16><<<grid, 256, smem, st>>>(tq, p);
-    } else {
-      e = ensure_smem(uf::block_mask_kernel<128, 32>, smem, g_mask128b_smem);
-      if (e == UF_OK) uf::block_mask_kernel<128, 32><<<grid, 256, smem, st>>>(tq, p);
-    }
-  } else {
-    if (nkv_max <= 512) {
-      e = ensure_smem(uf::block_mask_kernel<64, 16>, smem, g_mask64_smem);
-      if (e == UF_OK) uf::block_mask_kernel<64, 16><<<grid, 256, smem, st>>>(tq, p);
-    } else {
-      e = ensure_smem(uf::block_mask_kernel<64, 32>, smem, g_mask64b_smem);
-      if (e == UF_OK) uf::block_mask_kernel<64, 32><<<grid, 256, smem, st>>>(tq, p);
-    }
-  }
+  const int32_t e = c->blk == 128 ? launch_mask_per<128>(p, nkv_max, grid, smem, st)
+                                  : launch_mask_per<64>(p, nkv_max, grid, smem, st);
   if (e != UF_OK) return e;
   return launch_status();
 }
