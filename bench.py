@@ -224,14 +224,17 @@ def run_ours(args, cfg, rank, world, device):
     q_rot = torch.empty_like(dev_chunks[0]["q"]) if (args.rope or args.tiled) else None
     o_tiled = torch.empty_like(o) if args.tiled else None
 
-    def attention(q, idx_s, cnt_s, k_s, out):
+    def attention(q, idx_s, cnt_s, k_s, out, lse_out):
         if args.fp8:
             uf.uf_block_sparse_attn_fp8k(q, cfg.H, win.desc, win.k8, q_scale, k_scale, idx_s, cnt_s, k_s, scale,
-                                         out, lse)
+                                         out, lse_out)
         else:
-            uf.uf_block_sparse_attn(q, cfg.H, win.desc, idx_s, cnt_s, k_s, scale, out, lse)
+            uf.uf_block_sparse_attn(q, cfg.H, win.desc, idx_s, cnt_s, k_s, scale, out, lse_out)
 
-    def step(s, chunk, ev=None):
+    def step(s, chunk, ev=None, o_out=None, lse_out=None):
+        # every call goes to the current stream; outputs to o / lse unless given
+        o_out = o if o_out is None else o_out
+        lse_out = lse if lse_out is None else lse_out
         # RoPE variant: the chunk sits at stream position (W + s) * Lc
         pos0 = (cfg.W + s) * cfg.Lc
         if ev is not None:
@@ -253,7 +256,7 @@ def run_ours(args, cfg, rank, world, device):
         if cfg.dense:
             if ev is not None:
                 ev[2].record(stream)
-            attention(q, None, None, 0, o_tiled if args.tiled else o)
+            attention(q, None, None, 0, o_tiled if args.tiled else o_out, lse_out)
         else:
             if args.mask_local or args.mask_local_only:
                 uf.uf_block_mask_local(q, cfg.H, win.desc, k, args.mask_local, local_flags, idx[s], cnt[s])
@@ -261,11 +264,11 @@ def run_ours(args, cfg, rank, world, device):
                 uf.uf_block_mask(q, cfg.H, win.desc, k, idx[s], cnt[s])
             if ev is not None:
                 ev[2].record(stream)
-            attention(q, idx[s], cnt[s], k, o_tiled if args.tiled else o)
+            attention(q, idx[s], cnt[s], k, o_tiled if args.tiled else o_out, lse_out)
         if ev is not None:
             ev[3].record(stream)
         if args.tiled:                             # O back to row-major order (in the step, not in "attn")
-            uf.uf_tile_tokens(o_tiled, o, cfg.B, cfg.grid, cfg.H, inverse=True)
+            uf.uf_tile_tokens(o_tiled, o_out, cfg.B, cfg.grid, cfg.H, inverse=True)
 
     launches_per_step = (2 if cfg.dense else 3) + (1 if args.rope else 0) + (2 if args.tiled else 0)
     for s in range(args.warmup):
@@ -303,39 +306,44 @@ def run_ours(args, cfg, rank, world, device):
     flops_per_step = sum(flops) / len(flops)
     max_ms = all_max(elapsed_ms, world, device)
 
-    # e2e: the same steps through the C ABI from pinned host buffers, with the
-    # inputs copied in and O / LSE copied out inside the timed region
+    # e2e: the same steps through the C ABI from pinned host buffers, with each
+    # chunk's inputs copied in and its O / LSE copied out inside the timed
+    # region; ChunkPipeline overlaps chunk n's copy in and chunk n - 2's copy
+    # out with chunk n - 1's compute (three streams, two staging slots)
+    from block_sparse_causal_b200.pipeline import ChunkPipeline
     pinned = [{n: x.pin_memory() for n, x in c.items()} for c in host_chunks[cfg.W:]]
-    stage = {n: torch.empty_like(x, device=device) for n, x in dev_chunks[0].items()}
-    o_host = torch.empty(o.shape, dtype=o.dtype).pin_memory()
-    lse_host = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+    host_out = [{"o": torch.empty(o.shape, dtype=o.dtype).pin_memory(),
+                 "lse": torch.empty(lse.shape, dtype=lse.dtype).pin_memory()} for _ in range(2)]
     e2e_steps = max(3, min(args.steps, 50))
+    e2e_count = [0]
 
-    def e2e_step(s):
-        src = pinned[s % n_distinct]
-        for n in ("q", "k", "v"):
-            stage[n].copy_(src[n], non_blocking=True)
-        step(s % n_idx, stage)
-        o_host.copy_(o, non_blocking=True)
-        lse_host.copy_(lse, non_blocking=True)
+    def pipe_step(din, dout, st):
+        step(e2e_count[0] % n_idx, din, o_out=dout["o"], lse_out=dout["lse"])
+        e2e_count[0] += 1
 
-    e2e_step(0)
-    torch.cuda.synchronize()
+    pipe = ChunkPipeline({n: (tuple(x.shape), x.dtype) for n, x in dev_chunks[0].items()},
+                         {"o": (tuple(o.shape), o.dtype), "lse": (tuple(lse.shape), lse.dtype)},
+                         pipe_step, depth=2, device=device)
+    pipe.submit(pinned[0], host_out[0])
+    pipe.synchronize()
     sampler2 = ClockSampler(device)
     sampler2.start()
     barrier(world)
     torch.cuda.synchronize()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
+    e0.record(pipe.h2d)
     for s in range(e2e_steps):
-        e2e_step(s + 1)
-    e1.record(stream)
+        pipe.submit(pinned[(s + 1) % n_distinct], host_out[(s + 1) % 2])
+    e1.record(pipe.d2h)          # after the last copy out, which follows every earlier step
+    pipe.synchronize()
     torch.cuda.synchronize()
     barrier(world)
     sampler2.stop()
+    if uf.uf_get_error() != 0:
+        raise RuntimeError("device-side error during the end-to-end steps")
     e2e_ms = all_max(e0.elapsed_time(e1), world, device) / e2e_steps
-    h2d = sum(stage[n].numel() * stage[n].element_size() for n in ("q", "k", "v"))
+    h2d = sum(x.numel() * x.element_size() for x in pinned[0].values())
     d2h = o.numel() * o.element_size() + lse.numel() * lse.element_size()
 
     ms_per_step = max_ms / args.steps
@@ -403,7 +411,8 @@ def run_ours(args, cfg, rank, world, device):
                            + (" x 4/3: QK at the nominal e4m3/bf16 ratio of 2" if args.fp8 else ""),
         },
         "e2e": {"value": world * flops_per_step / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
-                "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+                "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "overlap": "ChunkPipeline: copy in / compute / copy out on three streams, two slots"},
         "clocks": clocks,
         "gpu_launches": launches_per_step * args.steps,
     }

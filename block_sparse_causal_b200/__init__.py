@@ -9,6 +9,7 @@ from ._uf import (UF_APPEND_ANCHOR, UF_APPEND_REPLACE_NEWEST, UF_EBOUNDS, UF_ECU
                   uf_block_sparse_attn, uf_block_sparse_attn_fp8k, uf_kv_append_fp8k, uf_debug_wait_timeout, uf_kv_append_rope, uf_kv_append_tiled, uf_rope, uf_tile_tokens,
                   uf_get_error, uf_kv_append, uf_kv_cache_bytes, uf_kv_cache_init, uf_kv_reset, uf_set_wait_limit,
                   uf_version)
+from .pipeline import ChunkPipeline
 from .window import KVWindow
 
 __all__ = [
@@ -16,5 +17,5 @@ __all__ = [
     "UF_MASK_LOCAL_ONLY", "UF_OK", "UfError", "UfKvCache", "strerror", "uf_block_mask", "uf_block_mask_local",
     "uf_block_sparse_attn", "uf_block_sparse_attn_fp8k", "uf_kv_append_fp8k", "uf_kv_append_rope", "uf_kv_append_tiled", "uf_rope", "uf_tile_tokens", "uf_debug_wait_timeout",
     "uf_get_error", "uf_kv_append", "uf_kv_cache_bytes", "uf_kv_cache_init", "uf_kv_reset", "uf_set_wait_limit",
-    "uf_version", "KVWindow",
+    "uf_version", "KVWindow", "ChunkPipeline",
 ]
