@@ -177,7 +177,7 @@ __global__ void __launch_bounds__(256) kv_append_kernel(const AppendParams p) {
   constexpr bool ROPE = MODE == APPEND_ROPE, TILED = MODE == APPEND_TILED, FP8K = MODE == APPEND_FP8K;
   constexpr int D = 128;
   constexpr int PASSES = BLK / 16;
-  const int r = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int g = blockIdx.x, r = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, tl = tid >> 4, dc = tid & 15;
 
   __shared__ int32_t s_plan[4];

@@ -215,7 +215,7 @@ int32_t append_impl(uf_kv_cache *c, const void *k_new, const void *v_new, int32_
   if (tiled) p.grid = *tile_grid;
   p.k8 = static_cast<uint8_t *>(k8);
   p.k8_inv_scale = 1.0f / k_scale;
-  const dim3 grid(p.nb, c->G, c->B);
+  const dim3 grid(c->G, p.nb, c->B);   // KV heads fastest: concurrent blocks read each token's heads together
   cudaGetLastError();
   const cudaStream_t st0 = reinterpret_cast<cudaStream_t>(s);
   const int mode = rope ? uf::APPEND_ROPE : tiled ? uf::APPEND_TILED : k8 ? uf::APPEND_FP8K : uf::APPEND_PLAIN;
