@@ -405,6 +405,7 @@ def run_ours(args, cfg, rank, world, device):
             "peak": peak,
             "unit": "TFLOP/s",
             "frac": attn_tflops / peak,
+            "frac_of_sustained": attn_tflops / (peaks["bf16_tflops_sustained"] * (4.0 / 3.0 if args.fp8 else 1.0)),
             "traffic": traffic,
             "kernel": "uf::attn_kernel<%d, %s>" % (cfg.blk, "true" if args.fp8 else "false"),
             "peak_source": f"{peaks_src} bf16 dense burst (cuBLAS 8192^3)"
@@ -478,8 +479,18 @@ def blas_threads():
 
 def cpu_baseline(cfg, seed, local=0, local_only=False, anchor=False, fp8=False):
     flops, dt, desc = OracleSample(cfg, seed, local, local_only, anchor, fp8).run(n_items=10_000, budget_s=12.0)
-    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
-            "sample": desc + f", {dt:.1f} s of fp64 numpy", "seconds": dt}
+    out = {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+           "sample": desc + f", {dt:.1f} s of fp64 numpy", "seconds": dt}
+    # the oracle on one core for the tiny workload (its whole mask and attention, repeated)
+    try:
+        from threadpoolctl import threadpool_limits
+        with threadpool_limits(1):
+            f1, t1, d1 = OracleSample(CONFIGS["tiny"], seed).run(n_items=10_000, budget_s=3.0)
+        out["tiny_1core"] = {"value": f1 / t1 / 1e12, "unit": "TFLOP/s", "cores": 1,
+                             "sample": "tiny workload: " + d1 + f", {t1:.1f} s"}
+    except ImportError:
+        out["tiny_1core"] = None
+    return out
 
 
 def run_reference(args, cfg):
