@@ -15,7 +15,8 @@
 // Both products run on the tensor core with the A operand in tensor memory
 // and a K-major B operand in shared memory:
 //   S_t = Q K_t^T   (Q staged by TMA in shared memory, copied into tensor
-//                    memory by the softmax threads once per item)
+//                    memory once per item by the QK issuer with tcgen05.cp;
+//                    the FP8 variant's e4m3 Q by the softmax threads)
 //   O  += P_t V_t   (P_t written to tensor memory by the softmax; V is stored
 //                    transposed in the window, so V_t^T is K-major too)
 // Tensor memory (512 columns): S buffers 0 and 1 [0,128) [128,256), O
@@ -169,7 +170,7 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
   // per-item barriers: Q landed in shared memory / free in tensor memory /
   // copied into tensor memory; O read by the epilogue; (m, l) exchange; O
   // staged by each warpgroup; staging tile read by the output stores
-  __shared__ uint64_t bar_qfull, bar_qtfree, bar_q, bar_ofree, bar_l, bar_st[2], bar_ostore;
+  __shared__ uint64_t bar_qfull, bar_qtfree, bar_q, bar_qcp, bar_ofree, bar_l, bar_st[2], bar_ostore;
   // per-block barriers
   __shared__ uint64_t bar_kfull[ATTN_KSTAGE], bar_kempty[ATTN_KSTAGE];
   __shared__ uint64_t bar_vfull[ATTN_VSTAGE], bar_vempty[ATTN_VSTAGE];
@@ -190,6 +191,7 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
     mbar_init(&bar_qfull, 1);
     mbar_init(&bar_qtfree, 1);
     mbar_init(&bar_q, ATTN_SOFTMAX_THREADS);
+    mbar_init(&bar_qcp, 1);
     mbar_init(&bar_ofree, ATTN_SOFTMAX_THREADS);
     mbar_init(&bar_l, ATTN_SOFTMAX_THREADS);
     mbar_init(&bar_st[0], ATTN_SOFTMAX_THREADS / 2);
@@ -315,8 +317,24 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
         }
         if (item < p.items) request_q(it);
         while (item < p.items && ok) {
-          // the item's Q is in tensor memory
-          if (!(ok = wait_bounded(&bar_q, kq & 1, abort_flag, p.wait_limit))) break;
+          if (FP8) {
+            // the softmax threads have written the item's e4m3 Q into tensor memory
+            if (!(ok = wait_bounded(&bar_q, kq & 1, abort_flag, p.wait_limit))) break;
+          } else {
+            // once the previous item's QK products have read Q's columns and
+            // this item's Q has landed: copy it into tensor memory here, one
+            // K = 16 slice per copy, and wait for the copies
+            if (kq > 0 && !(ok = wait_bounded(&bar_qtfree, (kq - 1) & 1, abort_flag, p.wait_limit))) break;
+            if (!(ok = wait_bounded(&bar_qfull, kq & 1, abort_flag, p.wait_limit))) break;
+            tc_fence_after();
+            const uint32_t q_base = smem_u32(sQ);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+              tmem_cp_128x256b(tb + TM_Q + kk * 8,
+                               sdesc_sw128(q_base + (kk >> 2) * (L::Q_BYTES / 2) + (kk & 3) * 32, 16, 1024));
+            mma_commit(&bar_qcp);
+            if (!(ok = wait_bounded(&bar_qcp, kq & 1, abort_flag, p.wait_limit))) break;
+          }
           tc_fence_after();
           int item_next = p.items;
           AttnItem nxt;
@@ -514,7 +532,7 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
 
     AttnItem cur;
     int item = next_live(blockIdx.x, cur);
-    bool ok = item >= p.items || load_q(0);
+    bool ok = item >= p.items || !FP8 || load_q(0);
     int kq = 0, g0 = 0;   // live items and kept blocks of this thread block so far
     while (item < p.items && ok) {
       const int n = cur.n;
@@ -651,7 +669,7 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
       // QK products run during this item's epilogue
       AttnItem nxt;
       const int item_next = next_live(item + gridDim.x, nxt);
-      if (item_next < p.items && !(ok = load_q(kq + 1))) break;
+      if (FP8 && item_next < p.items && !(ok = load_q(kq + 1))) break;
       // ---------------------------------------------------------- epilogue --
       // every PV of the item has completed once its last one has (one issuing
       // thread, completions in order)
@@ -674,6 +692,9 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(&bar_ofree);
+      // (bf16 path: the QK issuer's copy of the next item's Q out of the staging
+      // tile has completed)
+      if (!FP8 && item_next < p.items && !(ok = wwait(&bar_qcp, (kq + 1) & 1))) break;
       // this warpgroup's 64-column half of the bf16 row -> the staging tile
       // (the next item's Q has left it), 128-byte swizzled like a TMA tile:
       // 16-byte chunk c of row r at chunk c ^ (r mod 8)

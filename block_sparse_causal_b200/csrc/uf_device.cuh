@@ -221,6 +221,14 @@ __device__ __forceinline__ void mma_commit(uint64_t *bar) {
                : "memory");
 }
 
+// Shared memory -> tensor memory, issued by one thread: 128 rows of 256 bits
+// (one K = 16 slice of a bf16 operand) from the matrix `desc` describes into
+// lanes 0..127, columns taddr .. taddr + 7.  Completion is tracked like an MMA
+// (tcgen05.commit).
+__device__ __forceinline__ void tmem_cp_128x256b(uint32_t taddr, uint64_t desc) {
+  asm volatile("tcgen05.cp.cta_group::1.128x256b [%0], %1;" ::"r"(taddr), "l"(desc) : "memory");
+}
+
 // 32 consecutive columns of this thread's lane (32x32b shape, x32).
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
   asm volatile(
