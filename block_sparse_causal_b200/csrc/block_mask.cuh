@@ -7,17 +7,18 @@
 //
 // One thread block per (TQ = 8 consecutive q-blocks, query head h, batch b),
 // 256 threads (one warp per q-block), two thread blocks per SM:
-//   0. warp 0 starts bulk copies of the pooled K (written by the append call,
-//      one fp32 row per window block, 512 bytes; a window chunk's rows are
-//      contiguous, so one copy per run of a chunk's rows) into a ring of 3
-//      tiles of 32 rows, so the first tiles arrive while Q is pooled;
+//   0. the pooled K (written by the append call, one fp32 row per window
+//      block) streams through a ring of 4 tiles of 32 rows: stage s holds
+//      tiles s, s + 4, ... and belongs to warps 2s and 2s + 1, which fill it
+//      (one bulk copy per row, into rows padded to 132 floats) and consume it;
+//      the first four tiles are requested at entry, so they arrive while Q is
+//      pooled;
 //   1. pool: warp w sums q-block i0 + w over its tokens in fp32, each lane 8
 //      channels of every other token with 16-byte loads, 16 in flight;
-//   2. score: each lane keeps 4 channels of the 8 pooled queries in
-//      registers (as fp32 pairs for the packed f32x2 FMA); each warp takes 4
-//      kv rows of a tile, one 16-byte read per row and lane, and a 5-step
-//      reduce-scatter of the 8 partial dot products; the consumed tile's slot
-//      is refilled;
+//   2. score: on the tensor core, m16n8k8 tf32 MMAs with fp32 accuracy by a
+//      hi / lo split of both operands (hi.hi + hi.lo + lo.hi); each warp
+//      takes one 16-row half of its stage's tiles against the 8 pooled
+//      queries (held in registers as B fragments);
 //   3. select: one warp per q-block row finds the (k-1)-th largest
 //      non-diagonal score by a 32-step bitwise search over order-preserving
 //      integer keys, takes every key above it plus the lowest-index keys equal
@@ -32,12 +33,14 @@ constexpr int MASK_TQ = 8;        // q-blocks per thread block (= warps)
 constexpr int MASK_LOG_TQ = 3;
 constexpr int MASK_THREADS = 32 * MASK_TQ;
 constexpr int MASK_KT = 32;       // pooled-K rows per tile
-constexpr int MASK_KSTAGE = 3;    // pooled-K tiles in flight
+constexpr int MASK_KSTAGE = 4;    // pooled-K tiles in flight (stage s: warps 2s, 2s + 1)
+constexpr int MASK_KSTRIDE = 132; // floats per pooled-K row in shared memory (conflict-free A fragments)
+static_assert(2 * MASK_KSTAGE == MASK_TQ, "each warp pair owns one stage");
 constexpr int MASK_QLOADS = 16;   // 16-byte Q loads in flight per lane
 
 // Dynamic shared memory of the mask kernel for a window of nkv_max blocks.
 __host__ __device__ constexpr int mask_smem_bytes(int nkv_max) {
-  return (MASK_KSTAGE * MASK_KT * 128 + MASK_TQ * 128 + MASK_TQ * nkv_max) * 4;
+  return (MASK_KSTAGE * MASK_KT * MASK_KSTRIDE + MASK_TQ * 128 + MASK_TQ * nkv_max) * 4;
 }
 
 struct MaskParams {
@@ -74,8 +77,8 @@ __global__ void __launch_bounds__(MASK_THREADS, 2) block_mask_kernel(const MaskP
   constexpr int D = 128;
   constexpr long long kWait = 1LL << 31;
   extern __shared__ __align__(128) float mraw[];
-  float *s_kt = mraw;                                   // [KSTAGE][KT][D]
-  float *s_qpool = s_kt + MASK_KSTAGE * MASK_KT * D;    // [TQ][D]
+  float *s_kt = mraw;                                   // [KSTAGE][KT][KSTRIDE]
+  float *s_qpool = s_kt + MASK_KSTAGE * MASK_KT * MASK_KSTRIDE;   // [TQ][D]
   float *s_sc = s_qpool + MASK_TQ * D;                  // [TQ][W*nb]
   __shared__ int32_t s_meta[3];
   __shared__ uint64_t bar_k[MASK_KSTAGE];
@@ -118,7 +121,8 @@ __global__ void __launch_bounds__(MASK_THREADS, 2) block_mask_kernel(const MaskP
   // ---- 0. pooled-K tiles: one 512-byte bulk copy per window block ----------
   const float *kp_head = p.kpool + (static_cast<size_t>(b) * p.G + g) * nkv_max * D;
   const int ntiles = (NKV + MASK_KT - 1) / MASK_KT;
-  auto issue_tile = [&](int t) {          // all lanes of warp 0
+  const int pair = warp >> 1;            // this warp's stage; tiles pair, pair + KSTAGE, ...
+  auto issue_tile = [&](int t) {          // all lanes of warp 2 * (t mod KSTAGE)
     const int st = t % MASK_KSTAGE, j0 = t * MASK_KT;
     const int rows = min(MASK_KT, NKV - j0);
     if (lane == 0) mbar_arrive_expect_tx(&bar_k[st], static_cast<uint32_t>(rows) * D * 4);
@@ -126,17 +130,16 @@ __global__ void __launch_bounds__(MASK_THREADS, 2) block_mask_kernel(const MaskP
     if (lane < rows) {
       const int j = j0 + lane;
       const int c = j / p.nb, rr = j - c * p.nb;
-      if (lane == 0 || rr == 0) {         // first row of a run of one chunk's rows
-        const int len = min(rows - lane, p.nb - rr);
-        const int slot = window_slot(c, start, p.W, anchor);
-        bulk_load(s_kt + (st * MASK_KT + lane) * D, kp_head + (static_cast<size_t>(slot) * p.nb + rr) * D,
-                  static_cast<uint32_t>(len) * D * 4, &bar_k[st]);
-      }
+      const int slot = window_slot(c, start, p.W, anchor);
+      bulk_load(s_kt + (st * MASK_KT + lane) * MASK_KSTRIDE, kp_head + (static_cast<size_t>(slot) * p.nb + rr) * D,
+                D * 4, &bar_k[st]);
     }
   };
-  int issued = 0;                         // tiles issued (warp 0's count)
-  if (warp == 0)
-    for (; issued < min(MASK_KSTAGE, ntiles); ++issued) issue_tile(issued);
+  int last_issued = -1;                   // (even warps) last tile issued into this warp pair's stage
+  if ((warp & 1) == 0 && pair < ntiles) {
+    issue_tile(pair);
+    last_issued = pair;
+  }
 
   // ---- 1. pool the query blocks: warp w takes q-block i0 + w ----------------
   {
@@ -179,67 +182,69 @@ __global__ void __launch_bounds__(MASK_THREADS, 2) block_mask_kernel(const MaskP
   __syncthreads();                                      // s_qpool complete
 
   // ---- 2. pooled scores against every block of the window -----------------
-  // lane l keeps channels 4l .. 4l + 3 of the 8 pooled queries in registers,
-  // query (i ^ s) in slot i with s = lane >> 2, as fp32 pairs (slots 2i, 2i+1).
-  // Per kv row: one 16-byte read, 16 packed FMAs, then a reduce-scatter over
-  // the 32 lanes: at the steps xor 16, 8, 4 every lane keeps the lower half
-  // of its slots and sends the upper half (its partner's slot order is the
-  // same set of queries, so no selects), then xor 2 and 1 sum; each lane ends
-  // with the full dot product of query s.
-  static_assert(MASK_TQ == 8, "slot order below assumes 8 queries");
-  const int s_ord = lane >> 2;
-  uint64_t q2[MASK_TQ / 2][4];
+  // D[16 kv rows x 8 queries] += A[rows x 8 channels] B[8 channels x queries]
+  // over 16 channel steps, each operand split as x = hi + lo (tf32 parts).
+  // Fragments (m16n8k8, gid = lane / 4, tig = lane % 4): A rows gid, gid + 8
+  // and channels tig, tig + 4; B query gid, channels tig, tig + 4; D rows
+  // gid, gid + 8 and queries 2 tig, 2 tig + 1.
+  const int gid = lane >> 2, tig = lane & 3;
+  uint32_t bh[D / 8][2], bl[D / 8][2];
 #pragma unroll
-  for (int i = 0; i < MASK_TQ / 2; ++i) {
-    const float4 lo = *reinterpret_cast<const float4 *>(&s_qpool[((2 * i) ^ s_ord) * D + 4 * lane]);
-    const float4 hi = *reinterpret_cast<const float4 *>(&s_qpool[((2 * i + 1) ^ s_ord) * D + 4 * lane]);
-    q2[i][0] = f2_pack(lo.x, hi.x);
-    q2[i][1] = f2_pack(lo.y, hi.y);
-    q2[i][2] = f2_pack(lo.z, hi.z);
-    q2[i][3] = f2_pack(lo.w, hi.w);
-  }
-  const int q_own = s_ord;
-  for (int t = 0; t < ntiles; ++t) {
-    const int st = t % MASK_KSTAGE;
-    if (wait_bounded(&bar_k[st], (t / MASK_KSTAGE) & 1, &s_abort, kWait)) {
-      const float *kt = s_kt + st * MASK_KT * D;
+  for (int kk = 0; kk < D / 8; ++kk)
 #pragma unroll
-      for (int r = 0; r < MASK_KT / MASK_TQ; ++r) {
-        const int jl = r * MASK_TQ + warp;
-        const float4 kv = *reinterpret_cast<const float4 *>(&kt[jl * D + 4 * lane]);
-        const uint64_t k0 = f2_pack(kv.x, kv.x), k1 = f2_pack(kv.y, kv.y), k2 = f2_pack(kv.z, kv.z),
-                       k3 = f2_pack(kv.w, kv.w);
-        float a[MASK_TQ];
+    for (int e = 0; e < 2; ++e) {
+      const float v = s_qpool[gid * D + kk * 8 + tig + 4 * e];
+      bh[kk][e] = to_tf32(v);
+      bl[kk][e] = to_tf32(v - __uint_as_float(bh[kk][e]));
+    }
+  const int mh = warp & 1;                // this warp's 16-row half of each tile
+  for (int t = pair; t < ntiles; t += MASK_KSTAGE) {
+    // both warps of the pair run the same iterations (the named barrier below
+    // needs both); after an abort the waits return at once and nothing is issued
+    if (wait_bounded(&bar_k[pair], (t / MASK_KSTAGE) & 1, &s_abort, kWait)) {
+      const float *kt = s_kt + (pair * MASK_KT + mh * 16) * MASK_KSTRIDE;
+      float d[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int i = 0; i < MASK_TQ / 2; ++i) {
-          const uint64_t acc = f2_fma(q2[i][3], k3, f2_fma(q2[i][2], k2, f2_fma(q2[i][1], k1, f2_mul(q2[i][0], k0))));
-          f2_unpack(acc, a[2 * i], a[2 * i + 1]);
+      for (int kk = 0; kk < D / 8; ++kk) {
+        const float av[4] = {kt[gid * MASK_KSTRIDE + kk * 8 + tig], kt[(gid + 8) * MASK_KSTRIDE + kk * 8 + tig],
+                             kt[gid * MASK_KSTRIDE + kk * 8 + tig + 4],
+                             kt[(gid + 8) * MASK_KSTRIDE + kk * 8 + tig + 4]};
+        uint32_t ah[4], al[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          ah[e] = to_tf32(av[e]);
+          al[e] = to_tf32(av[e] - __uint_as_float(ah[e]));
         }
-#pragma unroll
-        for (int step = 0; step < MASK_LOG_TQ; ++step) {
-          const int m = 16 >> step, half = MASK_TQ >> (step + 1);
-#pragma unroll
-          for (int i = 0; i < half; ++i) a[i] += __shfl_xor_sync(0xffffffffu, a[i + half], m);
-        }
-        float sum = a[0];
-#pragma unroll
-        for (int m = 16 >> MASK_LOG_TQ; m >= 1; m >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, m);
-        const int j = t * MASK_KT + jl;
-        if ((lane & ((32 >> MASK_LOG_TQ) - 1)) == 0 && j < NKV) s_sc[q_own * nkv_max + j] = sum * p.scale;
+        mma_tf32_16x8x8(d, ah, bh[kk]);
+        mma_tf32_16x8x8(d, ah, bl[kk]);
+        mma_tf32_16x8x8(d, al, bh[kk]);
+      }
+      const int j = t * MASK_KT + mh * 16 + gid;
+      if (j < NKV) {
+        s_sc[(2 * tig) * nkv_max + j] = d[0] * p.scale;
+        s_sc[(2 * tig + 1) * nkv_max + j] = d[1] * p.scale;
+      }
+      if (j + 8 < NKV) {
+        s_sc[(2 * tig) * nkv_max + j + 8] = d[2] * p.scale;
+        s_sc[(2 * tig + 1) * nkv_max + j + 8] = d[3] * p.scale;
       }
     }
-    __syncthreads();                                    // tile consumed; every wait of this tile is over
-    if (*reinterpret_cast<volatile int32_t *>(&s_abort)) break;
-    if (warp == 0 && issued < ntiles) issue_tile(issued++);
+    // the pair is done with the stage: its even warp refills it
+    named_barrier(1 + pair, 64);
+    if (mh == 0 && t + MASK_KSTAGE < ntiles && !*reinterpret_cast<volatile int32_t *>(&s_abort)) {
+      issue_tile(t + MASK_KSTAGE);
+      last_issued = t + MASK_KSTAGE;
+    }
   }
+  __syncthreads();                                      // every score written
   if (*reinterpret_cast<volatile int32_t *>(&s_abort)) {
-    // a wait gave up: let the copies still in flight land (bounded) before exiting
-    if (tid == 0)
-      for (int t = max(0, issued - MASK_KSTAGE); t < issued; ++t) {
-        const long long t0 = clock64();
-        while (!mbar_try_wait(&bar_k[t % MASK_KSTAGE], (t / MASK_KSTAGE) & 1) && clock64() - t0 < kWait) {
-        }
+    // a wait gave up: each stage's filler lets its last copy land (bounded)
+    // before the block exits
+    if (mh == 0 && lane == 0 && last_issued >= 0) {
+      const long long t0 = clock64();
+      while (!mbar_try_wait(&bar_k[pair], (last_issued / MASK_KSTAGE) & 1) && clock64() - t0 < kWait) {
       }
+    }
     return;
   }
 

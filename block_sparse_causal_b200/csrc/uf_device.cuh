@@ -308,6 +308,27 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+// fp32 -> tf32 (round to nearest, ties away), kept in a 32-bit register.
+__device__ __forceinline__ uint32_t to_tf32(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return r;
+}
+
+// D += A B on the tensor core (warp-wide, m16n8k8, tf32 in, fp32 accumulate).
+__device__ __forceinline__ void mma_tf32_16x8x8(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+// Barrier among `count` threads (a multiple of 32) on named barrier `id` (1..15).
+__device__ __forceinline__ void named_barrier(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
 // Packed fp32 pairs (sm_100 f32x2 arithmetic): one instruction for two lanes of work.
 __device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
   uint64_t r;
