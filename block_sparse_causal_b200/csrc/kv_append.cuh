@@ -15,10 +15,10 @@
 // tokens contiguous) so that the attention's PV product reads it as a K-major
 // operand: each thread loads an 8-token x 8-channel bf16 tile, transposes it
 // in registers with byte permutes and writes 8 sixteen-byte token runs, so
-// each warp writes two contiguous 256-byte runs per instruction.  The last
-// thread block to finish commits the new window state to meta; every block
-// read the old state before counting in, so no block can observe a
-// half-updated window.
+// each warp writes two contiguous 256-byte runs per instruction.  Each block
+// counts itself in right after reading the old window state; the last one to
+// count in commits the new state to meta, so no block can observe a
+// half-updated window and no block waits for its own writes before retiring.
 //
 // With RoPE (uf_kv_append_rope) each K row is rotated at its stream position
 // before it is stored and pooled.  Rotary scores depend only on position
@@ -199,6 +199,18 @@ __global__ void __launch_bounds__(256) kv_append_kernel(const AppendParams p) {
     s_plan[1] = start2;
     s_plan[2] = n2;
     s_plan[3] = anc2;
+    // count this block's read of the window state; the last block to read it
+    // commits the new state (no block reads it again, and the next kernel on
+    // the stream sees this one's writes), so nothing waits at the block's end
+    __threadfence();
+    const int32_t total = static_cast<int32_t>(gridDim.x * gridDim.y * gridDim.z);
+    const int32_t prev = atomicAdd(p.meta + 2, 1);
+    if (prev == total - 1) {
+      atomicExch(p.meta + 0, start2);
+      atomicExch(p.meta + 1, n2);
+      atomicExch(p.meta + 3, anc2);
+      atomicExch(p.meta + 2, 0);
+    }
   }
   if (TILED && tid < BLK && r * BLK + tid < p.Lc) s_src[tid] = tile_token(p.grid, r * BLK + tid);
   __syncthreads();
@@ -311,20 +323,6 @@ __global__ void __launch_bounds__(256) kv_append_kernel(const AppendParams p) {
     p.kpool[prow * D + tid] = s / static_cast<float>(cnt);
   }
 
-  // commit the new window state once every block has read the old one
-  __syncthreads();
-  if (tid == 0) {
-    __threadfence();
-    const int32_t total = static_cast<int32_t>(gridDim.x * gridDim.y * gridDim.z);
-    const int32_t prev = atomicAdd(p.meta + 2, 1);
-    if (prev == total - 1) {
-      atomicExch(p.meta + 0, s_plan[1]);
-      atomicExch(p.meta + 1, s_plan[2]);
-      atomicExch(p.meta + 3, s_plan[3]);
-      atomicExch(p.meta + 2, 0);
-      __threadfence();
-    }
-  }
 }
 
 }  // namespace uf
