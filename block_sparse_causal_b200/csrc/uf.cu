@@ -362,7 +362,7 @@ const char *uf_strerror(int32_t status) {
     case UF_ECUDA: return "UF_ECUDA: CUDA call or kernel launch failed";
     case UF_ETIMEOUT: return "UF_ETIMEOUT: a kernel pipeline wait exceeded its bound";
     case UF_EBOUNDS: return "UF_EBOUNDS: a kernel found an out-of-range index or window state";
-    case UF_EUNSUPPORTED: return "UF_EUNSUPPORTED: request not supported by this build";
+    case UF_EUNSUPPORTED: return "UF_EUNSUPPORTED: valid request this library does not implement";
     default: return "UF_UNKNOWN";
   }
 }

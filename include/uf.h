@@ -53,7 +53,7 @@ typedef enum uf_status {
   UF_ECUDA = 2,       /* a CUDA runtime / driver call or launch failed         */
   UF_ETIMEOUT = 3,    /* a kernel pipeline wait exceeded its bound (device)    */
   UF_EBOUNDS = 4,     /* a kernel found an out-of-range index or state (device)*/
-  UF_EUNSUPPORTED = 5 /* valid request this build does not implement           */
+  UF_EUNSUPPORTED = 5 /* valid request this library does not implement         */
 } uf_status;
 
 /* Flags of uf_kv_append. */
