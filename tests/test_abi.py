@@ -166,6 +166,15 @@ def test_calls_reject_bad_arguments_before_launch(uf):
         uf.uf_block_sparse_attn(q, 2, c, None, None, 0, 0.088, FakeTensor(0xA00001), None, stream=0)
 
 
+def test_mask_beyond_1024_window_blocks_is_unsupported(uf):
+    # 5 chunks of 205 blocks = 1025 window blocks: one more than the selection holds
+    c = _cache(uf, G=1, W=5, Lc=205 * 128)
+    c.host_n_valid = 1
+    with pytest.raises(uf.UfError) as e:
+        uf.uf_block_mask(FakeTensor(0x500000), 1, c, 2, FakeTensor(0x800000), FakeTensor(0x900000), None, stream=0)
+    assert e.value.status == uf.UF_EUNSUPPORTED
+
+
 def test_wait_limit_bounds(uf):
     with pytest.raises(uf.UfError):
         uf.uf_set_wait_limit(10)

@@ -254,6 +254,21 @@ def test_full_size_sparse(name):
     assert_attention_ok(cfg, o2, lse2, orc.attention(last["q"], agree, oidx, ocnt), name + " e2e")
 
 
+def test_largest_window_the_mask_supports():
+    # W * nb = 1024 window blocks (32 selection keys per lane): 8 chunks of 128
+    # blocks, 64-token blocks with a ragged last one (8191 = 127 * 64 + 63)
+    cfg = scaled(CONFIGS["1k_sr"], H=2, G=1, Lc=8191, W=8, blk=64, density=0.1)
+    assert cfg.W * cfg.nb == 1024
+    gpu, orc, last, idx, cnt, scores, om, k = _mask_case(cfg, seed=12, want_scores=False)
+    rows, exact, ties, bad = compare_masks(cfg, idx, cnt, om, k)
+    assert not bad, bad[:3]
+    assert exact >= rows - 2
+    oidx, ocnt = oracle_idx_array(cfg, om)
+    o, lse = gpu.attention(last["q"], torch.from_numpy(oidx).cuda(), torch.from_numpy(ocnt).cuda(), oidx.shape[-1])
+    items = sample_items(cfg, 8, seed=3)
+    assert_attention_ok(cfg, o, lse, orc.attention(last["q"], items, oidx, ocnt), "1024-block window")
+
+
 def test_full_size_480p_dense():
     cfg = CONFIGS["480p_dense"]
     gpu, orc = GpuStream(cfg), OracleStream(cfg)
