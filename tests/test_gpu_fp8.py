@@ -159,3 +159,15 @@ def test_fp8_full_size_1k():
     items = sample_items(cfg, 12, seed=5)
     torch.cuda.synchronize()
     assert_attention_ok(cfg, o, lse, orc.attention_fp8(last["q"], items, qs, ks, oidx, ocnt), "1k fp8")
+
+
+def test_fp8_full_size_2k():
+    cfg = CONFIGS["2k_sr"]
+    gpu, orc, last, qs, ks = _stream(cfg, cfg.W + 1, seed=1)
+    k = cfg.k_for()
+    oidx, ocnt = oracle_idx_array(cfg, orc.mask(last["q"], k))
+    o, lse = gpu.attention_fp8(last["q"], qs, torch.from_numpy(oidx).cuda(), torch.from_numpy(ocnt).cuda(),
+                               oidx.shape[-1])
+    items = sample_items(cfg, 10, seed=6)
+    torch.cuda.synchronize()
+    assert_attention_ok(cfg, o, lse, orc.attention_fp8(last["q"], items, qs, ks, oidx, ocnt), "2k fp8")
