@@ -16,9 +16,9 @@
 // operand: each thread loads an 8-token x 8-channel bf16 tile, transposes it
 // in registers with byte permutes and writes 8 sixteen-byte token runs, so
 // each warp writes two contiguous 256-byte runs per instruction.  Each block
-// counts itself in right after reading the old window state; the last one to
-// count in commits the new state to meta, so no block can observe a
-// half-updated window and no block waits for its own writes before retiring.
+// counts itself out when done (it read the old window state at its start);
+// the last one commits the new state to meta, so no block can observe a
+// half-updated window, and no block waits for its own writes to drain.
 //
 // With RoPE (uf_kv_append_rope) each K row is rotated at its stream position
 // before it is stored and pooled.  Rotary scores depend only on position
@@ -199,18 +199,6 @@ __global__ void __launch_bounds__(256) kv_append_kernel(const AppendParams p) {
     s_plan[1] = start2;
     s_plan[2] = n2;
     s_plan[3] = anc2;
-    // count this block's read of the window state; the last block to read it
-    // commits the new state (no block reads it again, and the next kernel on
-    // the stream sees this one's writes), so nothing waits at the block's end
-    __threadfence();
-    const int32_t total = static_cast<int32_t>(gridDim.x * gridDim.y * gridDim.z);
-    const int32_t prev = atomicAdd(p.meta + 2, 1);
-    if (prev == total - 1) {
-      atomicExch(p.meta + 0, start2);
-      atomicExch(p.meta + 1, n2);
-      atomicExch(p.meta + 3, anc2);
-      atomicExch(p.meta + 2, 0);
-    }
   }
   if (TILED && tid < BLK && r * BLK + tid < p.Lc) s_src[tid] = tile_token(p.grid, r * BLK + tid);
   __syncthreads();
@@ -323,6 +311,20 @@ __global__ void __launch_bounds__(256) kv_append_kernel(const AppendParams p) {
     p.kpool[prow * D + tid] = s / static_cast<float>(cnt);
   }
 
+  // count this block out; the last one commits the new window state.  Thread
+  // 0 read the old state at the start (its value fed the plan above), so every
+  // block has read it before the last count, and no block reads it again; no
+  // fence: the next kernel on the stream sees all of this one's writes.
+  if (tid == 0) {
+    const int32_t total = static_cast<int32_t>(gridDim.x * gridDim.y * gridDim.z);
+    const int32_t prev = atomicAdd(p.meta + 2, 1);
+    if (prev == total - 1) {
+      atomicExch(p.meta + 0, s_plan[1]);
+      atomicExch(p.meta + 1, s_plan[2]);
+      atomicExch(p.meta + 3, s_plan[3]);
+      atomicExch(p.meta + 2, 0);
+    }
+  }
 }
 
 }  // namespace uf
