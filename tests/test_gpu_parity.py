@@ -254,6 +254,22 @@ def test_full_size_sparse(name):
     assert_attention_ok(cfg, o2, lse2, orc.attention(last["q"], agree, oidx, ocnt), name + " e2e")
 
 
+def test_single_chunk_window():
+    # W = 1: every append replaces the only chunk; the window is the newest chunk
+    cfg = scaled(CONFIGS["1k_sr"], H=4, G=2, Lc=1000, W=1)
+    gpu, orc, last, idx, cnt, scores, om, k = _mask_case(cfg, seed=13, n_chunks=3, want_scores=True)
+    rows, exact, ties, bad = compare_masks(cfg, idx, cnt, om, k)
+    assert not bad, bad[:3]
+    assert exact >= rows - 1
+    assert gpu.win.meta[1].item() == 1
+    oidx, ocnt = oracle_idx_array(cfg, om)
+    o, lse = gpu.attention(last["q"], torch.from_numpy(oidx).cuda(), torch.from_numpy(ocnt).cuda(), oidx.shape[-1])
+    items = [(b, h, i) for b in range(cfg.B) for h in range(cfg.H) for i in range(cfg.nb)]
+    assert_attention_ok(cfg, o, lse, orc.attention(last["q"], items, oidx, ocnt), "W = 1")
+    od, lsed = gpu.attention(last["q"])
+    assert_attention_ok(cfg, od, lsed, orc.attention(last["q"], items), "W = 1 dense")
+
+
 def test_largest_window_the_mask_supports():
     # W * nb = 1024 window blocks (32 selection keys per lane): 8 chunks of 128
     # blocks, 64-token blocks with a ragged last one (8191 = 127 * 64 + 63)
