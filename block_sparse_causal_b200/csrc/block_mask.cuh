@@ -30,7 +30,6 @@
 namespace uf {
 
 constexpr int MASK_TQ = 8;        // q-blocks per thread block (= warps)
-constexpr int MASK_LOG_TQ = 3;
 constexpr int MASK_THREADS = 32 * MASK_TQ;
 constexpr int MASK_KT = 32;       // pooled-K rows per tile
 constexpr int MASK_KSTAGE = 4;    // pooled-K tiles in flight (stage s: warps 2s, 2s + 1)
