@@ -39,6 +39,28 @@ def test_library_exports_every_declared_symbol(uf):
     assert set(declared_functions()) <= exported
 
 
+def declared_arity():
+    """Number of parameters of every uf_ prototype in the header."""
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    out = {}
+    for m in re.finditer(r"(uf_[a-z_0-9]+)\s*\(([^;{]*?)\)\s*;", text, flags=re.S):
+        args = m.group(2).strip()
+        out[m.group(1)] = 0 if args in ("", "void") else args.count(",") + 1
+    return out
+
+
+def test_binding_signatures_match_the_header(uf):
+    # every call the ctypes binding declares has the header's parameter count,
+    # and every declared call is bound
+    from block_sparse_causal_b200 import _uf
+    arity = declared_arity()
+    assert set(arity) == set(declared_functions())
+    for name, n in arity.items():
+        fn = getattr(_uf.lib, name)
+        assert fn.argtypes is not None, f"{name} is not bound"
+        assert len(fn.argtypes) == n, (name, len(fn.argtypes), n)
+
+
 def test_version_and_strerror(uf):
     assert uf.uf_version() >= 100
     for code in range(6):
