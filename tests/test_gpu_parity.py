@@ -270,6 +270,26 @@ def test_single_chunk_window():
     assert_attention_ok(cfg, od, lsed, orc.attention(last["q"], items), "W = 1 dense")
 
 
+def test_large_scores_exercise_the_rescale_path():
+    # queries scaled by 30: scores in the hundreds, rows sharply peaked, so the
+    # reference max rises by more than 2^8 many times within an item and O is
+    # rescaled in tensor memory; blocks in reversed order make it rise late
+    cfg = scaled(CONFIGS["1k_sr"], H=4, G=4, Lc=1000)
+    gpu, orc = GpuStream(cfg), OracleStream(cfg)
+    last = fill_window(cfg, 17, cfg.W, gpu, orc)
+    q = (last["q"].float() * 30).to(torch.bfloat16)
+    k = cfg.k_for()
+    oidx, ocnt = oracle_idx_array(cfg, orc.mask(q, k))
+    rev = np.ascontiguousarray(oidx[..., ::-1])
+    items = [(b, h, i) for b in range(cfg.B) for h in range(cfg.H) for i in range(cfg.nb)]
+    ref = orc.attention(q, items, oidx, ocnt)
+    for idx_arr in (oidx, rev):
+        o, lse = gpu.attention(q, torch.from_numpy(idx_arr).cuda(), torch.from_numpy(ocnt).cuda(), idx_arr.shape[-1])
+        assert_attention_ok(cfg, o, lse, ref, "large scores")
+    o, lse = gpu.attention(q)
+    assert_attention_ok(cfg, o, lse, orc.attention(q, items), "large scores dense")
+
+
 def test_largest_window_the_mask_supports():
     # W * nb = 1024 window blocks (32 selection keys per lane): 8 chunks of 128
     # blocks, 64-token blocks with a ragged last one (8191 = 127 * 64 + 63)
