@@ -347,7 +347,9 @@ def run_ours(args, cfg, rank, world, device):
     d2h = o.numel() * o.element_size() + lse.numel() * lse.element_size()
 
     ms_per_step = max_ms / args.steps
-    value = world * flops_per_step / (ms_per_step * 1e-3) / 1e12
+    # every rank ran its own seeded stream: the job's work is the sum of their kept FLOPs
+    job_flops_per_step = all_sum(flops_per_step, world, device)
+    value = job_flops_per_step / (ms_per_step * 1e-3) / 1e12
     peaks, peaks_src = load_peaks()
     attn_tflops = flops_per_step / (per["attn"] * 1e-3) / 1e12
     traffic = None if args.fp8 else attn_traffic_per_launch(args.config)
@@ -411,7 +413,7 @@ def run_ours(args, cfg, rank, world, device):
             "peak_source": f"{peaks_src} bf16 dense burst (cuBLAS 8192^3)"
                            + (" x 4/3: QK at the nominal e4m3/bf16 ratio of 2" if args.fp8 else ""),
         },
-        "e2e": {"value": world * flops_per_step / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+        "e2e": {"value": job_flops_per_step / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "overlap": "ChunkPipeline: copy in / compute / copy out on three streams, two slots"},
         "clocks": clocks,
@@ -524,6 +526,14 @@ def run_reference(args, cfg):
 def barrier(world):
     if world > 1:
         torch.distributed.barrier()
+
+
+def all_sum(x, world, device):
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.SUM)
+    return float(t.item())
 
 
 def all_max(x, world, device):

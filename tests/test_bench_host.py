@@ -79,6 +79,8 @@ def _rank_main(rank, world, port, out):
     bench.barrier(world)
     # each replica reports its own elapsed time; the job time is the slowest rank
     out[rank] = bench.all_max(10.0 + 5.0 * rank, world, "cpu")
+    # the job's work is the sum of every replica's kept FLOPs
+    out[(rank, "sum")] = bench.all_sum(1.0 + rank, world, "cpu")
     bench.barrier(world)
     dist.destroy_process_group()
 
@@ -95,8 +97,10 @@ def test_max_over_ranks_with_gloo():
         p.join(120)
         assert p.exitcode == 0
     assert out[0] == out[1] == 15.0
+    assert out[(0, "sum")] == out[(1, "sum")] == 3.0
 
 
 def test_world_of_one_needs_no_process_group():
     assert bench.all_max(3.5, 1, "cpu") == 3.5
+    assert bench.all_sum(3.5, 1, "cpu") == 3.5
     bench.barrier(1)
