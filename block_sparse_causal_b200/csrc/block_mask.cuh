@@ -19,10 +19,12 @@
 //      hi / lo split of both operands (hi.hi + hi.lo + lo.hi); each warp
 //      takes one 16-row half of its stage's tiles against the 8 pooled
 //      queries (held in registers as B fragments);
-//   3. select: one warp per q-block row finds the (k-1)-th largest
-//      non-diagonal score by a 32-step bitwise search over order-preserving
-//      integer keys, takes every key above it plus the lowest-index keys equal
-//      to it, and writes the kept ids in ascending order with the diagonal.
+//   3. select: one warp per q-block row forces the diagonal (or the local
+//      band around it), finds the need-th largest of the other scores (need =
+//      k minus the forced blocks) by a 32-step bitwise search over
+//      order-preserving integer keys, takes every key above it plus the
+//      lowest-index keys equal to it, and writes the kept ids in ascending
+//      order.
 #pragma once
 
 #include "uf_device.cuh"
