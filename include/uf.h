@@ -165,8 +165,8 @@ int32_t uf_kv_append(uf_kv_cache *c, const void *k_new, const void *v_new,
 /*
  * Rotary position embedding with positions relative to the window
  * (FlashDecoder, long video decoding: RoPE positions are assigned relative to
- * the current window rather than the absolute frame index; Algorithm 1:
- * "RoPE offset t * L_frm").  The pages do not give the rotation's form; it is
+ * the current window rather than the absolute frame index; Algorithm 1
+ * offsets the positions by the frame index times the tokens per frame).  The pages do not give the rotation's form; it is
  * RoFormer's (Su et al. 2021): channel pairs (x_2i, x_2i+1) rotate by
  * pos * theta_i, theta_i = base^(-2i / D).
  *
@@ -257,7 +257,8 @@ int32_t uf_block_mask(const void *q, int32_t H, const uf_kv_cache *c, int32_t k,
  * Block mask with a local sliding-window band (Ultra Flash notes, Method, key
  * design 3: each attention layer combines a local sliding-window mask with the
  * temporal causal mask, then keeps each head's top-k blocks; the ablation
- * table's "fixed local window instead of adaptive top-k" is the band alone).
+ * table's row that swaps adaptive top-k for a fixed local window is the band
+ * alone).
  * The pages do not define the band's shape; here it is the run of logical
  * kv blocks within `local` of the diagonal, [d_i - local, d_i + local]
  * clipped to [0, NKV).

@@ -23,7 +23,7 @@ Sources (page title, then section / equation):
 * FlashDecoder (xllm-io blog), Algorithm 1 (streaming inference): after each
   frame the cache becomes the tail (W_frm - 1) frames of the old cache followed
   by the new frame's K/V; causality comes from the processing order, not from a
-  token mask (Sec. 3.3, "causality through processing order").
+  token mask (Sec. 3.3).
 
 Readings taken where the pages are silent or ambiguous (each is listed in the
 design notes of the repository):
@@ -34,7 +34,7 @@ design notes of the repository):
 * The query chunk is the newest chunk of the window (it was appended just
   before attention).  Inside the window there is no token-level mask: each query
   token may attend to every token of every kept block, including blocks of its
-  own chunk ("chunk-causal").
+  own chunk (causal at chunk granularity).
 * Pooled block score = mean(q_block) . mean(k_block) / sqrt(D); no softmax is
   applied to pooled scores (it would not change the ranking).
 * Selection per (batch, query head, q-block i): the diagonal block
@@ -326,7 +326,8 @@ def rope(x: np.ndarray, pos: np.ndarray, base: float = 10000.0) -> np.ndarray:
     channel pairs (x_2i, x_2i+1) rotated by the angle pos * theta_i with
     theta_i = base^(-2i / D)).  The pages name RoPE but not its form
     (FlashDecoder, "long video decoding": positions relative to the current
-    window; Algorithm 1: "RoPE offset t * L_frm"); this is the published form.
+    window; Algorithm 1 offsets the positions by the frame index times the
+    tokens per frame); this is the published form.
 
     x [..., L, heads, D]; pos [L] integer positions of the L tokens.
     """
@@ -425,15 +426,15 @@ E4M3_MAX = 448.0
 
 def quantize_e4m3(x: np.ndarray, scale: float) -> np.ndarray:
     """Static-scale FP8 quantisation (FlashDecoder, inference optimisations:
-    statically calibrated FP8): the e4m3 value nearest to x / scale (ties to
-    even; e4m3 keeps 4 significant bits, exponent bias 7, subnormal spacing
-    2^-9, saturating at +-448), returned in e4m3 units as float64.
+    statically calibrated FP8): the e4m3 value nearest to the quotient
+    x / scale (ties to even; e4m3 keeps 4 significant bits, exponent bias 7,
+    subnormal spacing 2^-9, saturating at +-448), returned in e4m3 units as
+    float64.
 
-    The pages fix no precision for x / scale.  Because the quotient decides an
-    integer code, it is taken here as the kernels take it: in IEEE binary32,
-    x rounded to fp32 times the fp32 reciprocal of the fp32 scale."""
-    inv = np.float32(1.0) / np.float32(scale)
-    v = (np.asarray(x, dtype=np.float64).astype(np.float32) * inv).astype(np.float64)
+    The pages fix no precision for the quotient, so this takes its plain
+    definition: x / scale in float64 (relative error 2^-53, far below any
+    e4m3 spacing), then the rounding."""
+    v = np.asarray(x, dtype=np.float64) / float(scale)
     a = np.abs(v)
     e = np.floor(np.log2(np.where(a > 0, a, 1.0)))
     ulp = np.exp2(np.maximum(e, -6.0) - 3.0)             # normal spacing 2^(e-3); below 2^-6 the subnormal 2^-9

@@ -3,16 +3,19 @@ statically calibrated FP8): the e4m3 copy of K that the append writes, bit
 for bit, and the attention whose scores are e4m3 q . e4m3 k on the tensor
 cores, against the fp64 oracle's fp8_scores_attention on the same codes.
 
-The oracle quantises with the kernels' fp32 quotient, so both sides hold the
-same e4m3 codes; what remains between them is the fp32 accumulation of exact
-e4m3 products and the bf16 probabilities, as in the bf16 path, so the
-acceptance tolerances are the bf16 path's."""
+The oracle rounds the exact quotient x / scale; the kernels form it in fp32
+as x * fp32(1 / scale), within 2^-23 relative of the exact one.  The codes are
+compared with a near-boundary rule (uf_testlib.e4m3_codes_agree): equal,
+except where an e4m3 rounding boundary lies within that distance of the exact
+quotient.  Such flips are rare and move a score by one e4m3 step of one
+element, so the attention is held to the bf16 path's tolerances unchanged."""
 import numpy as np
 import pytest
 import torch
 
 import oracle
-from uf_testlib import (GpuStream, OracleStream, assert_attention_ok, oracle_idx_array, sample_items)
+from uf_testlib import (GpuStream, OracleStream, assert_attention_ok, e4m3_codes_agree, oracle_idx_array,
+                        sample_items)
 from workloads import CONFIGS, chunk_inputs, scaled
 
 pytestmark = [pytest.mark.gpu,
@@ -74,9 +77,30 @@ def test_fp8_k_codes_bit_exact(name, anchor):
         for c in range(orc.n_valid):
             slot = _slot(gpu.win, c)
             r0 = slot * gpu.win.lslot
-            want = oracle.quantize_e4m3(w.k[c][:, :, 0, :], ks)
-            assert np.array_equal(k8[:, g, r0:r0 + cfg.Lc], want), (g, c)
+            near, bad = e4m3_codes_agree(k8[:, g, r0:r0 + cfg.Lc], w.k[c][:, :, 0, :], ks)
+            assert not bad.any(), (g, c, int(bad.sum()))
             assert not raw[:, g, r0 + cfg.Lc:r0 + gpu.win.lslot].any(), "padding rows must be zero"
+
+
+def test_fp8_k_code_at_an_exact_midpoint():
+    # K = 175/512 with k_scale = 7/64: the exact quotient 3.125 is the midpoint
+    # between the e4m3 values 3.0 and 3.25 (the oracle takes 3.0, ties to even);
+    # the kernel's fp32 product lies just above it.  The near-boundary rule
+    # accepts either value there and nothing else
+    cfg = CASES["blk64"]
+    ks = 7.0 / 64.0
+    gpu = GpuStream(cfg, k_scale=ks)
+    inp = chunk_inputs(cfg, 25, 0)
+    inp["k"][:, : cfg.Lc // 2] = 175.0 / 512.0
+    gpu.append(inp)
+    torch.cuda.synchronize()
+    k8 = gpu.win.k8.view(torch.float8_e4m3fn).to(torch.float64).cpu().numpy()
+    r0 = _slot(gpu.win, 0) * gpu.win.lslot
+    got = k8[:, :, r0:r0 + cfg.Lc // 2]
+    assert set(np.unique(got).tolist()) <= {3.0, 3.25}
+    x = inp["k"][:, : cfg.Lc].double().numpy().transpose(0, 2, 1, 3)
+    near, bad = e4m3_codes_agree(k8[:, :, r0:r0 + cfg.Lc], x, ks)
+    assert not bad.any()
 
 
 @pytest.mark.parametrize("name", ["blk64", "gqa_w3", "sr_w3"])

@@ -719,17 +719,42 @@ def test_quantize_e4m3_matches_torch_float8():
     assert quantize_e4m3(np.array([1.0625, 1.1875]), 1.0).tolist() == [1.0, 1.25]    # ties to even
 
 
-def test_quantize_e4m3_scaled_decision_in_fp32():
-    # x / scale is taken as fp32(x) * fp32(1 / fp32(scale)) before the e4m3
-    # rounding; torch's own fp32 product and float8 cast give the same codes
+def test_quantize_e4m3_scaled_quotient_is_exact():
+    # power-of-two scales make x / scale exact in fp32 as well, so torch's
+    # float8 cast of the fp32 quotient is the reference there
     import torch
     from oracle import quantize_e4m3
     r = np.random.default_rng(16)
     x = (r.standard_normal(50000) * 3.0).astype(np.float32)
-    for scale in (0.01, 0.0123, 1.0 / 7.0, 3.3):
-        inv = torch.tensor(1.0, dtype=torch.float32) / torch.tensor(scale, dtype=torch.float32)
-        want = (torch.from_numpy(x) * inv).clamp(-448, 448).to(torch.float8_e4m3fn).to(torch.float64).numpy()
+    for scale in (2.0 ** -7, 2.0 ** -3, 0.5, 4.0):
+        want = (torch.from_numpy(x) / scale).clamp(-448, 448).to(torch.float8_e4m3fn).to(torch.float64).numpy()
         assert np.array_equal(quantize_e4m3(x, scale), want)
+
+
+def test_quantize_e4m3_rounds_the_exact_quotient_not_an_fp32_product():
+    # x = 175/512 and scale = 7/64 (both exact in bf16): x / scale = 25/8 =
+    # 3.125 exactly, the midpoint between the e4m3 values 3.0 (mantissa 100)
+    # and 3.25 (mantissa 101); ties to even give 3.0.  The fp32 reciprocal of
+    # 7/64 rounds up (64/7 = 9.142857142..., fp32 9.1428575516), so the fp32
+    # product x * fp32(1 / scale) = 3.1250002384 lies above the midpoint and
+    # would round to 3.25: an oracle that formed the quotient that way fails.
+    from oracle import quantize_e4m3
+    x, scale = 175.0 / 512.0, 7.0 / 64.0
+    assert quantize_e4m3(np.array([x, -x]), scale).tolist() == [3.0, -3.0]
+    inv32 = np.float32(1.0) / np.float32(scale)
+    assert float(np.float32(x) * inv32) > 3.125        # the fp32 product passes the midpoint
+    # just off the midpoint either way the nearest value wins
+    assert quantize_e4m3(np.array([3.125 * (1 + 2 ** -20), 3.125 * (1 - 2 ** -20)]), 1.0).tolist() == [3.25, 3.0]
+
+
+def test_e4m3_near_boundary_rule_of_the_gpu_comparison():
+    # the code comparison of the FP8 parity tests accepts a different code only
+    # next to an e4m3 rounding boundary, and only a neighbouring code
+    from uf_testlib import e4m3_codes_agree
+    x = np.array([175.0 / 512.0, 175.0 / 512.0, 175.0 / 512.0, 0.3, 0.3])
+    got = np.array([3.0, 3.25, 3.5, 2.75, 2.5])       # 0.3 / (7/64) = 2.742857 -> 2.75
+    near, bad = e4m3_codes_agree(got, x, 7.0 / 64.0)
+    assert near == 1 and bad.tolist() == [False, False, True, False, True]
 
 
 def test_quantize_e4m3_saturates_and_scales():

@@ -23,6 +23,9 @@ O_MAX_ABS = 2e-2
 O_MEAN_ABS = 2e-3
 LSE_ABS = 1e-3
 NEAR_TIE_REL = 1e-4
+# The kernels form the e4m3 quotient x / scale in fp32 as x * fp32(1 / scale):
+# two roundings, within 2^-23 relative of the exact quotient (plus 2^-48).
+E4M3_QUOTIENT_REL = 2.0 ** -22
 
 
 # ------------------------------------------------------------------ GPU side --
@@ -178,6 +181,23 @@ def compare_masks(cfg: Config, gpu_idx, gpu_cnt, orc: Dict[int, dict], k: int):
                 else:
                     bad.append((b, h, i, "idx", g_row[:k_eff].tolist(), oi[b, 0, i].tolist(), rel))
     return rows, exact, ties, bad
+
+
+def e4m3_codes_agree(gpu_codes: np.ndarray, x: np.ndarray, scale: float):
+    """Compare e4m3 values written by the kernels with the oracle's codes of
+    the exact quotient x / scale.  A value may differ only where an e4m3
+    rounding boundary lies within E4M3_QUOTIENT_REL (relative) of the exact
+    quotient, and it must then be one of the two values on either side of
+    that boundary: the kernels' fp32 quotient, within that distance of the
+    exact one, may fall on the other side.  Returns (mismatches accepted by
+    that rule, boolean mask of elements that break it)."""
+    want = oracle.quantize_e4m3(x, scale)
+    a = oracle.quantize_e4m3(x * (1.0 - E4M3_QUOTIENT_REL), scale)
+    b = oracle.quantize_e4m3(x * (1.0 + E4M3_QUOTIENT_REL), scale)
+    lo, hi = np.minimum(a, b), np.maximum(a, b)
+    same = gpu_codes == want
+    near = (~same) & (lo != hi) & (gpu_codes >= lo) & (gpu_codes <= hi)
+    return int(near.sum()), ~(same | near)
 
 
 def compare_attention(cfg: Config, o_gpu, lse_gpu, orc_res):
