@@ -29,6 +29,7 @@ class UfKvCache(ctypes.Structure):
         ("B", ctypes.c_int32), ("G", ctypes.c_int32), ("D", ctypes.c_int32),
         ("W", ctypes.c_int32), ("Lc", ctypes.c_int32), ("blk", ctypes.c_int32),
         ("host_start", ctypes.c_int32), ("host_n_valid", ctypes.c_int32), ("host_anchor", ctypes.c_int32),
+        ("err", ctypes.c_void_p),
     ]
 
 
@@ -49,10 +50,12 @@ def _load() -> ctypes.CDLL:
     pc = ctypes.POINTER(UfKvCache)
     sig = {
         "uf_version": ([], i32),
+        "uf_source_hash": ([], ctypes.c_char_p),
         "uf_strerror": ([i32], ctypes.c_char_p),
         "uf_kv_cache_bytes": ([i32, i32, i32, i32, i32, i32, ctypes.POINTER(sz), ctypes.POINTER(sz),
                                ctypes.POINTER(sz)], i32),
         "uf_kv_cache_init": ([pc, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32], i32),
+        "uf_kv_cache_set_error_word": ([pc, vp], i32),
         "uf_kv_reset": ([pc, vp], i32),
         "uf_kv_append": ([pc, vp, vp, i32, i32, vp], i32),
         "uf_kv_append_rope": ([pc, vp, vp, i32, i32, ctypes.c_int64, ctypes.c_float, vp], i32),
@@ -65,6 +68,7 @@ def _load() -> ctypes.CDLL:
         "uf_kv_append_fp8k": ([pc, vp, ctypes.c_float, vp, vp, i32, i32, vp], i32),
         "uf_block_sparse_attn_fp8k": ([vp, i32, pc, vp, ctypes.c_float, ctypes.c_float, vp, vp, i32, ctypes.c_float,
                                        vp, vp, vp], i32),
+        "uf_check_error": ([vp, vp], i32),
         "uf_get_error": ([ctypes.POINTER(i32), i32], i32),
         "uf_last_cuda_error": ([], ctypes.c_char_p),
         "uf_set_wait_limit": ([ctypes.c_int64], i32),
@@ -78,6 +82,19 @@ def _load() -> ctypes.CDLL:
 
 
 lib = _load()
+
+
+def _check_source_hash() -> None:
+    """Refuse a library built from sources other than the ones beside it."""
+    from .build import source_hash
+    built = lib.uf_source_hash().decode()
+    tree = source_hash()
+    if built != tree:
+        raise ImportError(f"{_LIB_PATH} was built from other sources (library {built}, tree {tree}): "
+                          f"run `python block_sparse_causal_b200/build.py`")
+
+
+_check_source_hash()
 
 
 def strerror(status: int) -> str:
@@ -113,6 +130,10 @@ def uf_kv_cache_init(k, v, kpool, meta, B, G, D, W, Lc, blk) -> UfKvCache:
     _check(lib.uf_kv_cache_init(ctypes.byref(c), _ptr(k), _ptr(v), _ptr(kpool), _ptr(meta), B, G, D, W, Lc, blk),
            "uf_kv_cache_init")
     return c
+
+
+def uf_kv_cache_set_error_word(cache: UfKvCache, err) -> None:
+    _check(lib.uf_kv_cache_set_error_word(ctypes.byref(cache), _ptr(err)), "uf_kv_cache_set_error_word")
 
 
 def uf_kv_reset(cache: UfKvCache, stream=None) -> None:
@@ -176,6 +197,12 @@ def uf_block_sparse_attn_fp8k(q, H: int, cache: UfKvCache, k8, q_scale: float, k
            "uf_block_sparse_attn_fp8k")
 
 
+def uf_check_error(dev_err_word, stream=None) -> None:
+    """Enqueue the move of the library's device error word into ``dev_err_word``
+    (a device int32 tensor) on ``stream``; no synchronisation."""
+    _check(lib.uf_check_error(_ptr(dev_err_word), _stream(stream)), "uf_check_error")
+
+
 def uf_get_error(clear: bool = True) -> int:
     st = ctypes.c_int32()
     _check(lib.uf_get_error(ctypes.byref(st), 1 if clear else 0), "uf_get_error")
@@ -192,3 +219,7 @@ def uf_debug_wait_timeout(cycles: int, stream=None) -> None:
 
 def uf_version() -> int:
     return lib.uf_version()
+
+
+def uf_source_hash() -> str:
+    return lib.uf_source_hash().decode()

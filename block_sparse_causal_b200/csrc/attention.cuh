@@ -88,8 +88,17 @@ struct AttnParams {
   uint32_t nb_mul;           // floor(2^32 / nb) (2^32 - 1 for nb = 1): j / nb without a divide
   float scale_log2;          // softmax scale * log2(e) (FP8 variant: times q_scale * k_scale)
   float q_inv_scale;         // FP8 variant: 1 / q_scale
-  long long wait_limit;
+  long long wait_limit;      // bound of every pipeline wait (cycles)
+  int32_t *err;              // the window's error word, or NULL (the module's)
 };
+
+// Bound of the waits that let copies and MMAs already in flight finish before
+// a thread block that gave up exits: never below 2^31 cycles (about a second),
+// whatever the pipeline bound, since tensor memory must not be released and
+// shared memory must not be abandoned while the hardware still uses them.
+__device__ __forceinline__ long long drain_limit(long long wait_limit) {
+  return wait_limit > (1LL << 31) ? wait_limit : (1LL << 31);
+}
 
 template <int BLK>
 struct AttnSmem {
@@ -215,7 +224,7 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
     mbar_init(&bar_p, ATTN_SOFTMAX_THREADS / 2);
     s_abort = 0;
     fence_mbar_init();
-    if (bad_meta && blockIdx.x == 0) record_error(UF_EBOUNDS);
+    if (bad_meta && blockIdx.x == 0) record_error(p.err, UF_EBOUNDS);
   }
   if (warp == 1) {
     tmem_alloc(&s_tbase, 512);
@@ -248,10 +257,10 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
           if (it.n < 1) continue;
           const int zc = it.b * p.G + it.g;
           for (int t = 0; t < it.n; ++t) {
-            if (!(ok = wait_bounded(&empty_bars[stage], phase ^ 1u, abort_flag, p.wait_limit))) break;
+            if (!(ok = wait_bounded(&empty_bars[stage], phase ^ 1u, abort_flag, p.wait_limit, p.err))) break;
             bool bad;
             const int jb = attn_block(it, t, NKV, bad);
-            if (bad) record_error(UF_EBOUNDS);
+            if (bad) record_error(p.err, UF_EBOUNDS);
             int row, valid;
             kv_block_coords(jb, start, p.W, anchor, p.nb, p.nb_mul, p.lslot, BLK, p.Lc, row, valid);
             uint64_t *full = &full_bars[stage];
@@ -287,7 +296,7 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
               s = nst - 1;
               ph ^= 1u;
             }
-            wait_bounded(&full_bars[s], ph, &never, p.wait_limit);
+            wait_bounded(&full_bars[s], ph, &never, drain_limit(p.wait_limit), p.err);
           }
         }
       }
@@ -319,13 +328,13 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
         while (item < p.items && ok) {
           if (FP8) {
             // the softmax threads have written the item's e4m3 Q into tensor memory
-            if (!(ok = wait_bounded(&bar_q, kq & 1, abort_flag, p.wait_limit))) break;
+            if (!(ok = wait_bounded(&bar_q, kq & 1, abort_flag, p.wait_limit, p.err))) break;
           } else {
             // once the previous item's QK products have read Q's columns and
             // this item's Q has landed: copy it into tensor memory here, one
             // K = 16 slice per copy, and wait for the copies
-            if (kq > 0 && !(ok = wait_bounded(&bar_qtfree, (kq - 1) & 1, abort_flag, p.wait_limit))) break;
-            if (!(ok = wait_bounded(&bar_qfull, kq & 1, abort_flag, p.wait_limit))) break;
+            if (kq > 0 && !(ok = wait_bounded(&bar_qtfree, (kq - 1) & 1, abort_flag, p.wait_limit, p.err))) break;
+            if (!(ok = wait_bounded(&bar_qfull, kq & 1, abort_flag, p.wait_limit, p.err))) break;
             tc_fence_after();
             const uint32_t q_base = smem_u32(sQ);
 #pragma unroll
@@ -333,7 +342,7 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
               tmem_cp_128x256b(tb + TM_Q + kk * 8,
                                sdesc_sw128(q_base + (kk >> 2) * (L::Q_BYTES / 2) + (kk & 3) * 32, 16, 1024));
             mma_commit(&bar_qcp);
-            if (!(ok = wait_bounded(&bar_qcp, kq & 1, abort_flag, p.wait_limit))) break;
+            if (!(ok = wait_bounded(&bar_qcp, kq & 1, abort_flag, p.wait_limit, p.err))) break;
           }
           tc_fence_after();
           int item_next = p.items;
@@ -342,9 +351,9 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
           for (int t = 0; t < it.n; ++t) {
             const int buf = (g0 + t) & 1;
             // the buffer's previous block has been read by the softmax
-            if (uses[buf] > 0 && !(ok = wait_bounded(&bar_sfree[buf], (uses[buf] - 1) & 1, abort_flag, p.wait_limit)))
+            if (uses[buf] > 0 && !(ok = wait_bounded(&bar_sfree[buf], (uses[buf] - 1) & 1, abort_flag, p.wait_limit, p.err)))
               break;
-            if (!(ok = wait_bounded(&bar_kfull[stage], phase, abort_flag, p.wait_limit))) break;
+            if (!(ok = wait_bounded(&bar_kfull[stage], phase, abort_flag, p.wait_limit, p.err))) break;
             tc_fence_after();
             const uint32_t k_addr = k_base + stage * L::STAGE;
             if (FP8) {
@@ -377,7 +386,7 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
                 if (nxt.n >= 1) break;
               }
               if (item_next < p.items) {
-                if (kq > 0 && !(ok = wait_bounded(&bar_ostore, (kq - 1) & 1, abort_flag, p.wait_limit))) break;
+                if (kq > 0 && !(ok = wait_bounded(&bar_ostore, (kq - 1) & 1, abort_flag, p.wait_limit, p.err))) break;
                 request_q(nxt);
               }
             }
@@ -395,8 +404,8 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
         // the previous one was copied out, so at most one)
         mma_commit(&bar_fin[0]);
         int32_t never = 0;
-        wait_bounded(&bar_fin[0], 0, &never, p.wait_limit);
-        if (!ok && q_loads > 0) wait_bounded(&bar_qfull, (q_loads - 1) & 1, &never, p.wait_limit);
+        wait_bounded(&bar_fin[0], 0, &never, drain_limit(p.wait_limit), p.err);
+        if (!ok && q_loads > 0) wait_bounded(&bar_qfull, (q_loads - 1) & 1, &never, drain_limit(p.wait_limit), p.err);
       }
     } else {
       // ------------------------------------------------------------ PV issuer -
@@ -412,9 +421,9 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
         // panel (rows past the q-block or past Lc are not written); the
         // staging tile is released once the stores have read it
         auto store_output = [&](const AttnItem &a, int k) -> bool {
-          if (!wait_bounded(&bar_ofree, k & 1, abort_flag, p.wait_limit)) return false;
-          if (!wait_bounded(&bar_st[0], k & 1, abort_flag, p.wait_limit)) return false;
-          if (!wait_bounded(&bar_st[1], k & 1, abort_flag, p.wait_limit)) return false;
+          if (!wait_bounded(&bar_ofree, k & 1, abort_flag, p.wait_limit, p.err)) return false;
+          if (!wait_bounded(&bar_st[0], k & 1, abort_flag, p.wait_limit, p.err)) return false;
+          if (!wait_bounded(&bar_st[1], k & 1, abort_flag, p.wait_limit, p.err)) return false;
           tma_store_4d(&tmO, sQ, 0, a.h, a.i * BLK, a.b);
           tma_store_4d(&tmO, sQ + L::Q_BYTES / 2, 64, a.h, a.i * BLK, a.b);
           bulk_commit();
@@ -430,8 +439,8 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
           if (kq > 0 && !(ok = store_output(prev, kq - 1))) break;
           for (int t = 0; t < it.n; ++t) {
             const int gb = g0 + t;
-            if (!(ok = wait_bounded(&bar_p, gb & 1, abort_flag, p.wait_limit))) break;
-            if (!(ok = wait_bounded(&bar_vfull[stage], phase, abort_flag, p.wait_limit))) break;
+            if (!(ok = wait_bounded(&bar_p, gb & 1, abort_flag, p.wait_limit, p.err))) break;
+            if (!(ok = wait_bounded(&bar_vfull[stage], phase, abort_flag, p.wait_limit, p.err))) break;
             tc_fence_after();
             const uint32_t v_addr = v_base + stage * L::STAGE;
 #pragma unroll
@@ -453,7 +462,7 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
         if (ok && kq > 0) ok = store_output(prev, kq - 1);
         mma_commit(&bar_fin[1]);
         int32_t never = 0;
-        wait_bounded(&bar_fin[1], 0, &never, p.wait_limit);
+        wait_bounded(&bar_fin[1], 0, &never, drain_limit(p.wait_limit), p.err);
       }
     }
   } else {
@@ -468,7 +477,7 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
     const uint64_t c2 = f2_pack(c_log2, c_log2);
     // tcgen05.ld / st are warp-collective: every wait result is made warp-uniform
     auto wwait = [&](uint64_t *bar, uint32_t parity) {
-      return __all_sync(0xffffffffu, wait_bounded(bar, parity, abort_flag, p.wait_limit));
+      return __all_sync(0xffffffffu, wait_bounded(bar, parity, abort_flag, p.wait_limit, p.err));
     };
     // an item with nothing to compute: zero output, -inf log-sum-exp
     auto write_empty = [&](const AttnItem &a) {
@@ -480,7 +489,7 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
         for (int e = 0; e < 8; ++e) dst[e] = make_uint4(0, 0, 0, 0);
         if (p.lse && x == 0) p.lse[(static_cast<size_t>(a.b) * p.H + a.h) * p.Lc + q_tok] = -INFINITY;
       }
-      if (threadIdx.x == 128) record_error(UF_EBOUNDS);
+      if (threadIdx.x == 128) record_error(p.err, UF_EBOUNDS);
     };
     // first item at or after `from` (in this block's sequence) with blocks to
     // compute; the empty ones on the way are written here

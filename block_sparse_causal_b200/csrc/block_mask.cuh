@@ -55,6 +55,7 @@ struct MaskParams {
   int32_t local;            // radius of the forced band of blocks around the diagonal
   int32_t local_only;       // keep the band only (no scored blocks)
   float scale;
+  int32_t *err;             // the window's error word, or NULL (the module's)
 };
 
 // Order-preserving map float -> uint32 (larger float -> larger key).
@@ -94,7 +95,7 @@ __global__ void __launch_bounds__(MASK_THREADS, 2) block_mask_kernel(const MaskP
   if (tid == 0) {
     int32_t start = __ldcg(p.meta + 0), n = __ldcg(p.meta + 1), anc = __ldcg(p.meta + 3);
     if (!window_state_ok(start, n, anc, p.W)) {
-      record_error(UF_EBOUNDS);
+      record_error(p.err, UF_EBOUNDS);
       n = 0;
       start = 0;
       anc = 0;
@@ -202,7 +203,7 @@ __global__ void __launch_bounds__(MASK_THREADS, 2) block_mask_kernel(const MaskP
   for (int t = pair; t < ntiles; t += MASK_KSTAGE) {
     // both warps of the pair run the same iterations (the named barrier below
     // needs both); after an abort the waits return at once and nothing is issued
-    if (wait_bounded(&bar_k[pair], (t / MASK_KSTAGE) & 1, &s_abort, kWait)) {
+    if (wait_bounded(&bar_k[pair], (t / MASK_KSTAGE) & 1, &s_abort, kWait, p.err)) {
       const float *kt = s_kt + (pair * MASK_KT + mh * 16) * MASK_KSTRIDE;
       float d[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll

@@ -88,6 +88,7 @@ struct AppendParams {
   uint8_t *k8;                 // FP8 variant: [B, G, W*Lslot, D] e4m3 copy of K (same slots)
   float k8_inv_scale;          // FP8 variant: 1 / k_scale
   double log2_base;
+  int32_t *err;                // the window's error word, or NULL (the module's)
 };
 
 // New window state and the slot the chunk goes to (see uf_kv_append).  With
@@ -188,7 +189,7 @@ __global__ void __launch_bounds__(256) kv_append_kernel(const AppendParams p) {
     int32_t start = __ldcg(p.meta + 0), n = __ldcg(p.meta + 1), anc = __ldcg(p.meta + 3);
     const bool empty = n == 0 && anc == 0 && start >= 0 && start < p.W;
     if (!empty && !window_state_ok(start, n, anc, p.W)) {
-      record_error(UF_EBOUNDS);
+      record_error(p.err, UF_EBOUNDS);
       start = 0;
       n = 0;
       anc = 0;

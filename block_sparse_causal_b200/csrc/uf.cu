@@ -19,7 +19,7 @@
 
 namespace {
 
-constexpr int32_t UF_VERSION = 100;   // 0.1.0
+constexpr int32_t UF_VERSION = 200;   // 0.2.0
 constexpr int32_t kMaxW = 64;
 constexpr int32_t kMaxMaskNKV = 1024; // window blocks: 32 selection keys per lane
 constexpr int32_t kMaxDevices = 64;
@@ -211,6 +211,7 @@ int32_t append_impl(uf_kv_cache *c, const void *k_new, const void *v_new, int32_
   p.make_anchor = make_anchor;
   p.pos0 = pos0;
   p.log2_base = log2_base;
+  p.err = c->err;
   const bool tiled = tile_grid != nullptr;
   if (tiled) p.grid = *tile_grid;
   p.k8 = static_cast<uint8_t *>(k8);
@@ -325,6 +326,7 @@ int32_t attn_impl(const void *q, int32_t H, const uf_kv_cache *c, const int32_t 
   p.scale_log2 = scale * q_scale * k_scale * 1.4426950408889634f;
   p.q_inv_scale = 1.0f / q_scale;
   p.wait_limit = g_wait_limit.load();
+  p.err = c->err;
   int sms = 0;
   const int32_t se = sm_count(&sms);
   if (se != UF_OK) return se;
@@ -354,6 +356,11 @@ int32_t attn_impl(const void *q, int32_t H, const uf_kv_cache *c, const int32_t 
 extern "C" {
 
 int32_t uf_version(void) { return UF_VERSION; }
+
+#ifndef UF_SOURCE_HASH
+#define UF_SOURCE_HASH "unknown"
+#endif
+const char *uf_source_hash(void) { return UF_SOURCE_HASH; }
 
 const char *uf_strerror(int32_t status) {
   switch (status) {
@@ -395,8 +402,16 @@ int32_t uf_kv_cache_init(uf_kv_cache *c, void *k, void *v, float *kpool, int32_t
   t.host_start = 0;
   t.host_n_valid = 0;
   t.host_anchor = 0;
+  t.err = nullptr;
   if (!cache_ok(&t)) return UF_EINVAL;
   *c = t;
+  return UF_OK;
+}
+
+int32_t uf_kv_cache_set_error_word(uf_kv_cache *c, int32_t *err) {
+  if (!cache_ok(c)) return UF_EINVAL;
+  if (reinterpret_cast<uintptr_t>(err) & 3u) return UF_EINVAL;
+  c->err = err;
   return UF_OK;
 }
 
@@ -478,6 +493,7 @@ int32_t uf_block_mask_local(const void *q, int32_t H, const uf_kv_cache *c, int3
   p.local = local;
   p.local_only = (flags & UF_MASK_LOCAL_ONLY) ? 1 : 0;
   p.scale = 1.0f / sqrtf(static_cast<float>(c->D));
+  p.err = c->err;
   const int smem = uf::mask_smem_bytes(nkv_max);
   const dim3 grid(ceil_div(nb, uf::MASK_TQ), H, c->B);
   const cudaStream_t st = reinterpret_cast<cudaStream_t>(s);
@@ -507,6 +523,13 @@ int32_t uf_kv_append_fp8k(uf_kv_cache *c, void *k8, float k_scale, const void *k
   return append_impl(c, k_new, v_new, keep_chunks, flags, 0, 0, 0.0, s, nullptr, k8, k_scale);
 }
 
+
+int32_t uf_check_error(int32_t *dev_err_word, uf_stream_t s) {
+  if (!dev_err_word || (reinterpret_cast<uintptr_t>(dev_err_word) & 3u)) return UF_EINVAL;
+  cudaGetLastError();
+  uf::check_error_kernel<<<1, 1, 0, reinterpret_cast<cudaStream_t>(s)>>>(dev_err_word);
+  return launch_status();
+}
 
 int32_t uf_get_error(int32_t *status, int32_t clear) {
   if (!status) return UF_EINVAL;

@@ -15,11 +15,20 @@
 namespace uf {
 
 // ------------------------------------------------------------ error word ----
-// First error recorded by any kernel of this module on this device.
+// First error recorded by a kernel of this module on this device, for calls
+// whose window has no error word of its own.
 __device__ int32_t g_error_word;
 
-__device__ __forceinline__ void record_error(int32_t code) {
-  atomicCAS(&g_error_word, 0, code);
+// Record `code` in `word` (the window's own error word) or, when that is NULL,
+// in the module's word; the first error recorded stays.
+__device__ __forceinline__ void record_error(int32_t *word, int32_t code) {
+  atomicCAS(word ? word : &g_error_word, 0, code);
+}
+
+// Move the module's word into a caller's word (kept when already non-zero).
+__global__ void check_error_kernel(int32_t *dst) {
+  const int32_t e = atomicExch(&g_error_word, 0);
+  if (e != 0 && *dst == 0) *dst = e;
 }
 
 // ------------------------------------------------------------ addresses -----
@@ -63,10 +72,11 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
 }
 
 // Wait until the phase with parity `parity` of `bar` has completed.  Returns
-// false (after recording UF_ETIMEOUT once and raising *abort) when the bound
-// is reached, or when another thread of the block has already raised *abort.
+// false (after recording UF_ETIMEOUT in `err` -- see record_error -- and
+// raising *abort) when the bound is reached, or when another thread of the
+// block has already raised *abort.
 __device__ __forceinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, volatile int32_t *abort,
-                                             long long limit) {
+                                             long long limit, int32_t *err = nullptr) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (true) {
@@ -74,7 +84,7 @@ __device__ __forceinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, vol
     if (*abort) return false;
     if (clock64() - t0 > limit) {
       *abort = 1;
-      record_error(UF_ETIMEOUT);
+      record_error(err, UF_ETIMEOUT);
       return false;
     }
   }

@@ -12,10 +12,12 @@ class KVWindow:
     """Allocates k, v, kpool and meta for a window of W chunks on ``device``
     (sizes from ``uf_kv_cache_bytes``) and holds the ``uf_kv_cache``
     descriptor that the library calls take.  With ``k_scale`` it also owns the
-    e4m3 copy of K (``k8``) that the FP8-score calls read and write."""
+    e4m3 copy of K (``k8``) that the FP8-score calls read and write.  With
+    ``error_word`` it owns a device int32 ``err`` in which the kernels of calls
+    on this window record their errors (``uf_kv_cache_set_error_word``)."""
 
     def __init__(self, B: int, G: int, W: int, Lc: int, blk: int = 128, D: int = 128, device="cuda",
-                 k_scale: float | None = None):
+                 k_scale: float | None = None, error_word: bool = False):
         kv_bytes, kpool_bytes, meta_bytes = _uf.uf_kv_cache_bytes(B, G, D, W, Lc, blk)
         self.B, self.G, self.D, self.W, self.Lc, self.blk = B, G, D, W, Lc, blk
         self.nb = math.ceil(Lc / blk)
@@ -28,6 +30,10 @@ class KVWindow:
         self.desc = _uf.uf_kv_cache_init(self.k, self.v, self.kpool, self.meta, B, G, D, W, Lc, blk)
         self.k_scale = k_scale
         self.k8 = None if k_scale is None else torch.zeros(B, G, W * self.lslot, D, dtype=torch.uint8, device=device)
+        self.err = None
+        if error_word:
+            self.err = torch.zeros(1, dtype=torch.int32, device=device)
+            _uf.uf_kv_cache_set_error_word(self.desc, self.err)
 
     @property
     def n_valid(self) -> int:

@@ -23,8 +23,12 @@
  *   - Every call returns a status (uf_status).  Argument errors are detected on
  *     the host before anything is enqueued (UF_EINVAL, nothing launched).  A
  *     launch failure returns UF_ECUDA.  Errors found by a kernel while running
- *     (an out-of-range block index, a pipeline wait that exceeded its bound)
- *     are recorded in a device-side error word, read with uf_get_error().
+ *     (an out-of-range block index, a bad window state, a pipeline wait that
+ *     exceeded its bound) are recorded in a device-side error word: the
+ *     window's own word when the caller gave it one (uf_kv_cache.err), else
+ *     the library's word of the current device, which uf_check_error() moves
+ *     into a caller's word in stream order and uf_get_error() reads after a
+ *     device synchronisation.  In either word the first error stays.
  *   - bf16 = IEEE bfloat16 (2 bytes), fp32 = IEEE binary32, int32 = int32_t.
  *   - Shapes are listed outermost first; the last dimension is contiguous.
  *
@@ -88,6 +92,12 @@ typedef enum uf_status {
  *   host_start, host_n_valid, host_anchor: host mirror of meta[0], meta[1],
  *          meta[3], updated by uf_kv_append / uf_kv_reset and used only for
  *          host-side argument checks.
+ *   err    optional device int32: errors that kernels of calls on this window
+ *          find (UF_EBOUNDS, UF_ETIMEOUT) are recorded here instead of in the
+ *          library's device-wide word, so that concurrent windows do not share
+ *          one flag.  The first error stays (a non-zero word is never
+ *          overwritten); the caller reads and clears it in stream order.  NULL
+ *          (set by uf_kv_cache_init) = the library's word.
  *
  * Sources: FlashDecoder (xllm-io blog), Sec. 3, Eq. 4 (cache shape
  * B x G x (W_frm L_frm) x D_h under grouped-query attention) and Algorithm 1
@@ -102,10 +112,19 @@ typedef struct uf_kv_cache {
   int32_t *meta;
   int32_t B, G, D, W, Lc, blk;
   int32_t host_start, host_n_valid, host_anchor;
+  int32_t *err;
 } uf_kv_cache;
 
 /* Library version: major * 10000 + minor * 100 + patch. */
 int32_t uf_version(void);
+
+/*
+ * Build identity, not a step of the method: the first 16 hex digits of the
+ * SHA-256 over the library's sources (static string, never NULL; "unknown"
+ * when built without it).  The Python binding compares it with the sources it
+ * ships beside and refuses a library built from others.
+ */
+const char *uf_source_hash(void);
 
 /* Human-readable name of a status code (static string, never NULL). */
 const char *uf_strerror(int32_t status);
@@ -127,6 +146,12 @@ int32_t uf_kv_cache_bytes(int32_t B, int32_t G, int32_t D, int32_t W, int32_t Lc
  */
 int32_t uf_kv_cache_init(uf_kv_cache *c, void *k, void *v, float *kpool, int32_t *meta,
                          int32_t B, int32_t G, int32_t D, int32_t W, int32_t Lc, int32_t blk);
+
+/*
+ * Give the window its own device error word (err: device int32, 4-byte
+ * aligned, caller-owned; NULL = back to the library's word).  Host only.
+ */
+int32_t uf_kv_cache_set_error_word(uf_kv_cache *c, int32_t *err);
 
 /* Empty the window: zero meta on stream s and reset the host mirror. */
 int32_t uf_kv_reset(uf_kv_cache *c, uf_stream_t s);
@@ -345,6 +370,20 @@ int32_t uf_block_sparse_attn_fp8k(const void *q, int32_t H, const uf_kv_cache *c
                                   float q_scale, float k_scale, const int32_t *idx,
                                   const int32_t *cnt, int32_t k, float scale, void *o, float *lse,
                                   uf_stream_t s);
+
+/*
+ * Stream-ordered error read (failure detection without a device
+ * synchronisation): enqueue on s one single-thread kernel that takes the
+ * library's device-wide error word of the current device (the first error a
+ * kernel of a window without its own word recorded since the last clear),
+ * clears it, and stores it into *dev_err_word unless that already holds a
+ * non-zero code (so one word collects the first error over many calls or
+ * graph replays; the caller zeroes it).  dev_err_word: device int32, 4-byte
+ * aligned, caller-owned.  Never synchronises; can be captured in a CUDA
+ * graph.  UF_EINVAL on a NULL or misaligned pointer, UF_ECUDA on a launch
+ * failure.
+ */
+int32_t uf_check_error(int32_t *dev_err_word, uf_stream_t s);
 
 /*
  * Read the device-side error word of the current device (the first error a

@@ -215,3 +215,46 @@ def test_binding_fails_loudly_without_library(tmp_path):
     code = "import block_sparse_causal_b200"
     res = subprocess.run([sys.executable, "-c", code], cwd=tmp_path, capture_output=True, text=True)
     assert res.returncode != 0 and "not built" in res.stderr
+
+
+def test_library_is_built_from_this_tree(uf):
+    # the source hash compiled into libuf.so is the hash of csrc/ and include/
+    from conftest import load_builder
+    assert uf.uf_source_hash() == load_builder().source_hash()
+
+
+def test_stale_library_is_refused(uf, monkeypatch):
+    # a library whose compiled-in hash differs from the tree's sources is refused
+    from block_sparse_causal_b200 import _uf, build
+    monkeypatch.setattr(build, "source_hash", lambda: "0" * 16)
+    with pytest.raises(ImportError, match="other sources"):
+        _uf._check_source_hash()
+
+
+def test_build_rejects_an_attention_register_count_it_cannot_split():
+    from conftest import load_builder
+    b = load_builder()
+    ok = ("ptxas info    : Compiling entry function '_ZN2uf11attn_kernelILi128ELb0EEEv' for 'sm_100a'\n"
+          "ptxas info    : Used 168 registers, used 1 barriers\n")
+    b.check_attention_registers(ok)
+    with pytest.raises(RuntimeError, match="160 registers"):
+        b.check_attention_registers(ok.replace("Used 168", "Used 160"))
+    with pytest.raises(RuntimeError):
+        b.check_attention_registers("ptxas info    : Used 64 registers\n")
+
+
+def test_error_word_calls_validate_on_host(uf):
+    # misaligned or NULL error words are refused before anything is enqueued
+    with pytest.raises(uf.UfError):
+        uf.uf_check_error(FakeTensor(0), stream=0)
+    with pytest.raises(uf.UfError):
+        uf.uf_check_error(FakeTensor(0xB00002), stream=0)
+    c = uf.uf_kv_cache_init(FakeTensor(0xA00000), FakeTensor(0xA10000), FakeTensor(0xA20000),
+                            FakeTensor(0xA30000), 1, 2, 128, 2, 256, 64)
+    assert c.err is None
+    with pytest.raises(uf.UfError):
+        uf.uf_kv_cache_set_error_word(c, FakeTensor(0xB00002))
+    uf.uf_kv_cache_set_error_word(c, FakeTensor(0xB00004))
+    assert c.err == 0xB00004
+    uf.uf_kv_cache_set_error_word(c, None)
+    assert c.err is None
