@@ -8,7 +8,11 @@ the window already full (steady state).  Inputs are resident in HBM before
 the timed region; every step's working set (Q, new K/V, the window, O) is
 larger than the 126 MB L2, so no flush is needed between steps.
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--config 1k_sr] [--impl ours|reference]
+The headline workload is the 2K SR-DiT chunk (the largest); the 1K chunk, the
+dense 480P chunk and the GQA decoder step are timed after it with fewer steps
+and reported under "other_workloads" of the same line (--others '' skips them).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--config 2k_sr] [--others LIST] [--impl ours|reference]
 
 Under torchrun (N > 1) every rank runs an independent replica on its own GPU
 (weak scaling; the path needs no data exchange).  Rank 0 prints one JSON line.
@@ -40,7 +44,8 @@ from workloads import CONFIGS, chunk_inputs  # noqa: E402
 METRIC = "block-sparse chunk attn ms/chunk & kept-block TFLOP/s (% bf16 peak), 1 B200"
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-ATTN_PROFILE = os.path.join(ROOT, "profiles", "attn_1k_sr_traffic.txt")
+DEFAULT_OTHERS = "1k_sr,480p_dense,gqa_decoder"
+PROFILES_DIR = os.path.join(ROOT, "profiles")
 ATTN_SOURCES = ["block_sparse_causal_b200/csrc/attention.cuh", "block_sparse_causal_b200/csrc/uf_device.cuh"]
 
 
@@ -63,11 +68,13 @@ def kernel_source_hash() -> str:
 
 
 def attn_traffic_per_launch(config_name: str):
-    """DRAM bytes per attention launch from the committed ncu summary, or None
-    when there is none for this workload or the kernel changed since."""
-    if config_name != "1k_sr" or not os.path.exists(ATTN_PROFILE):
+    """DRAM bytes per attention launch from the committed ncu summary of this
+    workload (profiles/attn_<workload>_traffic.txt), or None when there is none
+    or the kernel changed since."""
+    path = os.path.join(PROFILES_DIR, f"attn_{config_name}_traffic.txt")
+    if not os.path.exists(path):
         return None
-    txt = open(ATTN_PROFILE).read()
+    txt = open(path).read()
     m_hash = re.search(r"^source_hash:\s*(\S+)", txt, flags=re.M)
     m_bytes = re.search(r"^traffic_bytes_per_launch:\s*([0-9.eE+]+)", txt, flags=re.M)
     if not m_hash or not m_bytes or m_hash.group(1) != kernel_source_hash():
@@ -197,7 +204,7 @@ def mask_k(args, cfg):
     return max(k, 2 * args.mask_local + 1) if not cfg.dense else k
 
 
-def run_ours(args, cfg, rank, world, device):
+def run_ours(args, cfg, rank, world, device, do_e2e=True):
     import block_sparse_causal_b200 as uf
     stream = torch.cuda.current_stream()
     k = mask_k(args, cfg)
@@ -306,46 +313,9 @@ def run_ours(args, cfg, rank, world, device):
     flops_per_step = sum(flops) / len(flops)
     max_ms = all_max(elapsed_ms, world, device)
 
-    # e2e: the same steps through the C ABI from pinned host buffers, with each
-    # chunk's inputs copied in and its O / LSE copied out inside the timed
-    # region; ChunkPipeline overlaps chunk n's copy in and chunk n - 2's copy
-    # out with chunk n - 1's compute (three streams, two staging slots)
-    from block_sparse_causal_b200.pipeline import ChunkPipeline
-    pinned = [{n: x.pin_memory() for n, x in c.items()} for c in host_chunks[cfg.W:]]
-    host_out = [{"o": torch.empty(o.shape, dtype=o.dtype).pin_memory(),
-                 "lse": torch.empty(lse.shape, dtype=lse.dtype).pin_memory()} for _ in range(2)]
-    e2e_steps = max(3, min(args.steps, 50))
-    e2e_count = [0]
-
-    def pipe_step(din, dout, st):
-        step(e2e_count[0] % n_idx, din, o_out=dout["o"], lse_out=dout["lse"])
-        e2e_count[0] += 1
-
-    pipe = ChunkPipeline({n: (tuple(x.shape), x.dtype) for n, x in dev_chunks[0].items()},
-                         {"o": (tuple(o.shape), o.dtype), "lse": (tuple(lse.shape), lse.dtype)},
-                         pipe_step, depth=2, device=device)
-    pipe.submit(pinned[0], host_out[0])
-    pipe.synchronize()
-    sampler2 = ClockSampler(device)
-    sampler2.start()
-    barrier(world)
-    torch.cuda.synchronize()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(pipe.h2d)
-    for s in range(e2e_steps):
-        pipe.submit(pinned[(s + 1) % n_distinct], host_out[(s + 1) % 2])
-    e1.record(pipe.d2h)          # after the last copy out, which follows every earlier step
-    pipe.synchronize()
-    torch.cuda.synchronize()
-    barrier(world)
-    sampler2.stop()
-    if uf.uf_get_error() != 0:
-        raise RuntimeError("device-side error during the end-to-end steps")
-    e2e_ms = all_max(e0.elapsed_time(e1), world, device) / e2e_steps
-    h2d = sum(x.numel() * x.element_size() for x in pinned[0].values())
-    d2h = o.numel() * o.element_size() + lse.numel() * lse.element_size()
-
+    e2e = None
+    if do_e2e:
+        e2e = run_e2e(args, cfg, world, device, host_chunks, dev_chunks, step, o, lse, n_idx, n_distinct)
     ms_per_step = max_ms / args.steps
     # every rank ran its own seeded stream: the job's work is the sum of their kept FLOPs
     job_flops_per_step = all_sum(flops_per_step, world, device)
@@ -412,14 +382,87 @@ def run_ours(args, cfg, rank, world, device):
             "kernel": "uf::attn_kernel<%d, %s>" % (cfg.blk, "true" if args.fp8 else "false"),
             "peak_source": f"{peaks_src} bf16 dense burst (cuBLAS 8192^3)"
                            + (" x 4/3: QK at the nominal e4m3/bf16 ratio of 2" if args.fp8 else ""),
+            # the rate at the maximum SM clock: achieved x (max SM MHz / median SM MHz
+            # under load); separates kernel quality from the power cap's clock
+            "clock_normalised_tflops": (attn_tflops * clocks["sm_max_mhz"] / clocks["sm_mhz"]
+                                        if clocks and clocks.get("sm_mhz") and clocks.get("sm_max_mhz") else None),
         },
-        "e2e": {"value": job_flops_per_step / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
-                "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "overlap": "ChunkPipeline: copy in / compute / copy out on three streams, two slots"},
+        "e2e": None if e2e is None else {
+            "value": job_flops_per_step / (e2e[0] * 1e-3) / 1e12, "unit": "TFLOP/s",
+            "ms_per_step": e2e[0], "h2d_bytes_per_step": e2e[1], "d2h_bytes_per_step": e2e[2],
+            "overlap": "ChunkPipeline: copy in / compute / copy out on three streams, two slots"},
         "clocks": clocks,
         "gpu_launches": launches_per_step * args.steps,
     }
     return result
+
+
+def run_e2e(args, cfg, world, device, host_chunks, dev_chunks, step, o, lse, n_idx, n_distinct):
+    """End-to-end rate through the C ABI from pinned host buffers."""
+    import block_sparse_causal_b200 as uf
+    # e2e: the same steps through the C ABI from pinned host buffers, with each
+    # chunk's inputs copied in and its O / LSE copied out inside the timed
+    # region; ChunkPipeline overlaps chunk n's copy in and chunk n - 2's copy
+    # out with chunk n - 1's compute (three streams, two staging slots)
+    from block_sparse_causal_b200.pipeline import ChunkPipeline
+    pinned = [{n: x.pin_memory() for n, x in c.items()} for c in host_chunks[cfg.W:]]
+    host_out = [{"o": torch.empty(o.shape, dtype=o.dtype).pin_memory(),
+                 "lse": torch.empty(lse.shape, dtype=lse.dtype).pin_memory()} for _ in range(2)]
+    e2e_steps = max(3, min(args.steps, 50))
+    e2e_count = [0]
+
+    def pipe_step(din, dout, st):
+        step(e2e_count[0] % n_idx, din, o_out=dout["o"], lse_out=dout["lse"])
+        e2e_count[0] += 1
+
+    pipe = ChunkPipeline({n: (tuple(x.shape), x.dtype) for n, x in dev_chunks[0].items()},
+                         {"o": (tuple(o.shape), o.dtype), "lse": (tuple(lse.shape), lse.dtype)},
+                         pipe_step, depth=2, device=device)
+    pipe.submit(pinned[0], host_out[0])
+    pipe.synchronize()
+    sampler2 = ClockSampler(device)
+    sampler2.start()
+    barrier(world)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(pipe.h2d)
+    for s in range(e2e_steps):
+        pipe.submit(pinned[(s + 1) % n_distinct], host_out[(s + 1) % 2])
+    e1.record(pipe.d2h)          # after the last copy out, which follows every earlier step
+    pipe.synchronize()
+    torch.cuda.synchronize()
+    barrier(world)
+    sampler2.stop()
+    if uf.uf_get_error() != 0:
+        raise RuntimeError("device-side error during the end-to-end steps")
+    e2e_ms = all_max(e0.elapsed_time(e1), world, device) / e2e_steps
+    h2d = sum(x.numel() * x.element_size() for x in pinned[0].values())
+    d2h = o.numel() * o.element_size() + lse.numel() * lse.element_size()
+
+    return e2e_ms, h2d, d2h
+
+
+def run_others(args, rank, world, device):
+    """The other workloads with the same options, fewer steps and no e2e leg:
+    per workload its step time, kept-block rate and per-kernel figures."""
+    names = [n for n in args.others.split(",") if n and n != args.config]
+    out = {}
+    for name in names:
+        sub = argparse.Namespace(**vars(args))
+        sub.config = name
+        sub.steps = max(3, min(args.steps, 50))
+        sub.warmup = max(3, min(args.warmup, 5))
+        torch.cuda.empty_cache()
+        r = run_ours(sub, CONFIGS[name], rank, world, device, do_e2e=False)
+        out[name] = {"ms_per_step": r["ms_per_step"], "value": r["value"], "unit": r["unit"], "steps": sub.steps,
+                     "kernels": r["kernels"],
+                     "attn_frac": r["roofline"]["frac"],
+                     "attn_clock_normalised_tflops": r["roofline"]["clock_normalised_tflops"],
+                     "attn_traffic": r["roofline"]["traffic"],
+                     "k": r["config"]["k"], "kept_flops_per_step": r["config"]["kept_flops_per_step"],
+                     "clocks": r["clocks"], "gpu_launches": r["gpu_launches"]}
+    return out
 
 
 # --------------------------------------------------------- CPU oracle arm ---
@@ -549,7 +592,9 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--config", default="1k_sr", choices=sorted(CONFIGS))
+    ap.add_argument("--config", default="2k_sr", choices=sorted(CONFIGS))
+    ap.add_argument("--others", default=DEFAULT_OTHERS,
+                    help="comma-separated workloads timed after the headline one (fewer steps, no e2e leg)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing leg")
@@ -589,6 +634,7 @@ def main():
     torch.cuda.set_device(device)
     try:
         result = run_ours(args, cfg, rank, world, device)
+        result["other_workloads"] = run_others(args, rank, world, device)
         if rank == 0:
             if world == 1 and not args.no_cpu_baseline:
                 result["cpu_baseline"] = cpu_baseline(cfg, args.seed, args.mask_local, args.mask_local_only,

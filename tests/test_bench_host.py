@@ -45,9 +45,9 @@ def test_byte_accounting_1k():
 
 
 def test_traffic_is_dropped_when_the_kernel_changes(tmp_path, monkeypatch):
-    prof = tmp_path / "t.txt"
+    prof = tmp_path / "attn_1k_sr_traffic.txt"
     prof.write_text(f"source_hash: {bench.kernel_source_hash()}\ntraffic_bytes_per_launch: 123\n")
-    monkeypatch.setattr(bench, "ATTN_PROFILE", str(prof))
+    monkeypatch.setattr(bench, "PROFILES_DIR", str(tmp_path))
     assert bench.attn_traffic_per_launch("1k_sr") == 123.0
     assert bench.attn_traffic_per_launch("2k_sr") is None
     prof.write_text("source_hash: 0000\ntraffic_bytes_per_launch: 123\n")

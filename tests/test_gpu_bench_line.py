@@ -16,7 +16,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 def test_bench_prints_the_contract_line():
     out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--config", "tiny", "--steps", "3",
-                          "--warmup", "3", "--no-cpu-baseline"], capture_output=True, text=True, cwd=ROOT,
+                          "--warmup", "3", "--no-cpu-baseline", "--others", "gqa_decoder"], capture_output=True, text=True, cwd=ROOT,
                          timeout=600)
     assert out.returncode == 0, out.stderr[-2000:]
     lines = [l for l in out.stdout.splitlines() if l.startswith("{")]
@@ -39,3 +39,6 @@ def test_bench_prints_the_contract_line():
     assert e["h2d_bytes_per_step"] > 0 and e["d2h_bytes_per_step"] > 0 and e["value"] > 0
     for key in ("sm_mhz", "sm_max_mhz", "reasons"):
         assert key in d["clocks"], key
+    assert "clock_normalised_tflops" in r
+    other = d["other_workloads"]["gqa_decoder"]
+    assert other["ms_per_step"] > 0 and other["value"] > 0 and 0 < other["attn_frac"] < 1.5
