@@ -113,8 +113,9 @@ def append_bytes(cfg, fp8=False):
 
 
 def fp8_scales(chunk):
-    """Static per-tensor scales calibrated once on one chunk: amax / 448 (e4m3)."""
-    return (float(chunk["q"].float().abs().max()) / 448.0, float(chunk["k"].float().abs().max()) / 448.0)
+    """Static per-tensor scales calibrated once on one chunk: amax / 448 (e4m3),
+    rounded up to a power of two (the quotient x / scale is then exact)."""
+    return tuple(2.0 ** math.ceil(math.log2(float(chunk[n].float().abs().max()) / 448.0)) for n in ("q", "k"))
 
 
 def rope_q_bytes(cfg):
@@ -356,7 +357,7 @@ def run_ours(args, cfg, rank, world, device, do_e2e=True):
             "density": cfg.density, "kept_flops_per_step": flops_per_step,
             "mask_local": args.mask_local, "mask_local_only": bool(args.mask_local_only), "rope": bool(args.rope),
             "anchor": bool(args.anchor), "tiled": list(cfg.grid) if args.tiled else None,
-            "fp8": {"q_scale": q_scale, "k_scale": k_scale, "calibration": "amax / 448 of the first chunk"}
+            "fp8": {"q_scale": q_scale, "k_scale": k_scale, "calibration": "amax / 448 of the first chunk, rounded up to a power of two"}
             if args.fp8 else None,
             "step": ("uf_kv_append_rope + uf_rope + " if args.rope else
                      "uf_kv_append_tiled + uf_tile_tokens + " if args.tiled else

@@ -4,18 +4,24 @@ for bit, and the attention whose scores are e4m3 q . e4m3 k on the tensor
 cores, against the fp64 oracle's fp8_scores_attention on the same codes.
 
 The oracle rounds the exact quotient x / scale; the kernels form it in fp32
-as x * fp32(1 / scale), within 2^-23 relative of the exact one.  The codes are
-compared with a near-boundary rule (uf_testlib.e4m3_codes_agree): equal,
-except where an e4m3 rounding boundary lies within that distance of the exact
-quotient.  Such flips are rare and move a score by one e4m3 step of one
-element, so the attention is held to the bf16 path's tolerances unchanged."""
+as x * fp32(1 / scale), within 2^-23 relative of the exact one.  With an
+arbitrary scale the codes are compared with a near-boundary rule
+(uf_testlib.e4m3_codes_agree): equal, except where an e4m3 rounding boundary
+lies within that distance of the exact quotient.  One such flip moves a score
+by one e4m3 step of one element, up to 1/8 of a large code, which can move an
+LSE by 1e-2; so the attention is compared at the bf16 path's tolerances
+unchanged on (a) power-of-two scales, where the quotient is exact in fp32 and
+both sides hold the same codes, and (b) arbitrary scales, on every row that no
+near-boundary element of q or of its kept keys touches."""
+import math
+
 import numpy as np
 import pytest
 import torch
 
 import oracle
-from uf_testlib import (GpuStream, OracleStream, assert_attention_ok, e4m3_codes_agree, oracle_idx_array,
-                        sample_items)
+from uf_testlib import (E4M3_QUOTIENT_REL, LSE_ABS, O_MAX_ABS, O_MEAN_ABS, GpuStream, OracleStream,
+                        assert_attention_ok, e4m3_codes_agree, oracle_idx_array, sample_items)
 from workloads import CONFIGS, chunk_inputs, scaled
 
 pytestmark = [pytest.mark.gpu,
@@ -39,16 +45,23 @@ def _lib(built_lib):
     assert uf.uf_get_error(clear=True) == 0, "a kernel recorded a device-side error"
 
 
-def static_scales(cfg, seed):
-    """Per-tensor scales calibrated once on chunk 0 of the stream: amax / 448."""
+def static_scales(cfg, seed, pow2=True):
+    """Per-tensor scales calibrated once on chunk 0 of the stream: amax / 448,
+    rounded up to a power of two unless pow2 is False.  With a power-of-two
+    scale the quotient x / scale is exact in fp32, so the codes do not depend
+    on how it is formed."""
     inp = chunk_inputs(cfg, seed, 0)
     qs = float(inp["q"].float().abs().max()) / oracle.E4M3_MAX
     ks = float(inp["k"].float().abs().max()) / oracle.E4M3_MAX
+    if pow2:
+        qs, ks = 2.0 ** math.ceil(math.log2(qs)), 2.0 ** math.ceil(math.log2(ks))
+    else:   # the values the library receives (fp32)
+        qs, ks = float(np.float32(qs)), float(np.float32(ks))
     return qs, ks
 
 
-def _stream(cfg, n, seed, anchor=False):
-    qs, ks = static_scales(cfg, seed)
+def _stream(cfg, n, seed, anchor=False, pow2=True):
+    qs, ks = static_scales(cfg, seed, pow2)
     gpu, orc = GpuStream(cfg, k_scale=ks), OracleStream(cfg)
     last = None
     for t in range(n):
@@ -68,8 +81,9 @@ def _slot(win, c):
 
 @pytest.mark.parametrize("name,anchor", [("blk64", False), ("gqa_w3", False), ("sr_w3", True)])
 def test_fp8_k_codes_bit_exact(name, anchor):
+    # arbitrary (not power-of-two) scales: codes equal up to the near-boundary rule
     cfg = CASES[name]
-    gpu, orc, _, _, ks = _stream(cfg, cfg.W + 2, seed=21, anchor=anchor)
+    gpu, orc, _, _, ks = _stream(cfg, cfg.W + 2, seed=21, anchor=anchor, pow2=False)
     k8 = gpu.win.k8.view(torch.float8_e4m3fn).to(torch.float64).cpu().numpy()
     raw = gpu.win.k8.cpu().numpy()
     for g in range(cfg.G):
@@ -119,6 +133,56 @@ def test_fp8_attention_parity(name):
                                oidx.shape[-1])
     torch.cuda.synchronize()
     assert_attention_ok(cfg, o, lse, orc.attention_fp8(last["q"], items, qs, ks, oidx, ocnt), name)
+
+
+def _near_boundary(x, scale):
+    """Elements of x whose exact quotient x / scale lies within the kernels'
+    fp32 quotient error of an e4m3 rounding boundary."""
+    rel = E4M3_QUOTIENT_REL
+    return oracle.quantize_e4m3(x * (1 - rel), scale) != oracle.quantize_e4m3(x * (1 + rel), scale)
+
+
+@pytest.mark.parametrize("name", ["blk64", "sr_w3"])
+def test_fp8_attention_arbitrary_scales_untouched_rows(name):
+    # scales amax / 448 as they are: every row whose q and whose kept keys hold
+    # no near-boundary element must meet the bf16 tolerances; the rows that do
+    # are few
+    cfg = CASES[name]
+    gpu, orc, last, qs, ks = _stream(cfg, cfg.W + 1, seed=26, pow2=False)
+    k = cfg.k_for()
+    oidx, ocnt = oracle_idx_array(cfg, orc.mask(last["q"], k))
+    o, lse = gpu.attention_fp8(last["q"], qs, torch.from_numpy(oidx).cuda(), torch.from_numpy(ocnt).cuda(),
+                               oidx.shape[-1])
+    items = [(b, h, i) for b in range(cfg.B) for h in range(cfg.H) for i in range(cfg.nb)]
+    ref = orc.attention_fp8(last["q"], items, qs, ks, oidx, ocnt)
+    torch.cuda.synchronize()
+    og, lg = o.float().cpu().numpy(), lse.cpu().numpy()
+    qnear = _near_boundary(last["q"].double().numpy(), qs).any(axis=-1)            # [B, Lc, H]
+    kv_near = []                                                                    # per head group: [B, NKV*blk]
+    for g in range(cfg.G):
+        w = orc.windows[g]
+        toks = np.concatenate([_near_boundary(kc[:, :, 0, :], ks).any(axis=-1) for kc in w.k], axis=1)
+        kv_near.append(toks)
+    max_o = max_l = sum_o = 0.0
+    n_o = touched = rows = 0
+    for (b, h, i), (O, L) in ref.items():
+        g = h // (cfg.H // cfg.G)
+        s0, e0 = i * cfg.blk, min(cfg.Lc, (i + 1) * cfg.blk)
+        kept_touched = False
+        for j in oidx[b, h, i, :ocnt[b, h, i]]:
+            c, r = divmod(int(j), cfg.nb)
+            t0 = c * cfg.Lc + r * cfg.blk
+            kept_touched |= bool(kv_near[g][b, t0:min(t0 + cfg.blk, (c + 1) * cfg.Lc)].any())
+        for rr in range(e0 - s0):
+            rows += 1
+            if kept_touched or qnear[b, s0 + rr, h]:
+                touched += 1
+                continue
+            d = np.abs(og[b, s0 + rr, h] - O[rr])
+            max_o, sum_o, n_o = max(max_o, float(d.max())), sum_o + float(d.sum()), n_o + d.size
+            max_l = max(max_l, abs(float(lg[b, h, s0 + rr]) - float(L[rr])))
+    assert touched <= rows // 4, (touched, rows)
+    assert max_o <= O_MAX_ABS and sum_o / n_o <= O_MEAN_ABS and max_l <= LSE_ABS, (max_o, sum_o / n_o, max_l)
 
 
 def test_fp8_anchored_window_and_saturation():
