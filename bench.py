@@ -232,10 +232,15 @@ def run_ours(args, cfg, rank, world, device, do_e2e=True):
     q_rot = torch.empty_like(dev_chunks[0]["q"]) if (args.rope or args.tiled) else None
     o_tiled = torch.empty_like(o) if args.tiled else None
 
+    balanced = args.schedule == "balanced" and not args.fp8
+    ws = torch.empty(uf.uf_attn_workspace_bytes(), dtype=torch.uint8, device=device) if balanced else None
+
     def attention(q, idx_s, cnt_s, k_s, out, lse_out):
         if args.fp8:
             uf.uf_block_sparse_attn_fp8k(q, cfg.H, win.desc, win.k8, q_scale, k_scale, idx_s, cnt_s, k_s, scale,
                                          out, lse_out)
+        elif balanced:
+            uf.uf_block_sparse_attn_balanced(q, cfg.H, win.desc, idx_s, cnt_s, k_s, scale, out, lse_out, ws)
         else:
             uf.uf_block_sparse_attn(q, cfg.H, win.desc, idx_s, cnt_s, k_s, scale, out, lse_out)
 
@@ -363,12 +368,14 @@ def run_ours(args, cfg, rank, world, device, do_e2e=True):
                      "uf_kv_append_tiled + uf_tile_tokens + " if args.tiled else
                      "uf_kv_append_fp8k + " if args.fp8 else "uf_kv_append + ")
                     + ("" if cfg.dense else mask_call_name(args))
-                    + ("uf_block_sparse_attn_fp8k" if args.fp8 else "uf_block_sparse_attn")
+                    + ("uf_block_sparse_attn_fp8k" if args.fp8 else
+                       "uf_block_sparse_attn_balanced" if balanced else "uf_block_sparse_attn")
                     + (" + uf_tile_tokens (O)" if args.tiled else ""),
             "l2": "no flush: every step's working set (%.0f MB) exceeds the 126 MB L2" % (
                 (cfg.B * cfg.Lc * (cfg.H * 2 + cfg.G * 2) * cfg.D * 2
                  + 2 * cfg.B * cfg.G * cfg.nkv() * cfg.blk * cfg.D * 2) / 1e6),
             "parallelism": "replicas" if world > 1 else "single",
+            "schedule": "balanced" if balanced else "plain",
         },
         "ms_per_chunk": ms_per_step,
         "kernels": kernels,
@@ -609,6 +616,9 @@ def main():
                     help="rotary position embedding: K rotated in the append, Q by uf_rope, at stream positions")
     ap.add_argument("--fp8", action="store_true",
                     help="FP8 scores: e4m3 K written by the append, e4m3 q . k on the tensor cores (static scales)")
+    ap.add_argument("--schedule", default="balanced", choices=["balanced", "plain"],
+                    help="attention call: uf_block_sparse_attn_balanced (kept blocks spread evenly over the SMs when "
+                         "there are fewer than 8 items per SM; the plain schedule otherwise) or uf_block_sparse_attn")
     ap.add_argument("--mask-local-only", action="store_true",
                     help="keep the local band only (the fixed-local-window mask)")
     args = ap.parse_args()

@@ -66,6 +66,8 @@ def _load() -> ctypes.CDLL:
         "uf_block_mask_local": ([vp, i32, pc, i32, i32, i32, vp, vp, vp, vp], i32),
         "uf_block_sparse_attn": ([vp, i32, pc, vp, vp, i32, ctypes.c_float, vp, vp, vp], i32),
         "uf_kv_append_fp8k": ([pc, vp, ctypes.c_float, vp, vp, i32, i32, vp], i32),
+        "uf_block_sparse_attn_balanced": ([vp, i32, pc, vp, vp, i32, ctypes.c_float, vp, vp, vp, sz, vp], i32),
+        "uf_attn_workspace_bytes": ([ctypes.POINTER(sz)], i32),
         "uf_block_sparse_attn_fp8k": ([vp, i32, pc, vp, ctypes.c_float, ctypes.c_float, vp, vp, i32, ctypes.c_float,
                                        vp, vp, vp], i32),
         "uf_check_error": ([vp, vp], i32),
@@ -182,6 +184,22 @@ def uf_block_sparse_attn(q, H: int, cache: UfKvCache, idx, cnt, k: int, scale: f
                          stream=None) -> None:
     _check(lib.uf_block_sparse_attn(_ptr(q), H, ctypes.byref(cache), _ptr(idx), _ptr(cnt), k, scale, _ptr(o),
                                     _ptr(lse), _stream(stream)), "uf_block_sparse_attn")
+
+
+def uf_attn_workspace_bytes() -> int:
+    """Workspace bytes of uf_block_sparse_attn_balanced on the current device."""
+    n = ctypes.c_size_t()
+    _check(lib.uf_attn_workspace_bytes(ctypes.byref(n)), "uf_attn_workspace_bytes")
+    return n.value
+
+
+def uf_block_sparse_attn_balanced(q, H: int, cache: UfKvCache, idx, cnt, k: int, scale: float, o, lse, workspace,
+                                  stream=None) -> None:
+    """workspace: a device tensor of at least uf_attn_workspace_bytes() bytes."""
+    nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib.uf_block_sparse_attn_balanced(_ptr(q), H, ctypes.byref(cache), _ptr(idx), _ptr(cnt), k, scale,
+                                             _ptr(o), _ptr(lse), _ptr(workspace), nbytes, _stream(stream)),
+           "uf_block_sparse_attn_balanced")
 
 
 def uf_kv_append_fp8k(cache: UfKvCache, k8, k_scale: float, k_new, v_new, keep_chunks: int, flags: int = 0,

@@ -90,7 +90,17 @@ struct AttnParams {
   float q_inv_scale;         // FP8 variant: 1 / q_scale
   long long wait_limit;      // bound of every pipeline wait (cycles)
   int32_t *err;              // the window's error word, or NULL (the module's)
+  // balanced schedule (NULL: thread block c takes items c, c + grid, ...):
+  int32_t *ws_cnt;           // [grid] arrival counters of split items, zero at launch
+  float *ws_part;            // [2 * grid][ATTN_PART_FLOATS] partial results
 };
+
+// One part of a split item: its unnormalised O (fp32, 128 rows x 128
+// channels, stored as [half x][16-byte chunk c][row] so that a warp's stores
+// are contiguous), then the reference max m (exp2 domain) and the row sum l
+// of each row relative to it.
+constexpr int ATTN_PART_O = 128 * 128;
+constexpr int ATTN_PART_FLOATS = ATTN_PART_O + 2 * 128;
 
 // Bound of the waits that let copies and MMAs already in flight finish before
 // a thread block that gave up exits: never below 2^31 cycles (about a second),
@@ -127,15 +137,71 @@ __device__ __forceinline__ void kv_block_coords(int j, int start, int W, int anc
   valid = (r == nb - 1) ? (Lc - (nb - 1) * blk) : blk;
 }
 
-// One work item as every role of the thread block sees it.
-struct AttnItem {
-  int i, h, b, g;             // q-block, query head, batch, kv head
-  int n;                      // kept kv blocks (< 1: nothing to compute)
-  int diag;                   // the q-block's own block in the newest chunk
-  const int32_t *row_idx;     // its block list, or NULL (dense: block t is t)
+// Which items a thread block takes.  Plain: items c, c + grid, c + 2 grid, ...
+// Balanced: the positions (item, kept block t) of all items, item-major, with
+// every item counted at its nominal length n_nom (dense: NKV, sparse: the row
+// stride k), are cut into gridDim.x contiguous ranges of equal length, one per
+// thread block; an item that straddles a range boundary is computed in parts
+// by several thread blocks and merged (see the epilogue).  Every role of a
+// thread block derives the same sequence from this.
+struct AttnSched {
+  bool split;
+  int n_nom;
+  long long T;                // items * n_nom
+  long long lo, hi;           // this thread block's positions [lo, hi)
+  int begin, end, step;       // items visited: begin, begin + step, ... < end
 };
 
-__device__ __forceinline__ AttnItem attn_item(const AttnParams &p, int item, int NKV, int n_valid) {
+__device__ __forceinline__ long long sched_start(long long T, int grid, int c) {
+  return static_cast<long long>(c) * T / grid;
+}
+// The thread block whose range holds position x: the largest c with sched_start(c) <= x.
+__device__ __forceinline__ int sched_owner(long long T, int grid, long long x) {
+  return static_cast<int>(((x + 1) * grid - 1) / T);
+}
+
+__device__ __forceinline__ AttnSched attn_sched(const AttnParams &p, int NKV) {
+  AttnSched s;
+  s.split = p.ws_part != nullptr && NKV > 0;
+  s.n_nom = 0;
+  s.T = s.lo = s.hi = 0;
+  if (!s.split) {
+    s.begin = blockIdx.x;
+    s.end = p.items;
+    s.step = gridDim.x;
+    return s;
+  }
+  s.n_nom = p.idx ? p.k : NKV;
+  s.T = static_cast<long long>(p.items) * s.n_nom;
+  s.lo = sched_start(s.T, gridDim.x, blockIdx.x);
+  s.hi = sched_start(s.T, gridDim.x, blockIdx.x + 1);
+  s.begin = static_cast<int>(s.lo / s.n_nom);
+  s.end = s.hi > s.lo ? static_cast<int>((s.hi - 1) / s.n_nom) + 1 : s.begin;
+  s.step = 1;
+  return s;
+}
+
+// Workspace slot of the part that thread block c computes of item `item`: a
+// block's first item in slot 2c, its last (when both are split) in 2c + 1.
+__device__ __forceinline__ int part_slot(const AttnSched &s, int c, int item) {
+  return 2 * c + (item == static_cast<int>(sched_start(s.T, gridDim.x, c) / s.n_nom) ? 0 : 1);
+}
+
+// One work item -- or this thread block's segment of it -- as every role of
+// the thread block sees it.
+struct AttnItem {
+  int i, h, b, g;             // q-block, query head, batch, kv head
+  int n;                      // kept kv blocks of the segment (< 1: nothing to compute)
+  int t0;                     // the segment's first entry in the item's block list
+  int diag;                   // the q-block's own block in the newest chunk
+  const int32_t *row_idx;     // its block list, or NULL (dense: block t is t)
+  bool empty_out;             // nothing to compute: this thread block writes O = 0, LSE = -inf
+  int nparts;                 // thread blocks computing a part of the item (1: not split)
+  int part0;                  // the first of them
+};
+
+__device__ __forceinline__ AttnItem attn_item(const AttnParams &p, const AttnSched &s, int item, int NKV,
+                                              int n_valid) {
   AttnItem it;
   it.i = item % p.nb;
   const int bh = item / p.nb;
@@ -150,14 +216,34 @@ __device__ __forceinline__ AttnItem attn_item(const AttnParams &p, int item, int
     if (it.n > p.k) it.n = -1;   // malformed row
   }
   if (NKV < 1) it.n = -1;
+  it.t0 = 0;
+  it.nparts = 1;
+  it.part0 = blockIdx.x;
+  it.empty_out = it.n < 1;
+  if (s.split) {
+    const long long base = static_cast<long long>(item) * s.n_nom;
+    if (it.n < 1) {
+      // written once, by the thread block holding the item's first position
+      it.empty_out = sched_owner(s.T, gridDim.x, base) == static_cast<int>(blockIdx.x);
+      it.n = -1;
+    } else {
+      // this block's positions of the item, clipped to its true length
+      const long long tb = s.lo > base ? s.lo - base : 0;
+      const long long te = s.hi - base < it.n ? s.hi - base : it.n;
+      it.part0 = sched_owner(s.T, gridDim.x, base);
+      it.nparts = sched_owner(s.T, gridDim.x, base + it.n - 1) - it.part0 + 1;
+      it.t0 = static_cast<int>(tb);
+      it.n = te > tb ? static_cast<int>(te - tb) : 0;
+    }
+  }
   return it;
 }
 
-// Kept block t of an item -> logical kv block of the window; an out-of-range
-// entry reads the diagonal block instead (`bad` tells the producer to record
-// the error).
+// Kept block t of a segment -> logical kv block of the window; an
+// out-of-range entry reads the diagonal block instead (`bad` tells the
+// producer to record the error).
 __device__ __forceinline__ int attn_block(const AttnItem &it, int t, int NKV, bool &bad) {
-  const int jb = it.row_idx ? __ldg(it.row_idx + t) : t;
+  const int jb = it.row_idx ? __ldg(it.row_idx + it.t0 + t) : it.t0 + t;
   bad = jb < 0 || jb >= NKV;
   return bad ? it.diag : jb;
 }
@@ -185,6 +271,10 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
   __shared__ uint64_t bar_vfull[ATTN_VSTAGE], bar_vempty[ATTN_VSTAGE];
   __shared__ uint64_t bar_s[2], bar_sfree[2], bar_o[2], bar_turn[2], bar_p;
   __shared__ uint64_t bar_fin[2];
+  // split items: every softmax thread has written its part / the arrival ticket is known
+  __shared__ uint64_t bar_pw, bar_tk;
+  __shared__ int32_t s_last;      // this thread block's part of the split item finished last
+  __shared__ int32_t s_store[2];  // the output of live item k is written (k mod 2)
   __shared__ float s_mref[128];   // reference max of each row (exp2 domain), published block by block
   __shared__ float s_l[2][128];   // epilogue: each warpgroup's partial row sums
   __shared__ uint32_t s_tbase;
@@ -195,6 +285,7 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
   const int start = __ldcg(p.meta + 0), n_valid = __ldcg(p.meta + 1), anchor = __ldcg(p.meta + 3);
   const bool bad_meta = !window_state_ok(start, n_valid, anchor, p.W);
   const int NKV = bad_meta ? 0 : n_valid * p.nb;
+  const AttnSched S = attn_sched(p, NKV);
 
   if (threadIdx.x == 0) {
     mbar_init(&bar_qfull, 1);
@@ -222,6 +313,8 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
       mbar_init(&bar_fin[s], 1);
     }
     mbar_init(&bar_p, ATTN_SOFTMAX_THREADS / 2);
+    mbar_init(&bar_pw, ATTN_SOFTMAX_THREADS);
+    mbar_init(&bar_tk, 1);
     s_abort = 0;
     fence_mbar_init();
     if (bad_meta && blockIdx.x == 0) record_error(p.err, UF_EBOUNDS);
@@ -252,8 +345,8 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
         uint32_t phase = 0;
         int issued = 0;
         bool ok = true;
-        for (int item = blockIdx.x; item < p.items && ok; item += gridDim.x) {
-          const AttnItem it = attn_item(p, item, NKV, n_valid);
+        for (int item = S.begin; item < S.end && ok; item += S.step) {
+          const AttnItem it = attn_item(p, S, item, NKV, n_valid);
           if (it.n < 1) continue;
           const int zc = it.b * p.G + it.g;
           for (int t = 0; t < it.n; ++t) {
@@ -318,14 +411,14 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
           tma_load_4d(sQ + L::Q_BYTES / 2, &tmQ, &bar_qfull, 64, a.h, a.i * BLK, a.b);
           ++q_loads;
         };
-        int item = blockIdx.x;
+        int item = S.begin;
         AttnItem it;
-        for (; item < p.items; item += gridDim.x) {
-          it = attn_item(p, item, NKV, n_valid);
+        for (; item < S.end; item += S.step) {
+          it = attn_item(p, S, item, NKV, n_valid);
           if (it.n >= 1) break;
         }
-        if (item < p.items) request_q(it);
-        while (item < p.items && ok) {
+        if (item < S.end) request_q(it);
+        while (item < S.end && ok) {
           if (FP8) {
             // the softmax threads have written the item's e4m3 Q into tensor memory
             if (!(ok = wait_bounded(&bar_q, kq & 1, abort_flag, p.wait_limit, p.err))) break;
@@ -345,7 +438,7 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
             if (!(ok = wait_bounded(&bar_qcp, kq & 1, abort_flag, p.wait_limit, p.err))) break;
           }
           tc_fence_after();
-          int item_next = p.items;
+          int item_next = S.end;
           AttnItem nxt;
           const int t_request = it.n > 1 ? 1 : 0;
           for (int t = 0; t < it.n; ++t) {
@@ -381,11 +474,11 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
               // with the item's first products on their way: the next live
               // item's Q, once the previous item's output stores have read
               // the staging tile
-              for (item_next = item + gridDim.x; item_next < p.items; item_next += gridDim.x) {
-                nxt = attn_item(p, item_next, NKV, n_valid);
+              for (item_next = item + S.step; item_next < S.end; item_next += S.step) {
+                nxt = attn_item(p, S, item_next, NKV, n_valid);
                 if (nxt.n >= 1) break;
               }
-              if (item_next < p.items) {
+              if (item_next < S.end) {
                 if (kq > 0 && !(ok = wait_bounded(&bar_ostore, (kq - 1) & 1, abort_flag, p.wait_limit, p.err))) break;
                 request_q(nxt);
               }
@@ -424,16 +517,18 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
           if (!wait_bounded(&bar_ofree, k & 1, abort_flag, p.wait_limit, p.err)) return false;
           if (!wait_bounded(&bar_st[0], k & 1, abort_flag, p.wait_limit, p.err)) return false;
           if (!wait_bounded(&bar_st[1], k & 1, abort_flag, p.wait_limit, p.err)) return false;
-          tma_store_4d(&tmO, sQ, 0, a.h, a.i * BLK, a.b);
-          tma_store_4d(&tmO, sQ + L::Q_BYTES / 2, 64, a.h, a.i * BLK, a.b);
-          bulk_commit();
-          bulk_wait_read();
+          if (s_store[k & 1]) {   // (not for a part of a split item that another block merges)
+            tma_store_4d(&tmO, sQ, 0, a.h, a.i * BLK, a.b);
+            tma_store_4d(&tmO, sQ + L::Q_BYTES / 2, 64, a.h, a.i * BLK, a.b);
+            bulk_commit();
+            bulk_wait_read();
+          }
           mbar_arrive(&bar_ostore);
           return true;
         };
         AttnItem prev;
-        for (int item = blockIdx.x; item < p.items && ok; item += gridDim.x) {
-          const AttnItem it = attn_item(p, item, NKV, n_valid);
+        for (int item = S.begin; item < S.end && ok; item += S.step) {
+          const AttnItem it = attn_item(p, S, item, NKV, n_valid);
           if (it.n < 1) continue;
           // the previous item's output leaves (and its epilogue has read O)
           if (kq > 0 && !(ok = store_output(prev, kq - 1))) break;
@@ -494,12 +589,12 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
     // first item at or after `from` (in this block's sequence) with blocks to
     // compute; the empty ones on the way are written here
     auto next_live = [&](int from, AttnItem &out) -> int {
-      for (int j = from; j < p.items; j += gridDim.x) {
-        out = attn_item(p, j, NKV, n_valid);
+      for (int j = from; j < S.end; j += S.step) {
+        out = attn_item(p, S, j, NKV, n_valid);
         if (out.n >= 1) return j;
-        write_empty(out);
+        if (out.empty_out) write_empty(out);
       }
-      return p.items;
+      return S.end;
     };
     // Q of live item number kq -> tensor memory, once it has landed and the
     // previous item's QK products have completed: this warpgroup copies
@@ -540,10 +635,11 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
     };
 
     AttnItem cur;
-    int item = next_live(blockIdx.x, cur);
-    bool ok = item >= p.items || !FP8 || load_q(0);
+    int item = next_live(S.begin, cur);
+    bool ok = item >= S.end || !FP8 || load_q(0);
+    int ks = 0;           // parts of split items written so far (parity of bar_pw / bar_tk)
     int kq = 0, g0 = 0;   // live items and kept blocks of this thread block so far
-    while (item < p.items && ok) {
+    while (item < S.end && ok) {
       const int n = cur.n;
       float m_run = -INFINITY;   // reference max this warpgroup last saw
       float l_run = 0.f;         // this warpgroup's partial row sum, relative to m_run
@@ -677,8 +773,8 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
       // the next live item's Q goes into tensor memory now, so that its first
       // QK products run during this item's epilogue
       AttnItem nxt;
-      const int item_next = next_live(item + gridDim.x, nxt);
-      if (FP8 && item_next < p.items && !(ok = load_q(kq + 1))) break;
+      const int item_next = next_live(item + S.step, nxt);
+      if (FP8 && item_next < S.end && !(ok = load_q(kq + 1))) break;
       // ---------------------------------------------------------- epilogue --
       // every PV of the item has completed once its last one has (one issuing
       // thread, completions in order)
@@ -688,11 +784,11 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
       // brought to it
       mbar_arrive(&bar_l);
       if (!(ok = wwait(&bar_l, 0))) break;
-      const float m_fin = s_mref[row];
+      float m_fin = s_mref[row];
       s_l[x][row] = n_mine > 0 ? l_run * ex2_approx(m_run - m_fin) : 0.f;
       mbar_arrive(&bar_l);
       if (!(ok = wwait(&bar_l, 1))) break;
-      const float l_tot = s_l[0][row] + s_l[1][row];
+      float l_tot = s_l[0][row] + s_l[1][row];
       tc_fence_after();
       // this warpgroup's half of the O row; O then goes back to the PV issuer
       uint32_t o[64];
@@ -701,29 +797,92 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(&bar_ofree);
+      bool store = true;
+      if (cur.nparts > 1) {
+        // a part of a split item: (O relative to m_fin, m_fin, l_tot) goes to
+        // the workspace; the thread block whose part arrives last merges all
+        // parts (log-sum-exp: every part brought to the largest reference) and
+        // writes the output.  No thread block waits for another.
+        float *part = p.ws_part + static_cast<size_t>(part_slot(S, blockIdx.x, item)) * ATTN_PART_FLOATS;
+        float4 *po = reinterpret_cast<float4 *>(part) + x * 16 * 128 + row;
+#pragma unroll
+        for (int c = 0; c < 16; ++c)
+          po[c * 128] = make_float4(__uint_as_float(o[4 * c]), __uint_as_float(o[4 * c + 1]),
+                                    __uint_as_float(o[4 * c + 2]), __uint_as_float(o[4 * c + 3]));
+        if (x == 0) {
+          part[ATTN_PART_O + row] = m_fin;
+          part[ATTN_PART_O + 128 + row] = l_tot;
+        }
+        __threadfence();
+        mbar_arrive(&bar_pw);
+        if (threadIdx.x == 128) {
+          int32_t last = 0;
+          if (wait_bounded(&bar_pw, ks & 1, abort_flag, p.wait_limit, p.err)) {
+            __threadfence();
+            last = atomicAdd(p.ws_cnt + cur.part0, 1) == cur.nparts - 1;
+          }
+          s_last = last;
+          mbar_arrive(&bar_tk);
+        }
+        if (!(ok = wwait(&bar_tk, ks & 1))) break;
+        ++ks;
+        store = s_last != 0;
+        if (store) {
+          __threadfence();
+          float m_all = m_fin;
+          for (int q = cur.part0; q < cur.part0 + cur.nparts; ++q)
+            if (q != static_cast<int>(blockIdx.x))
+              m_all = fmaxf(m_all, __ldcg(p.ws_part + static_cast<size_t>(part_slot(S, q, item)) * ATTN_PART_FLOATS +
+                                          ATTN_PART_O + row));
+          const float f_own = ex2_approx(m_fin - m_all);
+          float l_all = l_tot * f_own;
+#pragma unroll
+          for (int e = 0; e < 64; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f_own);
+          for (int q = cur.part0; q < cur.part0 + cur.nparts; ++q) {
+            if (q == static_cast<int>(blockIdx.x)) continue;
+            const float *pq = p.ws_part + static_cast<size_t>(part_slot(S, q, item)) * ATTN_PART_FLOATS;
+            const float fq = ex2_approx(__ldcg(pq + ATTN_PART_O + row) - m_all);
+            l_all += __ldcg(pq + ATTN_PART_O + 128 + row) * fq;
+            const float4 *pq4 = reinterpret_cast<const float4 *>(pq) + x * 16 * 128 + row;
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+              const float4 v = __ldcg(pq4 + c * 128);
+              o[4 * c] = __float_as_uint(fmaf(v.x, fq, __uint_as_float(o[4 * c])));
+              o[4 * c + 1] = __float_as_uint(fmaf(v.y, fq, __uint_as_float(o[4 * c + 1])));
+              o[4 * c + 2] = __float_as_uint(fmaf(v.z, fq, __uint_as_float(o[4 * c + 2])));
+              o[4 * c + 3] = __float_as_uint(fmaf(v.w, fq, __uint_as_float(o[4 * c + 3])));
+            }
+          }
+          m_fin = m_all;
+          l_tot = l_all;
+        }
+      }
+      if (threadIdx.x == 128) s_store[kq & 1] = store;   // read by the PV issuer after bar_st
       // (bf16 path: the QK issuer's copy of the next item's Q out of the staging
       // tile has completed)
-      if (!FP8 && item_next < p.items && !(ok = wwait(&bar_qcp, (kq + 1) & 1))) break;
+      if (!FP8 && item_next < S.end && !(ok = wwait(&bar_qcp, (kq + 1) & 1))) break;
       // this warpgroup's 64-column half of the bf16 row -> the staging tile
       // (the next item's Q has left it), 128-byte swizzled like a TMA tile:
       // 16-byte chunk c of row r at chunk c ^ (r mod 8)
-      const float inv_l = 1.f / l_tot;
-      uint8_t *panel = sQ + x * (L::Q_BYTES / 2) + row * 128;
+      if (store) {
+        const float inv_l = 1.f / l_tot;
+        uint8_t *panel = sQ + x * (L::Q_BYTES / 2) + row * 128;
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        uint32_t w[4];
+        for (int c = 0; c < 8; ++c) {
+          uint32_t w[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int k0 = 8 * c + 2 * e;
-          w[e] = pack_bf16x2(__uint_as_float(o[k0]) * inv_l, __uint_as_float(o[k0 + 1]) * inv_l);
+          for (int e = 0; e < 4; ++e) {
+            const int k0 = 8 * c + 2 * e;
+            w[e] = pack_bf16x2(__uint_as_float(o[k0]) * inv_l, __uint_as_float(o[k0 + 1]) * inv_l);
+          }
+          *reinterpret_cast<uint4 *>(panel + ((c ^ (row & 7)) * 16)) = make_uint4(w[0], w[1], w[2], w[3]);
         }
-        *reinterpret_cast<uint4 *>(panel + ((c ^ (row & 7)) * 16)) = make_uint4(w[0], w[1], w[2], w[3]);
       }
       // (the PV issuer writes the tile out)
       fence_proxy_async_smem();
       mbar_arrive(&bar_st[x]);
       const int q_tok = cur.i * BLK + row;
-      if (row < BLK && q_tok < p.Lc && p.lse && x == 0)
+      if (store && row < BLK && q_tok < p.Lc && p.lse && x == 0)
         p.lse[(static_cast<size_t>(cur.b) * p.H + cur.h) * p.Lc + q_tok] = (m_fin + log2f(l_tot)) * 0.69314718055994531f;
       g0 += n;
       ++kq;

@@ -250,9 +250,22 @@ int32_t append_impl(uf_kv_cache *c, const void *k_new, const void *v_new, int32_
 }  // namespace
 
 namespace {
-// uf_block_sparse_attn and its FP8-score variant (k8 != NULL).
+// Workspace of the balanced schedule for `sms` thread blocks: arrival
+// counters (one per thread block, padded to 256 bytes), then two partial
+// results per thread block.
+size_t attn_ws_cnt_bytes(int sms) { return (static_cast<size_t>(sms) * 4 + 255) / 256 * 256; }
+size_t attn_ws_bytes(int sms) {
+  return attn_ws_cnt_bytes(sms) + 2 * static_cast<size_t>(sms) * uf::ATTN_PART_FLOATS * sizeof(float);
+}
+// The balanced schedule pays off when there are few items per SM (the last
+// round of items leaves SMs idle); with many items the plain one is as even.
+constexpr long long kBalancedItemsPerSm = 8;
+
+// uf_block_sparse_attn, its FP8-score variant (k8 != NULL) and the balanced
+// variant (ws != NULL: workspace of attn_ws_bytes(SM count) bytes).
 int32_t attn_impl(const void *q, int32_t H, const uf_kv_cache *c, const int32_t *idx, const int32_t *cnt, int32_t k,
-                  float scale, void *o, float *lse, uf_stream_t s, const void *k8, float q_scale, float k_scale) {
+                  float scale, void *o, float *lse, uf_stream_t s, const void *k8, float q_scale, float k_scale,
+                  void *ws = nullptr, size_t ws_bytes = 0) {
   if (!cache_ok(c)) return UF_EINVAL;
   if (!q || !o || !aligned16(q) || !aligned16(o)) return UF_EINVAL;
   if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return UF_EINVAL;
@@ -327,12 +340,25 @@ int32_t attn_impl(const void *q, int32_t H, const uf_kv_cache *c, const int32_t 
   p.q_inv_scale = 1.0f / q_scale;
   p.wait_limit = g_wait_limit.load();
   p.err = c->err;
+  p.ws_cnt = nullptr;
+  p.ws_part = nullptr;
   int sms = 0;
   const int32_t se = sm_count(&sms);
   if (se != UF_OK) return se;
-  const unsigned grid = static_cast<unsigned>(items < sms ? items : sms);
+  unsigned grid = static_cast<unsigned>(items < sms ? items : sms);
   cudaGetLastError();
   const cudaStream_t st = reinterpret_cast<cudaStream_t>(s);
+  if (ws) {
+    if (!aligned16(ws) || ws_bytes < attn_ws_bytes(sms)) return UF_EINVAL;
+    if (items < kBalancedItemsPerSm * sms) {
+      // balanced schedule: one thread block per SM, counters zeroed first
+      p.ws_cnt = static_cast<int32_t *>(ws);
+      p.ws_part = reinterpret_cast<float *>(static_cast<char *>(ws) + attn_ws_cnt_bytes(sms));
+      grid = static_cast<unsigned>(sms);
+      const int32_t e = cuda_status(cudaMemsetAsync(p.ws_cnt, 0, static_cast<size_t>(sms) * 4, st));
+      if (e != UF_OK) return e;
+    }
+  }
   const bool fp8 = k8 != nullptr;
   if (c->blk == 128) {
     constexpr int smem = uf::AttnSmem<128>::DYN;
@@ -507,6 +533,22 @@ int32_t uf_block_mask_local(const void *q, int32_t H, const uf_kv_cache *c, int3
 int32_t uf_block_sparse_attn(const void *q, int32_t H, const uf_kv_cache *c, const int32_t *idx, const int32_t *cnt,
                              int32_t k, float scale, void *o, float *lse, uf_stream_t s) {
   return attn_impl(q, H, c, idx, cnt, k, scale, o, lse, s, nullptr, 1.0f, 1.0f);
+}
+
+int32_t uf_attn_workspace_bytes(size_t *bytes) {
+  if (!bytes) return UF_EINVAL;
+  int sms = 0;
+  const int32_t se = sm_count(&sms);
+  if (se != UF_OK) return se;
+  *bytes = attn_ws_bytes(sms);
+  return UF_OK;
+}
+
+int32_t uf_block_sparse_attn_balanced(const void *q, int32_t H, const uf_kv_cache *c, const int32_t *idx,
+                                      const int32_t *cnt, int32_t k, float scale, void *o, float *lse,
+                                      void *workspace, size_t workspace_bytes, uf_stream_t s) {
+  if (!workspace) return UF_EINVAL;
+  return attn_impl(q, H, c, idx, cnt, k, scale, o, lse, s, nullptr, 1.0f, 1.0f, workspace, workspace_bytes);
 }
 
 int32_t uf_block_sparse_attn_fp8k(const void *q, int32_t H, const uf_kv_cache *c, const void *k8, float q_scale,

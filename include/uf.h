@@ -331,6 +331,43 @@ int32_t uf_block_sparse_attn(const void *q, int32_t H, const uf_kv_cache *c,
                              void *o, float *lse, uf_stream_t s);
 
 /*
+ * Balanced variant of uf_block_sparse_attn, for workloads with few work items
+ * per SM (grouped-query decoder steps, small chunks): the positions (item,
+ * kept block) of all (b, h, q-block) items, every item counted at its nominal
+ * length (dense: every block of the window; sparse: the row stride k), are
+ * cut into one contiguous range of equal length per SM, so every SM computes
+ * the same number of kept blocks.  An item whose blocks fall into several
+ * ranges is computed in parts; each part writes its unnormalised O, row max
+ * and row sum to the workspace, and the part that finishes last merges them
+ * (log-sum-exp, in fp32) and writes O and LSE.  No thread block waits for
+ * another.  Softmax attention is exact on its kept set, so the result is
+ * uf_block_sparse_attn's up to fp32 rounding (Ultra Flash notes, key design
+ * 3; FlashDecoder Sec. 3, Eq. 4).
+ *
+ *   workspace        device memory of at least uf_attn_workspace_bytes()
+ *                    bytes, 16-byte aligned, caller-owned; its contents need
+ *                    no initialisation (the call zeroes the counters it uses
+ *                    on stream s before the kernel).  Calls that may run at
+ *                    the same time need separate workspaces.
+ *   workspace_bytes  its size.
+ *   other arguments, outputs and errors as uf_block_sparse_attn.
+ *
+ * With many items per SM (at least 8) the plain schedule is already even
+ * and is used unchanged (the workspace is not touched).  One memset and one
+ * kernel launch.
+ */
+int32_t uf_block_sparse_attn_balanced(const void *q, int32_t H, const uf_kv_cache *c, const int32_t *idx,
+                                      const int32_t *cnt, int32_t k, float scale, void *o, float *lse,
+                                      void *workspace, size_t workspace_bytes, uf_stream_t s);
+
+/*
+ * Workspace size of uf_block_sparse_attn_balanced on the current device
+ * (two partial results of 65 KB per SM plus counters; 19.7 MB on a 148-SM
+ * B200), into *bytes.  Host only.
+ */
+int32_t uf_attn_workspace_bytes(size_t *bytes);
+
+/*
  * FP8-score variant, append side (FlashDecoder, inference optimisations:
  * statically calibrated FP8).  uf_kv_append(c, k_new, v_new, keep_chunks,
  * flags, s) that also writes an e4m3 copy of each appended K row:

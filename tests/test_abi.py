@@ -184,6 +184,10 @@ def test_calls_reject_bad_arguments_before_launch(uf):
         assert e.value.status == uf.UF_EINVAL
     with pytest.raises(uf.UfError):
         uf.uf_block_sparse_attn(q, 2, c, idx, cnt, 9, 0.088, FakeTensor(0xA00000), None, stream=0)
+    # balanced schedule: a workspace is required
+    with pytest.raises(uf.UfError) as e:
+        uf.uf_block_sparse_attn_balanced(q, 2, c, None, None, 0, 0.088, FakeTensor(0xA00000), None, None, stream=0)
+    assert e.value.status == uf.UF_EINVAL
     with pytest.raises(uf.UfError):
         uf.uf_block_sparse_attn(q, 2, c, None, None, 0, 0.088, FakeTensor(0xA00001), None, stream=0)
 
