@@ -140,13 +140,15 @@ __device__ __forceinline__ void kv_block_coords(int j, int start, int W, int anc
 // Which items a thread block takes.  Plain: items c, c + grid, c + 2 grid, ...
 // Balanced: the positions (item, kept block t) of all items, item-major, with
 // every item counted at its nominal length n_nom (dense: NKV, sparse: the row
-// stride k), are cut into gridDim.x contiguous ranges of equal length, one per
-// thread block; an item that straddles a range boundary is computed in parts
-// by several thread blocks and merged (see the epilogue).  Every role of a
-// thread block derives the same sequence from this.
+// stride k), are cut into g = min(gridDim.x, positions) contiguous ranges of
+// equal length (none empty), one per thread block c < g; an item that
+// straddles a range boundary is computed in parts by consecutive thread
+// blocks and merged (see the epilogue).  Every role of a thread block derives
+// the same sequence from this.
 struct AttnSched {
   bool split;
   int n_nom;
+  int g;                      // thread blocks with a range
   long long T;                // items * n_nom
   long long lo, hi;           // this thread block's positions [lo, hi)
   int begin, end, step;       // items visited: begin, begin + step, ... < end
@@ -164,6 +166,7 @@ __device__ __forceinline__ AttnSched attn_sched(const AttnParams &p, int NKV) {
   AttnSched s;
   s.split = p.ws_part != nullptr && NKV > 0;
   s.n_nom = 0;
+  s.g = gridDim.x;
   s.T = s.lo = s.hi = 0;
   if (!s.split) {
     s.begin = blockIdx.x;
@@ -173,8 +176,15 @@ __device__ __forceinline__ AttnSched attn_sched(const AttnParams &p, int NKV) {
   }
   s.n_nom = p.idx ? p.k : NKV;
   s.T = static_cast<long long>(p.items) * s.n_nom;
-  s.lo = sched_start(s.T, gridDim.x, blockIdx.x);
-  s.hi = sched_start(s.T, gridDim.x, blockIdx.x + 1);
+  s.g = static_cast<int>(s.T < gridDim.x ? s.T : gridDim.x);
+  if (static_cast<int>(blockIdx.x) >= s.g) {   // more thread blocks than positions: nothing to do
+    s.lo = s.hi = s.T;
+    s.begin = s.end = p.items;
+    s.step = 1;
+    return s;
+  }
+  s.lo = sched_start(s.T, s.g, blockIdx.x);
+  s.hi = sched_start(s.T, s.g, blockIdx.x + 1);
   s.begin = static_cast<int>(s.lo / s.n_nom);
   s.end = s.hi > s.lo ? static_cast<int>((s.hi - 1) / s.n_nom) + 1 : s.begin;
   s.step = 1;
@@ -184,7 +194,7 @@ __device__ __forceinline__ AttnSched attn_sched(const AttnParams &p, int NKV) {
 // Workspace slot of the part that thread block c computes of item `item`: a
 // block's first item in slot 2c, its last (when both are split) in 2c + 1.
 __device__ __forceinline__ int part_slot(const AttnSched &s, int c, int item) {
-  return 2 * c + (item == static_cast<int>(sched_start(s.T, gridDim.x, c) / s.n_nom) ? 0 : 1);
+  return 2 * c + (item == static_cast<int>(sched_start(s.T, s.g, c) / s.n_nom) ? 0 : 1);
 }
 
 // One work item -- or this thread block's segment of it -- as every role of
@@ -224,14 +234,14 @@ __device__ __forceinline__ AttnItem attn_item(const AttnParams &p, const AttnSch
     const long long base = static_cast<long long>(item) * s.n_nom;
     if (it.n < 1) {
       // written once, by the thread block holding the item's first position
-      it.empty_out = sched_owner(s.T, gridDim.x, base) == static_cast<int>(blockIdx.x);
+      it.empty_out = sched_owner(s.T, s.g, base) == static_cast<int>(blockIdx.x);
       it.n = -1;
     } else {
       // this block's positions of the item, clipped to its true length
       const long long tb = s.lo > base ? s.lo - base : 0;
       const long long te = s.hi - base < it.n ? s.hi - base : it.n;
-      it.part0 = sched_owner(s.T, gridDim.x, base);
-      it.nparts = sched_owner(s.T, gridDim.x, base + it.n - 1) - it.part0 + 1;
+      it.part0 = sched_owner(s.T, s.g, base);
+      it.nparts = sched_owner(s.T, s.g, base + it.n - 1) - it.part0 + 1;
       it.t0 = static_cast<int>(tb);
       it.n = te > tb ? static_cast<int>(te - tb) : 0;
     }
