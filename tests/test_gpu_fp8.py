@@ -21,7 +21,7 @@ import torch
 
 import oracle
 from uf_testlib import (E4M3_QUOTIENT_REL, LSE_ABS, O_MAX_ABS, O_MEAN_ABS, GpuStream, OracleStream,
-                        assert_attention_ok, e4m3_codes_agree, oracle_idx_array, sample_items)
+                        assert_attention_ok, e4m3_codes_agree, fill_window, oracle_idx_array, sample_items)
 from workloads import CONFIGS, chunk_inputs, scaled
 
 pytestmark = [pytest.mark.gpu,
@@ -84,6 +84,7 @@ def test_fp8_k_codes_bit_exact(name, anchor):
     # arbitrary (not power-of-two) scales: codes equal up to the near-boundary rule
     cfg = CASES[name]
     gpu, orc, _, _, ks = _stream(cfg, cfg.W + 2, seed=21, anchor=anchor, pow2=False)
+    n_near = 0
     k8 = gpu.win.k8.view(torch.float8_e4m3fn).to(torch.float64).cpu().numpy()
     raw = gpu.win.k8.cpu().numpy()
     for g in range(cfg.G):
@@ -93,6 +94,8 @@ def test_fp8_k_codes_bit_exact(name, anchor):
             r0 = slot * gpu.win.lslot
             near, bad = e4m3_codes_agree(k8[:, g, r0:r0 + cfg.Lc], w.k[c][:, :, 0, :], ks)
             assert not bad.any(), (g, c, int(bad.sum()))
+            n_near += near
+    print(f"{name}: {n_near} e4m3 codes differ from the oracle's, each next to a rounding boundary")
             assert not raw[:, g, r0 + cfg.Lc:r0 + gpu.win.lslot].any(), "padding rows must be zero"
 
 
@@ -144,11 +147,16 @@ def _near_boundary(x, scale):
 
 @pytest.mark.parametrize("name", ["blk64", "sr_w3"])
 def test_fp8_attention_arbitrary_scales_untouched_rows(name):
-    # scales amax / 448 as they are: every row whose q and whose kept keys hold
-    # no near-boundary element must meet the bf16 tolerances; the rows that do
-    # are few
+    # scales that are not powers of two: every row whose q and whose kept keys
+    # hold no near-boundary element must meet the bf16 tolerances.  The scales
+    # are amax / 448 times 1.0123457, not a simple fraction of the bf16 data's
+    # amax (amax / 448 itself puts many bf16 values exactly on e4m3 midpoints,
+    # e.g. 0.75 amax on 336; those cases are the code test's), so the rows
+    # touched are few
     cfg = CASES[name]
-    gpu, orc, last, qs, ks = _stream(cfg, cfg.W + 1, seed=26, pow2=False)
+    qs, ks = (float(np.float32(x * 1.0123457)) for x in static_scales(cfg, 26, pow2=False))
+    gpu, orc = GpuStream(cfg, k_scale=ks), OracleStream(cfg)
+    last = fill_window(cfg, 26, cfg.W + 1, gpu, orc)
     k = cfg.k_for()
     oidx, ocnt = oracle_idx_array(cfg, orc.mask(last["q"], k))
     o, lse = gpu.attention_fp8(last["q"], qs, torch.from_numpy(oidx).cuda(), torch.from_numpy(ocnt).cuda(),
