@@ -95,8 +95,8 @@ def test_fp8_k_codes_bit_exact(name, anchor):
             near, bad = e4m3_codes_agree(k8[:, g, r0:r0 + cfg.Lc], w.k[c][:, :, 0, :], ks)
             assert not bad.any(), (g, c, int(bad.sum()))
             n_near += near
-    print(f"{name}: {n_near} e4m3 codes differ from the oracle's, each next to a rounding boundary")
             assert not raw[:, g, r0 + cfg.Lc:r0 + gpu.win.lslot].any(), "padding rows must be zero"
+    print(f"{name}: {n_near} e4m3 codes differ from the oracle's, each next to a rounding boundary")
 
 
 def test_fp8_k_code_at_an_exact_midpoint():
