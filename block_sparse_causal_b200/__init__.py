@@ -7,6 +7,7 @@ of the hot path runs in the CUDA kernels.
 from ._uf import (UF_APPEND_ANCHOR, UF_APPEND_REPLACE_NEWEST, UF_EBOUNDS, UF_ECUDA, UF_EINVAL, UF_ETIMEOUT,
                   UF_EUNSUPPORTED, UF_MASK_LOCAL_ONLY, UF_OK, UfError, UfKvCache, strerror, uf_block_mask,
                   uf_attn_workspace_bytes, uf_block_mask_local, uf_block_sparse_attn, uf_block_sparse_attn_balanced,
+                  uf_block_sparse_attn_balanced_noalloc,
                   uf_block_sparse_attn_fp8k, uf_check_error,
                   uf_debug_wait_timeout, uf_get_error, uf_kv_append, uf_kv_append_fp8k, uf_kv_append_rope,
                   uf_kv_append_tiled, uf_kv_cache_bytes, uf_kv_cache_init, uf_kv_cache_set_error_word, uf_kv_reset,
@@ -18,6 +19,7 @@ __all__ = [
     "UF_APPEND_ANCHOR", "UF_APPEND_REPLACE_NEWEST", "UF_EBOUNDS", "UF_ECUDA", "UF_EINVAL", "UF_ETIMEOUT",
     "UF_EUNSUPPORTED", "UF_MASK_LOCAL_ONLY", "UF_OK", "UfError", "UfKvCache", "strerror", "uf_block_mask",
     "uf_attn_workspace_bytes", "uf_block_mask_local", "uf_block_sparse_attn", "uf_block_sparse_attn_balanced",
+    "uf_block_sparse_attn_balanced_noalloc",
     "uf_block_sparse_attn_fp8k", "uf_check_error",
     "uf_debug_wait_timeout", "uf_get_error", "uf_kv_append", "uf_kv_append_fp8k", "uf_kv_append_rope",
     "uf_kv_append_tiled", "uf_kv_cache_bytes", "uf_kv_cache_init", "uf_kv_cache_set_error_word", "uf_kv_reset",

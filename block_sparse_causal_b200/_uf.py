@@ -68,6 +68,7 @@ def _load() -> ctypes.CDLL:
         "uf_kv_append_fp8k": ([pc, vp, ctypes.c_float, vp, vp, i32, i32, vp], i32),
         "uf_block_sparse_attn_balanced": ([vp, i32, pc, vp, vp, i32, ctypes.c_float, vp, vp, vp, sz, vp], i32),
         "uf_attn_workspace_bytes": ([ctypes.POINTER(sz)], i32),
+        "uf_block_sparse_attn_balanced_noalloc": ([vp, i32, pc, vp, vp, i32, ctypes.c_float, vp, vp, vp], i32),
         "uf_block_sparse_attn_fp8k": ([vp, i32, pc, vp, ctypes.c_float, ctypes.c_float, vp, vp, i32, ctypes.c_float,
                                        vp, vp, vp], i32),
         "uf_check_error": ([vp, vp], i32),
@@ -200,6 +201,15 @@ def uf_block_sparse_attn_balanced(q, H: int, cache: UfKvCache, idx, cnt, k: int,
     _check(lib.uf_block_sparse_attn_balanced(_ptr(q), H, ctypes.byref(cache), _ptr(idx), _ptr(cnt), k, scale,
                                              _ptr(o), _ptr(lse), _ptr(workspace), nbytes, _stream(stream)),
            "uf_block_sparse_attn_balanced")
+
+
+def uf_block_sparse_attn_balanced_noalloc(q, H: int, cache: UfKvCache, idx, cnt, k: int, scale: float, o, lse=None,
+                                          stream=None) -> None:
+    """uf_block_sparse_attn_balanced with the library's own fixed scratch array
+    (no workspace argument, nothing allocated)."""
+    _check(lib.uf_block_sparse_attn_balanced_noalloc(_ptr(q), H, ctypes.byref(cache), _ptr(idx), _ptr(cnt), k,
+                                                     scale, _ptr(o), _ptr(lse), _stream(stream)),
+           "uf_block_sparse_attn_balanced_noalloc")
 
 
 def uf_kv_append_fp8k(cache: UfKvCache, k8, k_scale: float, k_new, v_new, keep_chunks: int, flags: int = 0,

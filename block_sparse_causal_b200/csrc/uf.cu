@@ -551,6 +551,62 @@ int32_t uf_block_sparse_attn_balanced(const void *q, int32_t H, const uf_kv_cach
   return attn_impl(q, H, c, idx, cnt, k, scale, o, lse, s, nullptr, 1.0f, 1.0f, workspace, workspace_bytes);
 }
 
+}  // extern "C"
+
+namespace {
+// Scratch memory of uf_block_sparse_attn_balanced_noalloc: one fixed array in
+// the library's device image, the balanced schedule's workspace for devices
+// of at most kNoAllocMaxSms SMs.  It exists on every device that loads the
+// library, from module load until the process exits.  Host code must not use
+// the symbol itself as an address (on the host it names a host-side shadow):
+// the device address comes from cudaGetSymbolAddress, once per device.
+constexpr int kNoAllocMaxSms = 160;
+constexpr size_t kNoAllocScratchBytes =
+    (static_cast<size_t>(kNoAllocMaxSms) * 4 + 255) / 256 * 256 +
+    2 * static_cast<size_t>(kNoAllocMaxSms) * uf::ATTN_PART_FLOATS * sizeof(float);
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+std::atomic<void *> g_noalloc_addr[kMaxDevices];
+std::mutex g_noalloc_mutex;
+
+// Device address of the scratch array on the current device (looked up on the
+// first call per device, with that device current).
+int32_t noalloc_scratch(void **out) {
+  int dev = 0;
+  const int32_t st = cuda_status(cudaGetDevice(&dev));
+  if (st != UF_OK) return st;
+  if (dev < 0 || dev >= kMaxDevices) return UF_EUNSUPPORTED;
+  void *p = g_noalloc_addr[dev].load();
+  if (!p) {
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    p = g_noalloc_addr[dev].load();
+    if (!p) {
+      const int32_t st2 = cuda_status(cudaGetSymbolAddress(&p, g_noalloc_scratch));
+      if (st2 != UF_OK) return st2;
+      if (!p) return UF_ECUDA;
+      g_noalloc_addr[dev].store(p);
+    }
+  }
+  *out = p;
+  return UF_OK;
+}
+}  // namespace
+
+extern "C" {
+
+int32_t uf_block_sparse_attn_balanced_noalloc(const void *q, int32_t H, const uf_kv_cache *c, const int32_t *idx,
+                                              const int32_t *cnt, int32_t k, float scale, void *o, float *lse,
+                                              uf_stream_t s) {
+  int sms = 0;
+  const int32_t se = sm_count(&sms);
+  if (se != UF_OK) return se;
+  if (attn_ws_bytes(sms) > kNoAllocScratchBytes) return UF_EUNSUPPORTED;   // more SMs than the array serves
+  void *ws = nullptr;
+  const int32_t sa = noalloc_scratch(&ws);
+  if (sa != UF_OK) return sa;
+  return attn_impl(q, H, c, idx, cnt, k, scale, o, lse, s, nullptr, 1.0f, 1.0f, ws, kNoAllocScratchBytes);
+}
+
 int32_t uf_block_sparse_attn_fp8k(const void *q, int32_t H, const uf_kv_cache *c, const void *k8, float q_scale,
                                   float k_scale, const int32_t *idx, const int32_t *cnt, int32_t k, float scale,
                                   void *o, float *lse, uf_stream_t s) {

@@ -361,6 +361,35 @@ int32_t uf_block_sparse_attn_balanced(const void *q, int32_t H, const uf_kv_cach
                                       void *workspace, size_t workspace_bytes, uf_stream_t s);
 
 /*
+ * uf_block_sparse_attn_balanced for callers that cannot allocate device
+ * memory.  The pages have no counterpart to this call: it only changes where
+ * the balanced schedule keeps its scratch data.  Some callers cannot call
+ * cudaMalloc or hand the library a buffer of their own: a plugin inside a host
+ * framework that owns every device byte through its own pool, a real-time
+ * streaming loop that must not allocate after start-up (an allocation can
+ * synchronise the device and stall the stream), or a process that has
+ * reserved all free memory for its KV windows.  This call allocates nothing:
+ * it calls no cudaMalloc, cudaFree or allocating library routine, and the
+ * scratch is a fixed array of 21,299,968 bytes compiled into the library (two
+ * 65 KB partial results per SM for up to 160 SMs, plus counters), which every
+ * device that loads the library holds until the process exits.
+ *
+ *   arguments, outputs and errors as uf_block_sparse_attn_balanced, without
+ *   workspace and workspace_bytes.  UF_EUNSUPPORTED when the current device
+ *   has more than 160 SMs (its scratch would not fit the array).
+ *
+ * The first call on a device looks up the array's device address (with that
+ * device current) and caches it; make that first call before any stream
+ * capture.  All calls on a device share the one array, and each call clears
+ * the counters it needs on stream s before its kernel: calls that may run on
+ * the GPU at the same time (other streams, other host threads) race on it and
+ * must be ordered by the caller.
+ */
+int32_t uf_block_sparse_attn_balanced_noalloc(const void *q, int32_t H, const uf_kv_cache *c,
+                                              const int32_t *idx, const int32_t *cnt, int32_t k, float scale,
+                                              void *o, float *lse, uf_stream_t s);
+
+/*
  * Workspace size of uf_block_sparse_attn_balanced on the current device
  * (two partial results of 65 KB per SM plus counters; 19.7 MB on a 148-SM
  * B200), into *bytes.  Host only.
