@@ -823,13 +823,17 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
           part[ATTN_PART_O + row] = m_fin;
           part[ATTN_PART_O + 128 + row] = l_tot;
         }
-        __threadfence();
+        // every thread's stores precede thread 128's fence (the barrier orders
+        // them within the block; the fence is cumulative), which precedes the
+        // arrival count; the part that counts last fences again before its
+        // threads read the other parts (from L2)
         mbar_arrive(&bar_pw);
         if (threadIdx.x == 128) {
           int32_t last = 0;
           if (wait_bounded(&bar_pw, ks & 1, abort_flag, p.wait_limit, p.err)) {
             __threadfence();
             last = atomicAdd(p.ws_cnt + cur.part0, 1) == cur.nparts - 1;
+            if (last) __threadfence();
           }
           s_last = last;
           mbar_arrive(&bar_tk);
@@ -838,7 +842,6 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
         ++ks;
         store = s_last != 0;
         if (store) {
-          __threadfence();
           float m_all = m_fin;
           for (int q = cur.part0; q < cur.part0 + cur.nparts; ++q)
             if (q != static_cast<int>(blockIdx.x))

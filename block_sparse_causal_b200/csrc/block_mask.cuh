@@ -16,9 +16,12 @@
 //   1. pool: warp w sums q-block i0 + w over its tokens in fp32, each lane 8
 //      channels of every other token with 16-byte loads, 16 in flight;
 //   2. score: on the tensor core, m16n8k8 tf32 MMAs with fp32 accuracy by a
-//      hi / lo split of both operands (hi.hi + hi.lo + lo.hi); each warp
-//      takes one 16-row half of its stage's tiles against the 8 pooled
-//      queries (held in registers as B fragments);
+//      hi / lo split of both operands (hi = the top 19 bits of the fp32
+//      value, lo = the exact remainder, which the MMA reads to 11 bits:
+//      products within 2^-21 relative), as hi.hi + hi.lo + lo.hi in three
+//      accumulators so the MMA chains overlap; each warp takes one 16-row
+//      half of its stage's tiles against the 8 pooled queries (held in
+//      registers as B fragments);
 //   3. select: one warp per q-block row forces the diagonal (or the local
 //      band around it), finds the need-th largest of the other scores (need =
 //      k minus the forced blocks) by a 32-step bitwise search over
@@ -196,8 +199,8 @@ __global__ void __launch_bounds__(MASK_THREADS, 2) block_mask_kernel(const MaskP
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
       const float v = s_qpool[gid * D + kk * 8 + tig + 4 * e];
-      bh[kk][e] = to_tf32(v);
-      bl[kk][e] = to_tf32(v - __uint_as_float(bh[kk][e]));
+      bh[kk][e] = __float_as_uint(v) & 0xFFFFE000u;
+      bl[kk][e] = __float_as_uint(v - __uint_as_float(bh[kk][e]));
     }
   const int mh = warp & 1;                // this warp's 16-row half of each tile
   for (int t = pair; t < ntiles; t += MASK_KSTAGE) {
@@ -205,7 +208,7 @@ __global__ void __launch_bounds__(MASK_THREADS, 2) block_mask_kernel(const MaskP
     // needs both); after an abort the waits return at once and nothing is issued
     if (wait_bounded(&bar_k[pair], (t / MASK_KSTAGE) & 1, &s_abort, kWait, p.err)) {
       const float *kt = s_kt + (pair * MASK_KT + mh * 16) * MASK_KSTRIDE;
-      float d[4] = {0.f, 0.f, 0.f, 0.f};
+      float dhh[4] = {0.f, 0.f, 0.f, 0.f}, dhl[4] = {0.f, 0.f, 0.f, 0.f}, dlh[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int kk = 0; kk < D / 8; ++kk) {
         const float av[4] = {kt[gid * MASK_KSTRIDE + kk * 8 + tig], kt[(gid + 8) * MASK_KSTRIDE + kk * 8 + tig],
@@ -214,13 +217,16 @@ __global__ void __launch_bounds__(MASK_THREADS, 2) block_mask_kernel(const MaskP
         uint32_t ah[4], al[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          ah[e] = to_tf32(av[e]);
-          al[e] = to_tf32(av[e] - __uint_as_float(ah[e]));
+          ah[e] = __float_as_uint(av[e]) & 0xFFFFE000u;
+          al[e] = __float_as_uint(av[e] - __uint_as_float(ah[e]));
         }
-        mma_tf32_16x8x8(d, ah, bh[kk]);
-        mma_tf32_16x8x8(d, ah, bl[kk]);
-        mma_tf32_16x8x8(d, al, bh[kk]);
+        mma_tf32_16x8x8(dhh, ah, bh[kk]);
+        mma_tf32_16x8x8(dhl, ah, bl[kk]);
+        mma_tf32_16x8x8(dlh, al, bh[kk]);
       }
+      float d[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) d[e] = dhh[e] + (dhl[e] + dlh[e]);
       const int j = t * MASK_KT + mh * 16 + gid;
       if (j < NKV) {
         s_sc[(2 * tig) * nkv_max + j] = d[0] * p.scale;

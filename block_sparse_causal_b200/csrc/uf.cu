@@ -257,9 +257,17 @@ size_t attn_ws_cnt_bytes(int sms) { return (static_cast<size_t>(sms) * 4 + 255) 
 size_t attn_ws_bytes(int sms) {
   return attn_ws_cnt_bytes(sms) + 2 * static_cast<size_t>(sms) * uf::ATTN_PART_FLOATS * sizeof(float);
 }
-// The balanced schedule pays off when there are few items per SM (the last
-// round of items leaves SMs idle); with many items the plain one is as even.
+// The balanced schedule pays off when there are few items per SM and the
+// plain schedule's last round of items leaves SMs idle: ceil(items / sms)
+// rounds against items / sms on average, more than 10% apart.  With many
+// items, or a whole number of rounds, the plain schedule is as even and keeps
+// the items that run at the same time closer together (L2 reuse of K / V).
 constexpr long long kBalancedItemsPerSm = 8;
+bool balanced_pays(long long items, int sms) {
+  if (items >= kBalancedItemsPerSm * sms) return false;
+  const long long rounds = (items + sms - 1) / sms;
+  return rounds * sms * 10 > items * 11;
+}
 
 // uf_block_sparse_attn, its FP8-score variant (k8 != NULL) and the balanced
 // variant (ws != NULL: workspace of attn_ws_bytes(SM count) bytes).
@@ -350,7 +358,7 @@ int32_t attn_impl(const void *q, int32_t H, const uf_kv_cache *c, const int32_t 
   const cudaStream_t st = reinterpret_cast<cudaStream_t>(s);
   if (ws) {
     if (!aligned16(ws) || ws_bytes < attn_ws_bytes(sms)) return UF_EINVAL;
-    if (items < kBalancedItemsPerSm * sms) {
+    if (balanced_pays(items, sms)) {
       // balanced schedule: one thread block per SM, counters zeroed first
       p.ws_cnt = static_cast<int32_t *>(ws);
       p.ws_part = reinterpret_cast<float *>(static_cast<char *>(ws) + attn_ws_cnt_bytes(sms));

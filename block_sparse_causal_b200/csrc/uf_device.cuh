@@ -307,13 +307,6 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
-// fp32 -> tf32 (round to nearest, ties away), kept in a 32-bit register.
-__device__ __forceinline__ uint32_t to_tf32(float x) {
-  uint32_t r;
-  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-  return r;
-}
-
 // D += A B on the tensor core (warp-wide, m16n8k8, tf32 in, fp32 accumulate).
 __device__ __forceinline__ void mma_tf32_16x8x8(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
   asm volatile(

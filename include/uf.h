@@ -352,9 +352,9 @@ int32_t uf_block_sparse_attn(const void *q, int32_t H, const uf_kv_cache *c,
  *   workspace_bytes  its size.
  *   other arguments, outputs and errors as uf_block_sparse_attn.
  *
- * With many items per SM (at least 8) the plain schedule is already even
- * and is used unchanged (the workspace is not touched).  One memset and one
- * kernel launch.
+ * Where the plain schedule is already even -- at least 8 items per SM, or
+ * its last round of items within 10% of full -- it is used unchanged (the
+ * workspace is not touched).  One memset and one kernel launch.
  */
 int32_t uf_block_sparse_attn_balanced(const void *q, int32_t H, const uf_kv_cache *c, const int32_t *idx,
                                       const int32_t *cnt, int32_t k, float scale, void *o, float *lse,
