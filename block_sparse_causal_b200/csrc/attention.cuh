@@ -842,20 +842,21 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
         ++ks;
         store = s_last != 0;
         if (store) {
+          // every part, this block's included, in thread-block order from the
+          // workspace: the merged result does not depend on which part
+          // finished last
           float m_all = m_fin;
           for (int q = cur.part0; q < cur.part0 + cur.nparts; ++q)
             if (q != static_cast<int>(blockIdx.x))
               m_all = fmaxf(m_all, __ldcg(p.ws_part + static_cast<size_t>(part_slot(S, q, item)) * ATTN_PART_FLOATS +
                                           ATTN_PART_O + row));
-          const float f_own = ex2_approx(m_fin - m_all);
-          float l_all = l_tot * f_own;
+          float l_all = 0.f;
 #pragma unroll
-          for (int e = 0; e < 64; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f_own);
+          for (int e = 0; e < 64; ++e) o[e] = __float_as_uint(0.f);
           for (int q = cur.part0; q < cur.part0 + cur.nparts; ++q) {
-            if (q == static_cast<int>(blockIdx.x)) continue;
             const float *pq = p.ws_part + static_cast<size_t>(part_slot(S, q, item)) * ATTN_PART_FLOATS;
             const float fq = ex2_approx(__ldcg(pq + ATTN_PART_O + row) - m_all);
-            l_all += __ldcg(pq + ATTN_PART_O + 128 + row) * fq;
+            l_all = fmaf(__ldcg(pq + ATTN_PART_O + 128 + row), fq, l_all);
             const float4 *pq4 = reinterpret_cast<const float4 *>(pq) + x * 16 * 128 + row;
 #pragma unroll
             for (int c = 0; c < 16; ++c) {

@@ -164,3 +164,32 @@ def test_balanced_full_size_480p_dense(_lib, ws):
     torch.cuda.synchronize()
     items = sample_items(cfg, 24, seed=4)
     assert_attention_ok(cfg, o, lse, orc.attention(last["q"], items), "480p balanced")
+
+
+def test_balanced_call_replays_in_a_captured_graph(_lib, ws):
+    # the call's counter memset and kernel capture into a CUDA graph; each
+    # replay (after a new chunk's queries are copied in) equals the eager call
+    # bit for bit
+    cfg = CASES["gqa_b2"]
+    gpu, orc = GpuStream(cfg), OracleStream(cfg)
+    fill_window(cfg, 55, cfg.W, gpu, orc)
+    qs = [chunk_inputs(cfg, 56, t)["q"].cuda() for t in range(3)]
+    q_static = torch.empty_like(qs[0])
+    o = torch.empty(cfg.B, cfg.Lc, cfg.H, cfg.D, dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty(cfg.B, cfg.H, cfg.Lc, dtype=torch.float32, device="cuda")
+    scale = 1.0 / math.sqrt(cfg.D)
+    eager = []
+    for q in qs:
+        _lib.uf_block_sparse_attn_balanced(q, cfg.H, gpu.win.desc, None, None, 0, scale, o, lse, ws)
+        eager.append((o.clone(), lse.clone()))
+    q_static.copy_(qs[0])
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        _lib.uf_block_sparse_attn_balanced(q_static, cfg.H, gpu.win.desc, None, None, 0, scale, o, lse, ws)
+    for t, q in enumerate(qs):
+        q_static.copy_(q)
+        graph.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(o, eager[t][0]) and torch.equal(lse, eager[t][1]), t
+    del graph
