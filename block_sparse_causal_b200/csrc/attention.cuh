@@ -137,21 +137,26 @@ __device__ __forceinline__ void kv_block_coords(int j, int start, int W, int anc
   valid = (r == nb - 1) ? (Lc - (nb - 1) * blk) : blk;
 }
 
-// Which items a thread block takes.  Plain: items c, c + grid, c + 2 grid, ...
-// Balanced: the positions (item, kept block t) of all items, item-major, with
-// every item counted at its nominal length n_nom (dense: NKV, sparse: the row
-// stride k), are cut into g = min(gridDim.x, positions) contiguous ranges of
-// equal length (none empty), one per thread block c < g; an item that
-// straddles a range boundary is computed in parts by consecutive thread
-// blocks and merged (see the epilogue).  Every role of a thread block derives
-// the same sequence from this.
+// Which items a thread block takes, as a sequence v = 0 .. count - 1.
+// Plain: items c, c + grid, c + 2 grid, ...  Balanced: the same for the
+// `rounds` full rounds of items (items / grid of them), then the remaining
+// items are shared out by position: their positions (item, kept block t),
+// item-major, with every item counted at its nominal length n_nom (dense:
+// NKV, sparse: the row stride k), are cut into g = min(gridDim.x, positions)
+// contiguous ranges of equal length (none empty), one per thread block c < g;
+// an item that straddles a range boundary is computed in parts by consecutive
+// thread blocks and merged (see the epilogue).  Every role of a thread block
+// derives the same sequence from this.
 struct AttnSched {
   bool split;
   int n_nom;
-  int g;                      // thread blocks with a range
-  long long T;                // items * n_nom
-  long long lo, hi;           // this thread block's positions [lo, hi)
-  int begin, end, step;       // items visited: begin, begin + step, ... < end
+  int rounds;                 // items taken in the plain order
+  int base;                   // first shared-out item: rounds * gridDim.x (split)
+  int g;                      // thread blocks with a range of the shared-out items
+  long long T;                // positions of the shared-out items
+  long long lo, hi;           // this thread block's positions [lo, hi) among them
+  int rbegin, rend;           // shared-out items this thread block visits
+  int count;                  // items visited in all
 };
 
 __device__ __forceinline__ long long sched_start(long long T, int grid, int c) {
@@ -164,37 +169,43 @@ __device__ __forceinline__ int sched_owner(long long T, int grid, long long x) {
 
 __device__ __forceinline__ AttnSched attn_sched(const AttnParams &p, int NKV) {
   AttnSched s;
+  const int c = blockIdx.x, grid = gridDim.x;
   s.split = p.ws_part != nullptr && NKV > 0;
   s.n_nom = 0;
-  s.g = gridDim.x;
+  s.g = grid;
   s.T = s.lo = s.hi = 0;
+  s.rbegin = s.rend = 0;
   if (!s.split) {
-    s.begin = blockIdx.x;
-    s.end = p.items;
-    s.step = gridDim.x;
+    s.rounds = c < p.items ? (p.items - c + grid - 1) / grid : 0;
+    s.base = p.items;
+    s.count = s.rounds;
     return s;
   }
   s.n_nom = p.idx ? p.k : NKV;
-  s.T = static_cast<long long>(p.items) * s.n_nom;
-  s.g = static_cast<int>(s.T < gridDim.x ? s.T : gridDim.x);
-  if (static_cast<int>(blockIdx.x) >= s.g) {   // more thread blocks than positions: nothing to do
-    s.lo = s.hi = s.T;
-    s.begin = s.end = p.items;
-    s.step = 1;
-    return s;
+  s.rounds = p.items / grid;
+  s.base = s.rounds * grid;
+  s.T = static_cast<long long>(p.items - s.base) * s.n_nom;
+  s.g = static_cast<int>(s.T < grid ? s.T : grid);
+  if (c < s.g) {
+    s.lo = sched_start(s.T, s.g, c);
+    s.hi = sched_start(s.T, s.g, c + 1);
+    s.rbegin = s.base + static_cast<int>(s.lo / s.n_nom);
+    s.rend = s.base + static_cast<int>((s.hi - 1) / s.n_nom) + 1;
   }
-  s.lo = sched_start(s.T, s.g, blockIdx.x);
-  s.hi = sched_start(s.T, s.g, blockIdx.x + 1);
-  s.begin = static_cast<int>(s.lo / s.n_nom);
-  s.end = s.hi > s.lo ? static_cast<int>((s.hi - 1) / s.n_nom) + 1 : s.begin;
-  s.step = 1;
+  s.count = s.rounds + (s.rend - s.rbegin);
   return s;
 }
 
-// Workspace slot of the part that thread block c computes of item `item`: a
-// block's first item in slot 2c, its last (when both are split) in 2c + 1.
+// The v-th item of this thread block's sequence.
+__device__ __forceinline__ int sched_item(const AttnSched &s, int v) {
+  return v < s.rounds ? static_cast<int>(blockIdx.x) + v * static_cast<int>(gridDim.x) : s.rbegin + (v - s.rounds);
+}
+
+// Workspace slot of the part that thread block c computes of shared-out item
+// `item`: a block's first such item in slot 2c, its last (when both are split)
+// in 2c + 1.
 __device__ __forceinline__ int part_slot(const AttnSched &s, int c, int item) {
-  return 2 * c + (item == static_cast<int>(sched_start(s.T, s.g, c) / s.n_nom) ? 0 : 1);
+  return 2 * c + (item == s.base + static_cast<int>(sched_start(s.T, s.g, c) / s.n_nom) ? 0 : 1);
 }
 
 // One work item -- or this thread block's segment of it -- as every role of
@@ -230,8 +241,8 @@ __device__ __forceinline__ AttnItem attn_item(const AttnParams &p, const AttnSch
   it.nparts = 1;
   it.part0 = blockIdx.x;
   it.empty_out = it.n < 1;
-  if (s.split) {
-    const long long base = static_cast<long long>(item) * s.n_nom;
+  if (s.split && item >= s.base) {
+    const long long base = static_cast<long long>(item - s.base) * s.n_nom;
     if (it.n < 1) {
       // written once, by the thread block holding the item's first position
       it.empty_out = sched_owner(s.T, s.g, base) == static_cast<int>(blockIdx.x);
@@ -355,8 +366,8 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
         uint32_t phase = 0;
         int issued = 0;
         bool ok = true;
-        for (int item = S.begin; item < S.end && ok; item += S.step) {
-          const AttnItem it = attn_item(p, S, item, NKV, n_valid);
+        for (int v = 0; v < S.count && ok; ++v) {
+          const AttnItem it = attn_item(p, S, sched_item(S, v), NKV, n_valid);
           if (it.n < 1) continue;
           const int zc = it.b * p.G + it.g;
           for (int t = 0; t < it.n; ++t) {
@@ -421,14 +432,14 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
           tma_load_4d(sQ + L::Q_BYTES / 2, &tmQ, &bar_qfull, 64, a.h, a.i * BLK, a.b);
           ++q_loads;
         };
-        int item = S.begin;
+        int v = 0;
         AttnItem it;
-        for (; item < S.end; item += S.step) {
-          it = attn_item(p, S, item, NKV, n_valid);
+        for (; v < S.count; ++v) {
+          it = attn_item(p, S, sched_item(S, v), NKV, n_valid);
           if (it.n >= 1) break;
         }
-        if (item < S.end) request_q(it);
-        while (item < S.end && ok) {
+        if (v < S.count) request_q(it);
+        while (v < S.count && ok) {
           if (FP8) {
             // the softmax threads have written the item's e4m3 Q into tensor memory
             if (!(ok = wait_bounded(&bar_q, kq & 1, abort_flag, p.wait_limit, p.err))) break;
@@ -448,7 +459,7 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
             if (!(ok = wait_bounded(&bar_qcp, kq & 1, abort_flag, p.wait_limit, p.err))) break;
           }
           tc_fence_after();
-          int item_next = S.end;
+          int v_next = S.count;
           AttnItem nxt;
           const int t_request = it.n > 1 ? 1 : 0;
           for (int t = 0; t < it.n; ++t) {
@@ -484,11 +495,11 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
               // with the item's first products on their way: the next live
               // item's Q, once the previous item's output stores have read
               // the staging tile
-              for (item_next = item + S.step; item_next < S.end; item_next += S.step) {
-                nxt = attn_item(p, S, item_next, NKV, n_valid);
+              for (v_next = v + 1; v_next < S.count; ++v_next) {
+                nxt = attn_item(p, S, sched_item(S, v_next), NKV, n_valid);
                 if (nxt.n >= 1) break;
               }
-              if (item_next < S.end) {
+              if (v_next < S.count) {
                 if (kq > 0 && !(ok = wait_bounded(&bar_ostore, (kq - 1) & 1, abort_flag, p.wait_limit, p.err))) break;
                 request_q(nxt);
               }
@@ -499,7 +510,7 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
           mma_commit(&bar_qtfree);
           g0 += it.n;
           ++kq;
-          item = item_next;
+          v = v_next;
           it = nxt;
         }
         // every MMA issued by this thread has completed once bar_fin flips, and
@@ -537,8 +548,8 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
           return true;
         };
         AttnItem prev;
-        for (int item = S.begin; item < S.end && ok; item += S.step) {
-          const AttnItem it = attn_item(p, S, item, NKV, n_valid);
+        for (int v = 0; v < S.count && ok; ++v) {
+          const AttnItem it = attn_item(p, S, sched_item(S, v), NKV, n_valid);
           if (it.n < 1) continue;
           // the previous item's output leaves (and its epilogue has read O)
           if (kq > 0 && !(ok = store_output(prev, kq - 1))) break;
@@ -599,12 +610,12 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
     // first item at or after `from` (in this block's sequence) with blocks to
     // compute; the empty ones on the way are written here
     auto next_live = [&](int from, AttnItem &out) -> int {
-      for (int j = from; j < S.end; j += S.step) {
-        out = attn_item(p, S, j, NKV, n_valid);
+      for (int j = from; j < S.count; ++j) {
+        out = attn_item(p, S, sched_item(S, j), NKV, n_valid);
         if (out.n >= 1) return j;
         if (out.empty_out) write_empty(out);
       }
-      return S.end;
+      return S.count;
     };
     // Q of live item number kq -> tensor memory, once it has landed and the
     // previous item's QK products have completed: this warpgroup copies
@@ -645,11 +656,12 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
     };
 
     AttnItem cur;
-    int item = next_live(S.begin, cur);
-    bool ok = item >= S.end || !FP8 || load_q(0);
+    int v = next_live(0, cur);
+    bool ok = v >= S.count || !FP8 || load_q(0);
     int ks = 0;           // parts of split items written so far (parity of bar_pw / bar_tk)
     int kq = 0, g0 = 0;   // live items and kept blocks of this thread block so far
-    while (item < S.end && ok) {
+    while (v < S.count && ok) {
+      const int item = sched_item(S, v);
       const int n = cur.n;
       float m_run = -INFINITY;   // reference max this warpgroup last saw
       float l_run = 0.f;         // this warpgroup's partial row sum, relative to m_run
@@ -783,8 +795,8 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
       // the next live item's Q goes into tensor memory now, so that its first
       // QK products run during this item's epilogue
       AttnItem nxt;
-      const int item_next = next_live(item + S.step, nxt);
-      if (FP8 && item_next < S.end && !(ok = load_q(kq + 1))) break;
+      const int v_next = next_live(v + 1, nxt);
+      if (FP8 && v_next < S.count && !(ok = load_q(kq + 1))) break;
       // ---------------------------------------------------------- epilogue --
       // every PV of the item has completed once its last one has (one issuing
       // thread, completions in order)
@@ -874,7 +886,7 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
       if (threadIdx.x == 128) s_store[kq & 1] = store;   // read by the PV issuer after bar_st
       // (bf16 path: the QK issuer's copy of the next item's Q out of the staging
       // tile has completed)
-      if (!FP8 && item_next < S.end && !(ok = wwait(&bar_qcp, (kq + 1) & 1))) break;
+      if (!FP8 && v_next < S.count && !(ok = wwait(&bar_qcp, (kq + 1) & 1))) break;
       // this warpgroup's 64-column half of the bf16 row -> the staging tile
       // (the next item's Q has left it), 128-byte swizzled like a TMA tile:
       // 16-byte chunk c of row r at chunk c ^ (r mod 8)
@@ -900,7 +912,7 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
         p.lse[(static_cast<size_t>(cur.b) * p.H + cur.h) * p.Lc + q_tok] = (m_fin + log2f(l_tot)) * 0.69314718055994531f;
       g0 += n;
       ++kq;
-      item = item_next;
+      v = v_next;
       cur = nxt;
     }
   }

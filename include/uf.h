@@ -332,11 +332,12 @@ int32_t uf_block_sparse_attn(const void *q, int32_t H, const uf_kv_cache *c,
 
 /*
  * Balanced variant of uf_block_sparse_attn, for workloads with few work items
- * per SM (grouped-query decoder steps, small chunks): the positions (item,
- * kept block) of all (b, h, q-block) items, every item counted at its nominal
- * length (dense: every block of the window; sparse: the row stride k), are
- * cut into one contiguous range of equal length per SM, so every SM computes
- * the same number of kept blocks.  An item whose blocks fall into several
+ * per SM (grouped-query decoder steps, small chunks): the full rounds of
+ * (b, h, q-block) items go to the SMs whole, and the positions (item, kept
+ * block) of the remaining items, every item counted at its nominal length
+ * (dense: every block of the window; sparse: the row stride k), are cut into
+ * one contiguous range of equal length per SM, so every SM computes the same
+ * number of kept blocks.  An item whose blocks fall into several
  * ranges is computed in parts; each part writes its unnormalised O, row max
  * and row sum to the workspace, and the part that finishes last merges them
  * (log-sum-exp, in fp32) and writes O and LSE.  No thread block waits for
