@@ -24,8 +24,9 @@
 //      registers as B fragments);
 //   3. select: one warp per q-block row forces the diagonal (or the local
 //      band around it), finds the need-th largest of the other scores (need =
-//      k minus the forced blocks) by a 32-step bitwise search over
-//      order-preserving integer keys, takes every key above it plus the
+//      k minus the forced blocks) by a bitwise search over order-preserving
+//      integer keys (at most 32 steps; it stops as soon as exactly need keys
+//      lie at or above the candidate), takes every key above it plus the
 //      lowest-index keys equal to it, and writes the kept ids in ascending
 //      order.
 #pragma once
@@ -284,14 +285,20 @@ __global__ void __launch_bounds__(MASK_THREADS, 2) block_mask_kernel(const MaskP
     uint32_t T = 0xFFFFFFFFu;              // threshold key (need == 0: nothing passes)
     int take_eq = 0;
     if (need > 0) {
-      // the need-th largest key: largest T with #(key >= T) >= need, bit by bit
+      // the need-th largest key: largest T with #(key >= T) >= need, bit by
+      // bit; once exactly need keys are >= T the kept set is fixed (the
+      // search could only raise T among keys that are all kept), so it stops
       T = 0u;
       for (int bit = 31; bit >= 0; --bit) {
         const uint32_t cand = T | (1u << bit);
         int c = 0;
 #pragma unroll
         for (int m = 0; m < MAXPER; ++m) c += key[m] >= cand;
-        if (__reduce_add_sync(0xffffffffu, c) >= need) T = cand;
+        const int tot = __reduce_add_sync(0xffffffffu, c);
+        if (tot >= need) {
+          T = cand;
+          if (tot == need) break;
+        }
       }
       int gt = 0;
 #pragma unroll
