@@ -138,7 +138,7 @@ class ClockSampler:
 
     FIELDS = ("index,pci.bus_id,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap,enforced.power.limit")
 
     def __init__(self, device=None):
         self.pci = ""
@@ -169,33 +169,50 @@ class ClockSampler:
             self.proc.wait(timeout=5)
         except subprocess.TimeoutExpired:
             self.proc.kill()
-        rows = []
-        for line in open(self.path):
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 10:
-                continue
-            if self.pci and not parts[1].lower().endswith(self.pci):
-                continue
-            rows.append(parts)
+        with open(self.path) as f:
+            lines = f.readlines()
         os.unlink(self.path)
-        if not rows:
-            return None
+        return summarise_clock_rows(lines, self.pci)
 
-        def num(x):
-            try:
-                return float(x)
-            except ValueError:
-                return None
-        sm = [num(r[2]) for r in rows if num(r[2]) is not None]
-        reasons = set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for r in rows:
-            for n, v in zip(names, r[6:10]):
-                if v.lower().startswith("active"):
-                    reasons.add(n)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": num(rows[0][3]),
-                "power_w_max": max((num(r[4]) or 0.0) for r in rows), "samples": len(rows),
-                "reasons": sorted(reasons)}
+
+def summarise_clock_rows(lines, pci=""):
+    """Summary of nvidia-smi rows in ClockSampler.FIELDS order (rows of other
+    GPUs, when pci is given, and malformed rows are skipped); None if none."""
+    rows = []
+    for line in lines:
+        parts = [p.strip() for p in line.split(",")]
+        if len(parts) < 11:
+            continue
+        if pci and not parts[1].lower().endswith(pci):
+            continue
+        rows.append(parts)
+    if not rows:
+        return None
+
+    def num(x):
+        try:
+            return float(x)
+        except ValueError:
+            return None
+    sm = [num(r[2]) for r in rows if num(r[2]) is not None]
+    reasons = set()
+    names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    for r in rows:
+        for n, v in zip(names, r[6:10]):
+            if v.lower().startswith("active"):
+                reasons.add(n)
+    return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": num(rows[0][3]),
+            "power_w_max": max((num(r[4]) or 0.0) for r in rows), "power_limit_w": num(rows[0][10]),
+            "samples": len(rows), "reasons": sorted(reasons)}
+
+
+def clock_normalised(tflops, clocks):
+    """tflops scaled to the maximum SM clock from the clock the kernel ran at
+    (its in-kernel effective clock, else the sampled median); None if unknown."""
+    if not clocks or not clocks.get("sm_max_mhz"):
+        return None
+    mhz = clocks.get("attn_sm_mhz") or clocks.get("sm_mhz")
+    return tflops * clocks["sm_max_mhz"] / mhz if mhz else None
 
 
 # --------------------------------------------------------------- GPU arm ----
@@ -293,17 +310,27 @@ def run_ours(args, cfg, rank, world, device, do_e2e=True):
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
+    # the attention kernel's own clock: its thread blocks add their SM cycles
+    # and global-timer nanoseconds here (atomic adds when each block ends)
+    clk = torch.zeros(2, dtype=torch.int64, device=device)
     sampler = ClockSampler(device)
     sampler.start()
     barrier(world)
     torch.cuda.synchronize()
+    uf.uf_set_clock_counters(clk)
     t_start.record(stream)
     for s in range(args.steps):
         step(args.warmup + s, dev_chunks[cfg.W + (args.warmup + s) % n_distinct], evs[s])
     t_end.record(stream)
     torch.cuda.synchronize()
+    uf.uf_set_clock_counters(None)
     barrier(world)
     clocks = sampler.stop()
+    cycles, ns = (int(v) for v in clk.tolist())
+    attn_mhz = cycles / ns * 1e3 if ns > 0 else None
+    if clocks is None:
+        clocks = {}
+    clocks["attn_sm_mhz"] = attn_mhz
     elapsed_ms = t_start.elapsed_time(t_end)
     per = {"append": 0.0, "mask": 0.0, "attn": 0.0}
     for ev in evs:
@@ -390,10 +417,10 @@ def run_ours(args, cfg, rank, world, device, do_e2e=True):
             "kernel": "uf::attn_kernel<%d, %s>" % (cfg.blk, "true" if args.fp8 else "false"),
             "peak_source": f"{peaks_src} bf16 dense burst (cuBLAS 8192^3)"
                            + (" x 4/3: QK at the nominal e4m3/bf16 ratio of 2" if args.fp8 else ""),
-            # the rate at the maximum SM clock: achieved x (max SM MHz / median SM MHz
-            # under load); separates kernel quality from the power cap's clock
-            "clock_normalised_tflops": (attn_tflops * clocks["sm_max_mhz"] / clocks["sm_mhz"]
-                                        if clocks and clocks.get("sm_mhz") and clocks.get("sm_max_mhz") else None),
+            # the rate at the maximum SM clock: achieved x (max SM MHz / the SM clock
+            # the attention kernel ran at, from its own cycle and timer counts);
+            # separates kernel quality from the power cap's clock
+            "clock_normalised_tflops": clock_normalised(attn_tflops, clocks),
         },
         "e2e": None if e2e is None else {
             "value": job_flops_per_step / (e2e[0] * 1e-3) / 1e12, "unit": "TFLOP/s",

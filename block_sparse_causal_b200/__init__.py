@@ -11,7 +11,7 @@ from ._uf import (UF_APPEND_ANCHOR, UF_APPEND_REPLACE_NEWEST, UF_EBOUNDS, UF_ECU
                   uf_block_sparse_attn_fp8k, uf_check_error,
                   uf_debug_wait_timeout, uf_get_error, uf_kv_append, uf_kv_append_fp8k, uf_kv_append_rope,
                   uf_kv_append_tiled, uf_kv_cache_bytes, uf_kv_cache_init, uf_kv_cache_set_error_word, uf_kv_reset,
-                  uf_rope, uf_set_wait_limit, uf_source_hash, uf_tile_tokens, uf_version)
+                  uf_rope, uf_set_clock_counters, uf_set_wait_limit, uf_source_hash, uf_tile_tokens, uf_version)
 from .pipeline import ChunkPipeline
 from .window import KVWindow
 
@@ -23,5 +23,5 @@ __all__ = [
     "uf_block_sparse_attn_fp8k", "uf_check_error",
     "uf_debug_wait_timeout", "uf_get_error", "uf_kv_append", "uf_kv_append_fp8k", "uf_kv_append_rope",
     "uf_kv_append_tiled", "uf_kv_cache_bytes", "uf_kv_cache_init", "uf_kv_cache_set_error_word", "uf_kv_reset",
-    "uf_rope", "uf_set_wait_limit", "uf_source_hash", "uf_tile_tokens", "uf_version", "KVWindow", "ChunkPipeline",
+    "uf_rope", "uf_set_clock_counters", "uf_set_wait_limit", "uf_source_hash", "uf_tile_tokens", "uf_version", "KVWindow", "ChunkPipeline",
 ]

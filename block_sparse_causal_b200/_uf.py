@@ -75,6 +75,7 @@ def _load() -> ctypes.CDLL:
         "uf_get_error": ([ctypes.POINTER(i32), i32], i32),
         "uf_last_cuda_error": ([], ctypes.c_char_p),
         "uf_set_wait_limit": ([ctypes.c_int64], i32),
+        "uf_set_clock_counters": ([vp], i32),
         "uf_debug_wait_timeout": ([ctypes.c_int64, vp], i32),
     }
     for name, (args, res) in sig.items():
@@ -239,6 +240,14 @@ def uf_get_error(clear: bool = True) -> int:
 
 def uf_set_wait_limit(cycles: int) -> None:
     _check(lib.uf_set_wait_limit(cycles), "uf_set_wait_limit")
+
+
+def uf_set_clock_counters(counters) -> None:
+    """counters: a device int64 tensor of 2 zeroed elements (or None to stop):
+    attention launches add their SM cycles and nanoseconds to it."""
+    if counters is not None and (counters.numel() < 2 or counters.element_size() != 8 or not counters.is_cuda):
+        raise ValueError("counters must be a device tensor of at least 2 eight-byte elements")
+    _check(lib.uf_set_clock_counters(_ptr(counters)), "uf_set_clock_counters")
 
 
 def uf_debug_wait_timeout(cycles: int, stream=None) -> None:

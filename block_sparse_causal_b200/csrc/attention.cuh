@@ -93,6 +93,9 @@ struct AttnParams {
   // balanced schedule (NULL: thread block c takes items c, c + grid, ...):
   int32_t *ws_cnt;           // [grid] arrival counters of split items, zero at launch
   float *ws_part;            // [2 * grid][ATTN_PART_FLOATS] partial results
+  // optional [2]: every thread block adds its SM clock cycles and its global
+  // timer nanoseconds from start to end (the kernel's effective SM clock)
+  unsigned long long *clk;
 };
 
 // One part of a split item: its unnormalised O (fp32, 128 rows x 128
@@ -278,6 +281,13 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
                 const AttnParams p) {
   using L = AttnSmem<BLK>;
+  // start of this thread block, when the launch records its clock
+  __shared__ long long s_clk0;
+  __shared__ unsigned long long s_ns0;
+  if (p.clk && threadIdx.x == 0) {
+    s_clk0 = clock64();
+    s_ns0 = global_ns();
+  }
   extern __shared__ uint8_t smem_raw[];
   uint8_t *sQ = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *sK = sQ + L::Q_BYTES;
@@ -922,6 +932,10 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tb, 512);
+  }
+  if (p.clk && threadIdx.x == 0) {
+    atomicAdd(p.clk, static_cast<unsigned long long>(clock64() - s_clk0));
+    atomicAdd(p.clk + 1, global_ns() - s_ns0);
   }
 }
 

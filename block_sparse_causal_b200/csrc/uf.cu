@@ -19,11 +19,13 @@
 
 namespace {
 
-constexpr int32_t UF_VERSION = 200;   // 0.2.0
+constexpr int32_t UF_VERSION = 300;   // 0.3.0
 constexpr int32_t kMaxW = 64;
 constexpr int32_t kMaxMaskNKV = 1024; // window blocks: 32 selection keys per lane
 constexpr int32_t kMaxDevices = 64;
 std::atomic<long long> g_wait_limit{1LL << 31};
+// attention launches add their cycles / nanoseconds here when set
+std::atomic<unsigned long long *> g_clock_counters{nullptr};
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -350,6 +352,7 @@ int32_t attn_impl(const void *q, int32_t H, const uf_kv_cache *c, const int32_t 
   p.err = c->err;
   p.ws_cnt = nullptr;
   p.ws_part = nullptr;
+  p.clk = g_clock_counters.load();
   int sms = 0;
   const int32_t se = sm_count(&sms);
   if (se != UF_OK) return se;
@@ -658,6 +661,12 @@ const char *uf_last_cuda_error(void) { return t_last_cuda_error; }
 int32_t uf_set_wait_limit(int64_t cycles) {
   if (cycles < 1000) return UF_EINVAL;
   g_wait_limit.store(cycles);
+  return UF_OK;
+}
+
+int32_t uf_set_clock_counters(uint64_t *dev_counters) {
+  if (reinterpret_cast<uintptr_t>(dev_counters) & 7u) return UF_EINVAL;
+  g_clock_counters.store(reinterpret_cast<unsigned long long *>(dev_counters));
   return UF_OK;
 }
 

@@ -90,6 +90,13 @@ __device__ __forceinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, vol
   }
 }
 
+// Nanoseconds of the global timer (one clock for every SM, unlike clock64).
+__device__ __forceinline__ unsigned long long global_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
 // ------------------------------------------------------------ window -------
 // Window state (meta): {start, n_valid, counter, anchor}.  Without an anchor
 // the W slots form one ring and logical chunk c (0 = oldest) lives in slot

@@ -474,6 +474,22 @@ const char *uf_last_cuda_error(void);
 int32_t uf_set_wait_limit(int64_t cycles);
 
 /*
+ * Measurement hook (the pages have no counterpart: it serves the benchmark's
+ * clock record).  dev_counters: NULL (off, the default) or a device uint64[2],
+ * 8-byte aligned, owned by the caller, who zeroes it.  While set, every thread
+ * block of every attention launch made after the call adds, when it ends, the
+ * SM clock cycles (clock64) and the global-timer nanoseconds that passed since
+ * it started to dev_counters[0] and dev_counters[1] (atomic adds).  The ratio
+ * cycles / nanoseconds is the attention kernel's effective SM clock in GHz,
+ * averaged over its thread blocks: the clock it really ran at, which a sampled
+ * clock reading taken every few hundred milliseconds does not show.  The
+ * buffer must stay valid until every such launch has completed; set NULL to
+ * stop.  Host only; one setting for all devices and threads.  UF_EINVAL on a
+ * misaligned pointer.
+ */
+int32_t uf_set_clock_counters(uint64_t *dev_counters);
+
+/*
  * Self-test of the bounded-wait path: launch one thread that waits on a
  * pipeline barrier that nothing will ever complete, with a bound of `cycles`.
  * The kernel records UF_ETIMEOUT and returns; it never hangs.  For tests.

@@ -7,6 +7,7 @@ import re
 import subprocess
 
 import pytest
+import torch
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "uf.h")
@@ -262,3 +263,15 @@ def test_error_word_calls_validate_on_host(uf):
     assert c.err == 0xB00004
     uf.uf_kv_cache_set_error_word(c, None)
     assert c.err is None
+
+
+def test_clock_counters_validate_on_host(uf):
+    # a misaligned counter pair is refused; NULL (off) is always accepted
+    lib = uf._uf.lib
+    assert lib.uf_set_clock_counters(0xB00004) == uf.UF_EINVAL
+    try:
+        assert lib.uf_set_clock_counters(0xB00008) == uf.UF_OK
+    finally:
+        assert lib.uf_set_clock_counters(None) == uf.UF_OK
+    with pytest.raises(ValueError):
+        uf.uf_set_clock_counters(torch.zeros(2, dtype=torch.int64))      # host memory

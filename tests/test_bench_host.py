@@ -54,6 +54,29 @@ def test_traffic_is_dropped_when_the_kernel_changes(tmp_path, monkeypatch):
     assert bench.attn_traffic_per_launch("1k_sr") is None
 
 
+def test_clock_rows_summary():
+    row = "0, 00000000:1B:00.0, {sm}, 1965, {w}, 0x4, Not Active, Not Active, Not Active, {cap}, 1000.00\n"
+    lines = [row.format(sm=1500, w=700.5, cap="Active"), row.format(sm=1550, w=760.2, cap="Not Active"),
+             row.format(sm=1600, w=650.0, cap="Not Active"),
+             "1, 00000000:2A:00.0, 900, 1965, 100.0, 0x0, Not Active, Active, Not Active, Not Active, 1000.00\n",
+             "garbage\n"]
+    c = bench.summarise_clock_rows(lines, pci="1b:00.0")
+    assert c["sm_mhz"] == 1550 and c["sm_max_mhz"] == 1965 and c["samples"] == 3
+    assert c["power_w_max"] == 760.2 and c["power_limit_w"] == 1000.0
+    assert c["reasons"] == ["sw_power_cap"]                 # the other GPU's thermal slowdown is not ours
+    assert bench.summarise_clock_rows(["garbage\n"]) is None
+    na = bench.summarise_clock_rows([row.format(sm=1965, w=300, cap="Not Active").replace("1000.00", "[N/A]")])
+    assert na["power_limit_w"] is None and na["reasons"] == []
+
+
+def test_clock_normalisation_prefers_the_kernels_own_clock():
+    assert bench.clock_normalised(1000.0, None) is None
+    assert bench.clock_normalised(1000.0, {"sm_max_mhz": 1965.0}) is None
+    assert bench.clock_normalised(1000.0, {"sm_max_mhz": 1965.0, "sm_mhz": 1965.0}) == 1000.0
+    c = {"sm_max_mhz": 1965.0, "sm_mhz": 1965.0, "attn_sm_mhz": 1572.0}
+    assert math.isclose(bench.clock_normalised(1000.0, c), 1000.0 * 1965.0 / 1572.0)
+
+
 def test_reference_arm_json_line():
     env = dict(os.environ, OMP_NUM_THREADS="2", OPENBLAS_NUM_THREADS="2")
     res = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--config", "tiny",

@@ -40,5 +40,8 @@ def test_bench_prints_the_contract_line():
     for key in ("sm_mhz", "sm_max_mhz", "reasons"):
         assert key in d["clocks"], key
     assert "clock_normalised_tflops" in r
+    # the attention kernel's own clock, from its cycle and timer counts
+    assert 300.0 < d["clocks"]["attn_sm_mhz"] <= d["clocks"]["sm_max_mhz"] * 1.02
+    assert r["clock_normalised_tflops"] >= r["achieved"] * 0.98
     other = d["other_workloads"]["gqa_decoder"]
     assert other["ms_per_step"] > 0 and other["value"] > 0 and 0 < other["attn_frac"] < 1.5
