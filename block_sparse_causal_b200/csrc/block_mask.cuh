@@ -7,21 +7,20 @@
 //
 // One thread block per (TQ = 8 consecutive q-blocks, query head h, batch b),
 // 256 threads (one warp per q-block), two thread blocks per SM:
-//   0. the pooled K (written by the append call, one fp32 row per window
-//      block) streams through a ring of 4 tiles of 32 rows: stage s holds
-//      tiles s, s + 4, ... and belongs to warps 2s and 2s + 1, which fill it
-//      (one bulk copy per row, into rows padded to 132 floats) and consume it;
-//      the first four tiles are requested at entry, so they arrive while Q is
-//      pooled;
 //   1. pool: warp w sums q-block i0 + w over its tokens in fp32, each lane 8
 //      channels of every other token with 16-byte loads, 16 in flight;
 //   2. score: on the tensor core, m16n8k8 tf32 MMAs with fp32 accuracy by a
 //      hi / lo split of both operands (hi = the top 19 bits of the fp32
 //      value, lo = the exact remainder, which the MMA reads to 11 bits:
 //      products within 2^-21 relative), as hi.hi + hi.lo + lo.hi in three
-//      accumulators so the MMA chains overlap; each warp takes one 16-row
-//      half of its stage's tiles against the 8 pooled queries (held in
-//      registers as B fragments);
+//      accumulators so the MMA chains overlap.  The pooled K (written by the
+//      append call, one fp32 row per window block) is read from L2 straight
+//      into A fragments: each warp takes 16-row slices of the window in turn,
+//      each lane loading 4 consecutive channels of its two rows per 16-byte
+//      load.  The MMA's k index runs over the channels in that load order
+//      (any order of the channels gives the same dot product), and the 8
+//      pooled queries' B fragments, split once, follow the same order from
+//      shared memory;
 //   3. select: one warp per q-block row forces the diagonal (or the local
 //      band around it), finds the need-th largest of the other scores (need =
 //      k minus the forced blocks) by a bitwise search over order-preserving
@@ -37,15 +36,13 @@ namespace uf {
 
 constexpr int MASK_TQ = 8;        // q-blocks per thread block (= warps)
 constexpr int MASK_THREADS = 32 * MASK_TQ;
-constexpr int MASK_KT = 32;       // pooled-K rows per tile
-constexpr int MASK_KSTAGE = 4;    // pooled-K tiles in flight (stage s: warps 2s, 2s + 1)
-constexpr int MASK_KSTRIDE = 132; // floats per pooled-K row in shared memory (conflict-free A fragments)
-static_assert(2 * MASK_KSTAGE == MASK_TQ, "each warp pair owns one stage");
 constexpr int MASK_QLOADS = 16;   // 16-byte Q loads in flight per lane
 
-// Dynamic shared memory of the mask kernel for a window of nkv_max blocks.
+// Dynamic shared memory of the mask kernel for a window of nkv_max blocks:
+// pooled queries, their split B fragments (16 k-steps x 32 lanes x 16 bytes)
+// and the scores.
 __host__ __device__ constexpr int mask_smem_bytes(int nkv_max) {
-  return (MASK_KSTAGE * MASK_KT * MASK_KSTRIDE + MASK_TQ * 128 + MASK_TQ * nkv_max) * 4;
+  return (MASK_TQ * 128 + 16 * 32 * 4 + MASK_TQ * nkv_max) * 4;
 }
 
 struct MaskParams {
@@ -81,14 +78,11 @@ __device__ __forceinline__ int warp_excl_scan(int v, int lane) {
 template <int BLK, int MAXPER>
 __global__ void __launch_bounds__(MASK_THREADS, 2) block_mask_kernel(const MaskParams p) {
   constexpr int D = 128;
-  constexpr long long kWait = 1LL << 31;
   extern __shared__ __align__(128) float mraw[];
-  float *s_kt = mraw;                                   // [KSTAGE][KT][KSTRIDE]
-  float *s_qpool = s_kt + MASK_KSTAGE * MASK_KT * MASK_KSTRIDE;   // [TQ][D]
-  float *s_sc = s_qpool + MASK_TQ * D;                  // [TQ][W*nb]
+  float *s_qpool = mraw;                                          // [TQ][D]
+  uint4 *s_bfrag = reinterpret_cast<uint4 *>(s_qpool + MASK_TQ * D);   // [D / 8][32 lanes]
+  float *s_sc = reinterpret_cast<float *>(s_bfrag + (D / 8) * 32);   // [TQ][W*nb]
   __shared__ int32_t s_meta[3];
-  __shared__ uint64_t bar_k[MASK_KSTAGE];
-  __shared__ int32_t s_abort;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int h = blockIdx.y, b = blockIdx.z;
@@ -107,9 +101,6 @@ __global__ void __launch_bounds__(MASK_THREADS, 2) block_mask_kernel(const MaskP
     s_meta[0] = start;
     s_meta[1] = n;
     s_meta[2] = anc;
-    for (int q = 0; q < MASK_KSTAGE; ++q) mbar_init(&bar_k[q], 1);
-    s_abort = 0;
-    fence_mbar_init();
   }
   __syncthreads();
   const int start = s_meta[0], n_valid = s_meta[1], anchor = s_meta[2];
@@ -122,29 +113,6 @@ __global__ void __launch_bounds__(MASK_THREADS, 2) block_mask_kernel(const MaskP
     }
     if (tid < tq_count) p.cnt[(static_cast<size_t>(b) * p.H + h) * p.nb + i0 + tid] = 0;
     return;
-  }
-
-  // ---- 0. pooled-K tiles: one 512-byte bulk copy per window block ----------
-  const float *kp_head = p.kpool + (static_cast<size_t>(b) * p.G + g) * nkv_max * D;
-  const int ntiles = (NKV + MASK_KT - 1) / MASK_KT;
-  const int pair = warp >> 1;            // this warp's stage; tiles pair, pair + KSTAGE, ...
-  auto issue_tile = [&](int t) {          // all lanes of warp 2 * (t mod KSTAGE)
-    const int st = t % MASK_KSTAGE, j0 = t * MASK_KT;
-    const int rows = min(MASK_KT, NKV - j0);
-    if (lane == 0) mbar_arrive_expect_tx(&bar_k[st], static_cast<uint32_t>(rows) * D * 4);
-    __syncwarp();
-    if (lane < rows) {
-      const int j = j0 + lane;
-      const int c = j / p.nb, rr = j - c * p.nb;
-      const int slot = window_slot(c, start, p.W, anchor);
-      bulk_load(s_kt + (st * MASK_KT + lane) * MASK_KSTRIDE, kp_head + (static_cast<size_t>(slot) * p.nb + rr) * D,
-                D * 4, &bar_k[st]);
-    }
-  };
-  int last_issued = -1;                   // (even warps) last tile issued into this warp pair's stage
-  if ((warp & 1) == 0 && pair < ntiles) {
-    issue_tile(pair);
-    last_issued = pair;
   }
 
   // ---- 1. pool the query blocks: warp w takes q-block i0 + w ----------------
@@ -188,74 +156,78 @@ __global__ void __launch_bounds__(MASK_THREADS, 2) block_mask_kernel(const MaskP
   __syncthreads();                                      // s_qpool complete
 
   // ---- 2. pooled scores against every block of the window -----------------
-  // D[16 kv rows x 8 queries] += A[rows x 8 channels] B[8 channels x queries]
-  // over 16 channel steps, each operand split as x = hi + lo (tf32 parts).
-  // Fragments (m16n8k8, gid = lane / 4, tig = lane % 4): A rows gid, gid + 8
-  // and channels tig, tig + 4; B query gid, channels tig, tig + 4; D rows
-  // gid, gid + 8 and queries 2 tig, 2 tig + 1.
+  // D[16 kv rows x 8 queries] += A[rows x 8 k] B[8 k x queries] over 16 k-steps,
+  // each operand split as x = hi + lo (tf32 parts).  Fragments (m16n8k8, gid =
+  // lane / 4, tig = lane % 4): A rows gid, gid + 8 at k = tig, tig + 4; B
+  // query gid at k = tig, tig + 4; D rows gid, gid + 8 and queries 2 tig,
+  // 2 tig + 1.  Channel of (k-step kk, k = tig + 4 s):
+  //   16 (kk / 2) + 4 tig + 2 (kk mod 2) + s,
+  // so that one 16-byte load of channels 16 m + 4 tig .. + 3 holds the A
+  // values of k-steps 2 m and 2 m + 1.
   const int gid = lane >> 2, tig = lane & 3;
-  uint32_t bh[D / 8][2], bl[D / 8][2];
+  for (int e = tid; e < (D / 8) * 32; e += MASK_THREADS) {
+    const int kk = e >> 5, ln = e & 31, qg = ln >> 2, qt = ln & 3;
+    const int c0 = 16 * (kk >> 1) + 4 * qt + 2 * (kk & 1);
+    const float v0 = s_qpool[qg * D + c0], v1 = s_qpool[qg * D + c0 + 1];
+    const uint32_t h0 = __float_as_uint(v0) & 0xFFFFE000u, h1 = __float_as_uint(v1) & 0xFFFFE000u;
+    s_bfrag[e] = make_uint4(h0, h1, __float_as_uint(v0 - __uint_as_float(h0)),
+                            __float_as_uint(v1 - __uint_as_float(h1)));
+  }
+  __syncthreads();                                      // B fragments complete
+
+  const float *kp_head = p.kpool + (static_cast<size_t>(b) * p.G + g) * nkv_max * D;
+  // logical window block j -> its pooled-K row (channels 4 tig .. of each 16)
+  auto krow = [&](int j) -> const float4 * {
+    const int c = j / p.nb, rr = j - c * p.nb;
+    const int slot = window_slot(c, start, p.W, anchor);
+    return reinterpret_cast<const float4 *>(kp_head + (static_cast<size_t>(slot) * p.nb + rr) * D) + tig;
+  };
+  const int nslices = (NKV + 15) / 16;
+#pragma unroll 1
+  for (int sl = warp; sl < nslices; sl += MASK_TQ) {
+    const int j = sl * 16 + gid;
+    float4 r0[8], r1[8];
+    {
+      const bool ok0 = j < NKV, ok1 = j + 8 < NKV;
+      const float4 *k0 = ok0 ? krow(j) : nullptr;
+      const float4 *k1 = ok1 ? krow(j + 8) : nullptr;
 #pragma unroll
-  for (int kk = 0; kk < D / 8; ++kk)
-#pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      const float v = s_qpool[gid * D + kk * 8 + tig + 4 * e];
-      bh[kk][e] = __float_as_uint(v) & 0xFFFFE000u;
-      bl[kk][e] = __float_as_uint(v - __uint_as_float(bh[kk][e]));
-    }
-  const int mh = warp & 1;                // this warp's 16-row half of each tile
-  for (int t = pair; t < ntiles; t += MASK_KSTAGE) {
-    // both warps of the pair run the same iterations (the named barrier below
-    // needs both); after an abort the waits return at once and nothing is issued
-    if (wait_bounded(&bar_k[pair], (t / MASK_KSTAGE) & 1, &s_abort, kWait, p.err)) {
-      const float *kt = s_kt + (pair * MASK_KT + mh * 16) * MASK_KSTRIDE;
-      float dhh[4] = {0.f, 0.f, 0.f, 0.f}, dhl[4] = {0.f, 0.f, 0.f, 0.f}, dlh[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int kk = 0; kk < D / 8; ++kk) {
-        const float av[4] = {kt[gid * MASK_KSTRIDE + kk * 8 + tig], kt[(gid + 8) * MASK_KSTRIDE + kk * 8 + tig],
-                             kt[gid * MASK_KSTRIDE + kk * 8 + tig + 4],
-                             kt[(gid + 8) * MASK_KSTRIDE + kk * 8 + tig + 4]};
-        uint32_t ah[4], al[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          ah[e] = __float_as_uint(av[e]) & 0xFFFFE000u;
-          al[e] = __float_as_uint(av[e] - __uint_as_float(ah[e]));
-        }
-        mma_tf32_16x8x8(dhh, ah, bh[kk]);
-        mma_tf32_16x8x8(dhl, ah, bl[kk]);
-        mma_tf32_16x8x8(dlh, al, bh[kk]);
-      }
-      float d[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) d[e] = dhh[e] + (dhl[e] + dlh[e]);
-      const int j = t * MASK_KT + mh * 16 + gid;
-      if (j < NKV) {
-        s_sc[(2 * tig) * nkv_max + j] = d[0] * p.scale;
-        s_sc[(2 * tig + 1) * nkv_max + j] = d[1] * p.scale;
-      }
-      if (j + 8 < NKV) {
-        s_sc[(2 * tig) * nkv_max + j + 8] = d[2] * p.scale;
-        s_sc[(2 * tig + 1) * nkv_max + j + 8] = d[3] * p.scale;
+      for (int m = 0; m < 8; ++m) {
+        r0[m] = ok0 ? __ldg(k0 + 4 * m) : make_float4(0.f, 0.f, 0.f, 0.f);
+        r1[m] = ok1 ? __ldg(k1 + 4 * m) : make_float4(0.f, 0.f, 0.f, 0.f);
       }
     }
-    // the pair is done with the stage: its even warp refills it
-    named_barrier(1 + pair, 64);
-    if (mh == 0 && t + MASK_KSTAGE < ntiles && !*reinterpret_cast<volatile int32_t *>(&s_abort)) {
-      issue_tile(t + MASK_KSTAGE);
-      last_issued = t + MASK_KSTAGE;
+    float dhh[4] = {0.f, 0.f, 0.f, 0.f}, dhl[4] = {0.f, 0.f, 0.f, 0.f}, dlh[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int kk = 0; kk < D / 8; ++kk) {
+      const float4 &x0 = r0[kk >> 1], &x1 = r1[kk >> 1];
+      const float av[4] = {(kk & 1) ? x0.z : x0.x, (kk & 1) ? x1.z : x1.x, (kk & 1) ? x0.w : x0.y,
+                           (kk & 1) ? x1.w : x1.y};
+      uint32_t ah[4], al[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        ah[e] = __float_as_uint(av[e]) & 0xFFFFE000u;
+        al[e] = __float_as_uint(av[e] - __uint_as_float(ah[e]));
+      }
+      const uint4 bf = s_bfrag[kk * 32 + lane];
+      const uint32_t bh[2] = {bf.x, bf.y}, bl[2] = {bf.z, bf.w};
+      mma_tf32_16x8x8(dhh, ah, bh);
+      mma_tf32_16x8x8(dhl, ah, bl);
+      mma_tf32_16x8x8(dlh, al, bh);
+    }
+    float d[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) d[e] = dhh[e] + (dhl[e] + dlh[e]);
+    if (j < NKV) {
+      s_sc[(2 * tig) * nkv_max + j] = d[0] * p.scale;
+      s_sc[(2 * tig + 1) * nkv_max + j] = d[1] * p.scale;
+    }
+    if (j + 8 < NKV) {
+      s_sc[(2 * tig) * nkv_max + j + 8] = d[2] * p.scale;
+      s_sc[(2 * tig + 1) * nkv_max + j + 8] = d[3] * p.scale;
     }
   }
   __syncthreads();                                      // every score written
-  if (*reinterpret_cast<volatile int32_t *>(&s_abort)) {
-    // a wait gave up: each stage's filler lets its last copy land (bounded)
-    // before the block exits
-    if (mh == 0 && lane == 0 && last_issued >= 0) {
-      const long long t0 = clock64();
-      while (!mbar_try_wait(&bar_k[pair], (last_issued / MASK_KSTAGE) & 1) && clock64() - t0 < kWait) {
-      }
-    }
-    return;
-  }
 
   // ---- 3. per-row selection (one warp per q-block) --------------------------
   if (warp < tq_count) {
