@@ -179,9 +179,9 @@ int32_t uf_kv_reset(uf_kv_cache *c, uf_stream_t s);
  *                 the anchor overwrites the anchor.
  *
  * Writes the chunk into its ring slot of k (BLGD -> BGLD) and v (BLGD ->
- * BGDL),
- * zeroes the slot's padding rows, writes the slot's block means into kpool and
- * advances meta (the last thread block to finish commits the new state).
+ * BGDL), zeroes the slot's padding rows, writes the slot's block means into
+ * kpool and advances meta (the last thread block to finish commits the new
+ * state).
  * One kernel launch.  Calls on the same cache must be stream-ordered.
  */
 int32_t uf_kv_append(uf_kv_cache *c, const void *k_new, const void *v_new,
@@ -191,9 +191,10 @@ int32_t uf_kv_append(uf_kv_cache *c, const void *k_new, const void *v_new,
  * Rotary position embedding with positions relative to the window
  * (FlashDecoder, long video decoding: RoPE positions are assigned relative to
  * the current window rather than the absolute frame index; Algorithm 1
- * offsets the positions by the frame index times the tokens per frame).  The pages do not give the rotation's form; it is
- * RoFormer's (Su et al. 2021): channel pairs (x_2i, x_2i+1) rotate by
- * pos * theta_i, theta_i = base^(-2i / D).
+ * offsets the positions by the frame index times the tokens per frame).  The
+ * pages do not give the rotation's form; it is RoFormer's (Su et al. 2021):
+ * channel pairs (x_2i, x_2i+1) rotate by pos * theta_i,
+ * theta_i = base^(-2i / D).
  *
  * Rotary scores q(m) . k(n) depend only on m - n, and so do the pooled block
  * scores, so rotating every token at its position in the stream gives the
@@ -210,8 +211,9 @@ int32_t uf_kv_append(uf_kv_cache *c, const void *k_new, const void *v_new,
  *
  * pos0 >= 0 and pos0 + Lc (resp. L) <= 2^40; base > 1 and finite (10000 is
  * RoFormer's).  Angles are formed and reduced in fp64 (within 1.2e-4 rad below
- * 2^40), sine / cosine in fp32, results rounded to bf16 (nearest even).  UF_EINVAL on bad arguments,
- * otherwise as uf_kv_append.  One kernel launch each.
+ * 2^40), sine / cosine in fp32, results rounded to bf16 (nearest even).
+ * UF_EINVAL on bad arguments, otherwise as uf_kv_append.  One kernel launch
+ * each.
  */
 int32_t uf_kv_append_rope(uf_kv_cache *c, const void *k_new, const void *v_new,
                           int32_t keep_chunks, int32_t flags, int64_t pos0, float base,
