@@ -112,3 +112,24 @@ def test_full_size_1k_local_band():
     assert len(items) >= 3
     oidx, ocnt = oracle_idx_array(cfg, {h: om[h] for h in heads})
     assert_attention_ok(cfg, o, lse, orc.attention(last["q"], items, oidx, ocnt), "1k local")
+
+
+def test_full_size_1k_fixed_local_window_every_item_of_a_head():
+    # the fixed-local-window workload at the full 1K size (band of 9 blocks, the
+    # row stride k = 74): the mask is exactly the band on every row of two heads,
+    # and the attention matches the oracle on every item of one of them
+    cfg = CONFIGS["1k_sr"]
+    k, local = cfg.k_for(), 4
+    gpu, orc = GpuStream(cfg), OracleStream(cfg)
+    last = fill_window(cfg, 7, cfg.W, gpu, orc)
+    idx, cnt, _ = gpu.mask(last["q"], k, want_scores=False, local=local, local_only=True)
+    o, lse = gpu.attention(last["q"], idx, cnt, k)
+    heads = [0, 11]
+    om = orc.mask(last["q"], k, heads=heads, local=local, local_only=True)
+    torch.cuda.synchronize()
+    rows, exact, ties, bad = compare_masks(cfg, idx, cnt, om, k)
+    assert not bad and exact == rows == cfg.B * cfg.nb * len(heads)
+    oidx, ocnt = oracle_idx_array(cfg, om)
+    items = [(b, 11, i) for b in range(cfg.B) for i in range(cfg.nb)]
+    assert_attention_ok(cfg, o, lse, orc.attention(last["q"], items, oidx, ocnt),
+                        f"1k fixed local window, {len(items)} items of head 11")
