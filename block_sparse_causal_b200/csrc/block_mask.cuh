@@ -18,9 +18,9 @@
 //      into A fragments: each warp takes 16-row slices of the window in turn,
 //      each lane loading 4 consecutive channels of its two rows per 16-byte
 //      load.  The MMA's k index runs over the channels in that load order
-//      (any order of the channels gives the same dot product), and the 8
-//      pooled queries' B fragments, split once, follow the same order from
-//      shared memory;
+//      (the dot product does not depend on the order of its channels, up to
+//      rounding), and the 8 pooled queries' B fragments, split once, follow
+//      the same order from shared memory;
 //   3. select: one warp per q-block row forces the diagonal (or the local
 //      band around it), finds the need-th largest of the other scores (need =
 //      k minus the forced blocks) by a bitwise search over order-preserving
